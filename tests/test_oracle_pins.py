@@ -1,0 +1,506 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these compares the oracle with a copy of itself.  Each pin is one of:
+a figure the pages print (tests/golden/), a closed form, an invariant, a
+special case that reduces to a library routine (numpy), or a brute-force
+pure-Python evaluation on tiny inputs.  test_planted_mistakes_are_caught
+plants plausible mistakes in a copy of the oracle's C source and checks that
+these pins catch every one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import mla_workloads as W
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bits(x):
+    return W.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+# ------------------------------------------------------------ tiny workloads
+def tiny_case(rng, B=2, s=1, H=2, d_c=4, d_r=2, d_h=2, bs=2, lens=(3, 2), ints=True, paged=True):
+    """Small-integer MLA inputs (exact in bf16) with a random block table."""
+    lens = np.asarray(lens, np.int32)
+    D = d_c + d_r
+    nblk = [(int(L) + bs - 1) // bs for L in lens]
+    nphys = sum(nblk)
+    perm = rng.permutation(nphys) if paged else np.arange(nphys)
+    maxb = max(nblk)
+    table = np.full((B, maxb), -1, np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :nblk[b]] = perm[off:off + nblk[b]]
+        off += nblk[b]
+    draw = (lambda *sh: rng.integers(-3, 4, size=sh).astype(np.float32)) if ints else \
+        (lambda *sh: rng.standard_normal(sh).astype(np.float32))
+    logical = [draw(int(L), D) for L in lens]
+    cache = np.full((nphys, bs, D), W.BF16_NAN, np.uint16)
+    for b in range(B):
+        for j in range(lens[b]):
+            cache[table[b, j // bs], j % bs] = bits(logical[b][j])
+    T = B * s
+    q_nope = W.bf16_bits_to_f32(bits(draw(T, H, d_h))).astype(np.float64)
+    q_rope = W.bf16_bits_to_f32(bits(draw(T, H, d_r))).astype(np.float64)
+    w_uk = W.bf16_bits_to_f32(bits(draw(H, d_h, d_c))).astype(np.float64)
+    w_uv = W.bf16_bits_to_f32(bits(draw(H, d_h, d_c))).astype(np.float64)
+    t = np.tile(np.arange(s), B)
+    q_pos = (np.repeat(lens, s) - s + 1 + t).astype(np.int32)
+    logical = [W.bf16_bits_to_f32(bits(x)).astype(np.float64) for x in logical]
+    return dict(lens=lens, table=table, cache=cache, logical=logical, q_nope=q_nope,
+                q_rope=q_rope, w_uk=w_uk, w_uv=w_uv, q_pos=q_pos, s=s, B=B, H=H,
+                d_c=d_c, d_r=d_r, d_h=d_h, bs=bs)
+
+
+# -------------------------------------------------- brute force (pure Python)
+def py_rope(x, pos, base=10000.0):
+    d = len(x)
+    y = [0.0] * d
+    for k in range(d // 2):
+        ang = pos * base ** (-2.0 * k / d)
+        y[2 * k] = x[2 * k] * math.cos(ang) - x[2 * k + 1] * math.sin(ang)
+        y[2 * k + 1] = x[2 * k] * math.sin(ang) + x[2 * k + 1] * math.cos(ang)
+    return y
+
+
+def brute_force(c, scale_dims=None):
+    """Textbook MLA decode straight from the pages' formulas, plain Python."""
+    d_c, d_r, d_h, s, H = c["d_c"], c["d_r"], c["d_h"], c["s"], c["H"]
+    scale = 1.0 / math.sqrt(scale_dims if scale_dims else d_h + d_r)
+    outs, lses, probs = {}, {}, {}
+    for b in range(c["B"]):
+        L = int(c["lens"][b])
+        rows = c["logical"][b]
+        for t in range(s):
+            row = b * s + t
+            nvis = L - s + t + 1
+            for i in range(H):
+                if nvis <= 0:
+                    outs[row, i] = [0.0] * d_h
+                    lses[row, i] = -math.inf
+                    continue
+                qc = list(c["q_nope"][row, i])
+                qr = py_rope(list(c["q_rope"][row, i]), int(c["q_pos"][row]))
+                scores = []
+                for j in range(nvis):
+                    cj = list(rows[j][:d_c])
+                    kr = py_rope(list(rows[j][d_c:]), j)
+                    kc = [sum(c["w_uk"][i, k, m] * cj[m] for m in range(d_c)) for k in range(d_h)]
+                    scores.append((sum(qc[k] * kc[k] for k in range(d_h)) +
+                                   sum(qr[m] * kr[m] for m in range(d_r))) * scale)
+                mx = max(scores)
+                e = [math.exp(x - mx) for x in scores]
+                den = sum(e)
+                a = [x / den for x in e]
+                o = [0.0] * d_h
+                for j in range(nvis):
+                    cj = list(rows[j][:d_c])
+                    for k in range(d_h):
+                        o[k] += a[j] * sum(c["w_uv"][i, k, m] * cj[m] for m in range(d_c))
+                outs[row, i] = o
+                lses[row, i] = mx + math.log(den)
+                probs[row, i] = a
+    return outs, lses, probs
+
+
+def run_expanded(o, c, probs_stride=0):
+    return o.decode_expanded(c["cache"], c["table"], c["lens"], c["s"], c["q_nope"], c["q_rope"],
+                             c["w_uk"], c["w_uv"], q_pos=c["q_pos"], block_size=c["bs"],
+                             d_r=c["d_r"], probs_stride=probs_stride)
+
+
+def check_brute(o, c, tol=1e-13):
+    out, lse, _ = run_expanded(o, c)
+    ref, rlse, _ = brute_force(c)
+    n = 0
+    for row in range(c["B"] * c["s"]):
+        for i in range(c["H"]):
+            np.testing.assert_allclose(out[n], ref[row, i], rtol=tol, atol=tol)
+            if math.isinf(rlse[row, i]):
+                assert math.isinf(lse[n])
+            else:
+                assert abs(lse[n] - rlse[row, i]) < tol * max(1, abs(rlse[row, i]))
+            n += 1
+
+
+# ------------------------------------------------------------------- pins
+def test_golden_cache_accounting():
+    """The row layout (576 values, 1152 bytes in bf16) reproduces every
+    cache-size figure the pages print."""
+    g = json.load(open(os.path.join(GOLD, "cache_accounting.json")))
+    row = W.D_C + W.D_R
+    assert row == g["mla_elements_per_token_per_layer"]["value"]
+    assert row * g["v2_layers"]["value"] == g["v2_elements_per_token"]["value"]
+    assert row / (2 * 128) == g["gqa_equivalent_groups"]["value"]
+    assert round(100 * row / (2 * 128 * 128), 2) == g["mha_ratio_percent"]["value"]
+    b67 = 95 * 2 * 8 * 128 * 2
+    assert b67 == g["dense67b_bytes_per_token"]["value"]
+    b6 = 60 * row * 6 // 8
+    assert b6 == g["v2_bytes_per_token_6bit"]["value"]
+    assert round(100 * (1 - b6 / b67), 2) == g["reduction_percent_6bit"]["value"]
+    b16 = 60 * row * 2
+    assert b16 == g["v2_bytes_per_token_16bit"]["value"]
+    assert round(100 * (1 - b16 / b67), 2) == g["reduction_percent_16bit"]["value"]
+    assert round(27 * row / 1000, 1) == g["table9_small_mla_elements_k"]["value"]
+    assert round(2 * 16 * 128 * 27 / 1000, 1) == g["table9_small_mha_elements_k"]["value"]
+    assert round(60 * row / 1000, 1) == g["table9_large_mla_elements_k"]["value"]
+    assert W.D_H + W.D_R == g["score_scale_dims"]["value"]
+    lite = g["v2lite_shapes"]["value"]
+    c2 = W.CONFIGS["v2lite"]
+    assert (c2.H, c2.d_h, c2.d_c, c2.d_r, c2.d_model) == (
+        lite["heads"], lite["head_dim"], lite["d_c"], lite["d_r"], lite["hidden"])
+
+
+def test_rope_identity_at_zero(oracle_mod):
+    x = np.random.default_rng(0).standard_normal(64)
+    assert np.array_equal(oracle_mod.rope(x, 0.0), x)
+
+
+def test_rope_closed_forms(oracle_mod):
+    # pair 0 turns by exactly pos radians
+    e0 = np.zeros(64); e0[0] = 1.0
+    y = oracle_mod.rope(e0, math.pi / 2)
+    np.testing.assert_allclose(y[:2], [0.0, 1.0], atol=1e-15)
+    # pair 16 of 32 has theta = 10000^(-1/2) = 1/100, so position 100 turns it by 1 rad
+    e32 = np.zeros(64); e32[32] = 1.0
+    y = oracle_mod.rope(e32, 100.0)
+    np.testing.assert_allclose(y[32:34], [math.cos(1.0), math.sin(1.0)], atol=1e-14)
+    assert np.count_nonzero(np.abs(np.delete(y, [32, 33])) > 0) == 0
+    # the last pair turns slowest: theta_31 = 10000^(-62/64) < theta_30
+    e62 = np.zeros(64); e62[62] = 1.0
+    e60 = np.zeros(64); e60[60] = 1.0
+    a62 = math.atan2(oracle_mod.rope(e62, 1.0)[63], 1.0)
+    a60 = math.atan2(oracle_mod.rope(e60, 1.0)[61], 1.0)
+    assert 0 < a62 < a60 < 1e-3
+
+
+def test_rope_norm_and_relative_position(oracle_mod):
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m in (0, 5, 1000, 131071):
+        np.testing.assert_allclose(np.linalg.norm(oracle_mod.rope(q, m)), np.linalg.norm(q), rtol=1e-14)
+    for m, n, dlt in ((3, 10, 7), (100, 4000, 123), (0, 9, 50000)):
+        a = oracle_mod.rope(q, m) @ oracle_mod.rope(k, n)
+        b = oracle_mod.rope(q, m + dlt) @ oracle_mod.rope(k, n + dlt)
+        assert abs(a - b) < 1e-10 * (1 + abs(a))
+    # composition: R_m R_n = R_{m+n}
+    np.testing.assert_allclose(oracle_mod.rope(oracle_mod.rope(q, 17), 25), oracle_mod.rope(q, 42),
+                               atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,s,lens", [(0, 1, (3, 2)), (1, 2, (3, 4)), (2, 1, (1, 5)), (3, 2, (2, 1))])
+def test_brute_force_tiny(oracle_mod, seed, s, lens):
+    c = tiny_case(np.random.default_rng(seed), B=2, s=s, lens=lens)
+    check_brute(oracle_mod, c)
+
+
+def test_brute_force_tiny_gaussian(oracle_mod):
+    c = tiny_case(np.random.default_rng(11), B=2, s=2, H=3, d_c=6, d_r=4, d_h=3, bs=3,
+                  lens=(7, 4), ints=False)
+    check_brute(oracle_mod, c)
+
+
+def test_scale_guard(oracle_mod):
+    """The scale is 1/sqrt(d_h + d_r) (192 for the real shapes), not
+    1/sqrt(d_c + d_r) (576): the two give clearly different outputs."""
+    c = tiny_case(np.random.default_rng(5), B=1, s=1, H=2, d_c=16, d_r=4, d_h=8, bs=4,
+                  lens=(6,), ints=False)
+    c["w_uk"] = c["w_uk"] / 4.0  # keep the logits O(1), where the scale matters most
+    out, _, _ = run_expanded(oracle_mod, c)
+    good, _, _ = brute_force(c)
+    wrong, _, _ = brute_force(c, scale_dims=c["d_c"] + c["d_r"])
+    for i in range(2):
+        np.testing.assert_allclose(out[i], good[0, i], atol=1e-13)
+        assert np.max(np.abs(np.asarray(wrong[0, i]) - out[i])) > 2e-2
+
+
+def test_softmax_rows_sum_to_one(oracle_mod):
+    c = tiny_case(np.random.default_rng(2), B=2, s=2, lens=(6, 3), ints=False)
+    _, _, probs = run_expanded(oracle_mod, c, probs_stride=8)
+    n = 0
+    for b in range(2):
+        for t in range(2):
+            nvis = c["lens"][b] - 2 + t + 1
+            for i in range(c["H"]):
+                p = probs[n]
+                assert np.all(p >= 0)
+                assert abs(p.sum() - 1.0) < 1e-14
+                assert np.all(p[nvis:] == 0)
+                n += 1
+
+
+def _absorbed_vs_expanded(o, cfg_inputs, rows=None, heads=None):
+    d = cfg_inputs
+    cfg = d["cfg"]
+    q_abs = o.absorb_q(o.bf16_to_f64(d["q_nope"]), o.bf16_to_f64(d["q_rope"]),
+                       o.bf16_to_f64(d["w_uk"]), q_pos=d["q_pos"])
+    lat, lse_a = o.decode_latent(d["cache"], d["block_table"], d["seq_lens"], cfg.s, q_abs,
+                                 rows=rows, heads=heads)
+    exp, lse_e, _ = o.decode_expanded(d["cache"], d["block_table"], d["seq_lens"], cfg.s,
+                                      o.bf16_to_f64(d["q_nope"]), o.bf16_to_f64(d["q_rope"]),
+                                      o.bf16_to_f64(d["w_uk"]), o.bf16_to_f64(d["w_uv"]),
+                                      q_pos=d["q_pos"], rows=rows, heads=heads)
+    pr = rows if rows is not None else np.repeat(np.arange(cfg.T), cfg.H)
+    ph = heads if heads is not None else np.tile(np.arange(cfg.H), cfg.T)
+    w_uv = o.bf16_to_f64(d["w_uv"])
+    o_abs = np.einsum("nkm,nm->nk", w_uv[ph], lat)
+    return exp, o_abs, lse_e, lse_a
+
+
+def test_absorbed_equals_expanded_tiny_config(oracle_mod):
+    """The absorption identities (DeepSeek-V2 paper review, section 2) hold in
+    fp64 on the tiny decode workload (H=16, L=256)."""
+    d = W.make_decode_inputs(W.CONFIGS["tiny"])
+    exp, o_abs, lse_e, lse_a = _absorbed_vs_expanded(oracle_mod, d)
+    assert np.max(np.abs(exp - o_abs)) <= 1e-12 * np.max(np.abs(exp))
+    np.testing.assert_allclose(lse_e, lse_a, rtol=1e-12)
+
+
+def test_absorbed_equals_expanded_paged_ragged(oracle_mod):
+    cfg = W.MLAConfig("t", B=3, s=2, H=4, L=0, paged=True, seed=77, d_model=64,
+                      seq_lens=(130, 2, 64))
+    d = W.make_decode_inputs(cfg)
+    exp, o_abs, lse_e, lse_a = _absorbed_vs_expanded(oracle_mod, d)
+    assert np.max(np.abs(exp - o_abs)) <= 1e-12 * np.max(np.abs(exp))
+    np.testing.assert_allclose(lse_e, lse_a, rtol=1e-12)
+
+
+def test_absorb_q_matches_library_matmul(oracle_mod):
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, 3, 128)); qr = rng.standard_normal((5, 3, 64))
+    U = rng.standard_normal((3, 128, 512))
+    out = oracle_mod.absorb_q(q, qr, U)
+    np.testing.assert_allclose(out[..., :512], np.einsum("hkm,thk->thm", U, q), rtol=1e-12, atol=1e-12)
+    assert np.array_equal(out[..., 512:], qr)
+    # the score identity: ((U^K)^T q)^T c == q^T (U^K c)
+    c = rng.standard_normal(512)
+    for t in range(5):
+        for h in range(3):
+            assert abs(out[t, h, :512] @ c - q[t, h] @ (U[h] @ c)) < 1e-9
+    # with positions, the RoPE part is rotated
+    pos = np.array([0, 1, 2, 3, 4], np.int32)
+    out2 = oracle_mod.absorb_q(q, qr, U, q_pos=pos)
+    assert np.array_equal(out2[0, :, 512:], qr[0])
+    assert abs(np.linalg.norm(out2[3, 1, 512:]) - np.linalg.norm(qr[3, 1])) < 1e-12
+
+
+def test_single_token_closed_form(oracle_mod):
+    """With one visible key the softmax weight is 1: o = U^V c_0 and the
+    latent output is c_0 exactly."""
+    cfg = W.MLAConfig("t", B=2, s=1, H=4, L=1, paged=True, seed=5, d_model=64)
+    d = W.make_decode_inputs(cfg)
+    q_abs = oracle_mod.absorb_q(oracle_mod.bf16_to_f64(d["q_nope"]), oracle_mod.bf16_to_f64(d["q_rope"]),
+                                oracle_mod.bf16_to_f64(d["w_uk"]), q_pos=d["q_pos"])
+    lat, _ = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 1, q_abs)
+    c0 = oracle_mod.bf16_to_f64(d["c_kv"])  # token 0 of each sequence, sequence-major
+    for b in range(2):
+        for h in range(4):
+            assert np.array_equal(lat[b * 4 + h], c0[b])
+    exp, _, _ = oracle_mod.decode_expanded(d["cache"], d["block_table"], d["seq_lens"], 1,
+                                           oracle_mod.bf16_to_f64(d["q_nope"]),
+                                           oracle_mod.bf16_to_f64(d["q_rope"]),
+                                           oracle_mod.bf16_to_f64(d["w_uk"]),
+                                           oracle_mod.bf16_to_f64(d["w_uv"]), q_pos=d["q_pos"])
+    Uv = oracle_mod.bf16_to_f64(d["w_uv"])
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_allclose(exp[b * 4 + h], Uv[h] @ c0[b], rtol=1e-12, atol=1e-14)
+
+
+def test_uniform_attention_closed_form(oracle_mod):
+    """q^C = 0 and q^R = 0 make every logit 0: the latent output is the mean
+    of the visible latents."""
+    cfg = W.MLAConfig("t", B=2, s=2, H=2, L=0, paged=True, seed=9, d_model=64, seq_lens=(70, 5))
+    d = W.make_decode_inputs(cfg)
+    q_abs = np.zeros((cfg.T, cfg.H, 576))
+    lat, lse = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 2, q_abs)
+    c = oracle_mod.bf16_to_f64(d["c_kv"])
+    starts = [0, 70]
+    n = 0
+    for b, L in enumerate((70, 5)):
+        for t in range(2):
+            nvis = L - 2 + t + 1
+            for h in range(2):
+                np.testing.assert_allclose(lat[n], c[starts[b]:starts[b] + nvis].mean(0), atol=1e-14)
+                assert abs(lse[n] - math.log(nvis)) < 1e-14
+                n += 1
+
+
+def test_one_hot_limit(oracle_mod):
+    """A query aligned with one key and scaled up puts all weight on it."""
+    cfg = W.MLAConfig("t", B=1, s=1, H=1, L=40, paged=True, seed=13, d_model=64)
+    d = W.make_decode_inputs(cfg)
+    c = oracle_mod.bf16_to_f64(d["c_kv"])
+    kr = oracle_mod.bf16_to_f64(d["k_rope"])
+    k = 17
+    key = np.concatenate([c[k], oracle_mod.rope(kr[k], k)])
+    q_abs = (60.0 * key / np.linalg.norm(key))[None, None, :] * math.sqrt(192)
+    lat, _ = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 1, q_abs)
+    np.testing.assert_allclose(lat[0], c[k], atol=1e-9)
+
+
+def test_heads_are_independent(oracle_mod):
+    """Permuting the heads of q, U^K and U^V permutes the outputs (each head
+    has its own a_ij; DeepSeek-V2 paper review, section 2)."""
+    cfg = W.MLAConfig("t", B=2, s=1, H=5, L=0, paged=True, seed=21, d_model=64, seq_lens=(33, 8))
+    d = W.make_decode_inputs(cfg)
+    f = oracle_mod.bf16_to_f64
+    perm = np.array([3, 0, 4, 1, 2])
+    a, _, _ = oracle_mod.decode_expanded(d["cache"], d["block_table"], d["seq_lens"], 1, f(d["q_nope"]),
+                                         f(d["q_rope"]), f(d["w_uk"]), f(d["w_uv"]), q_pos=d["q_pos"])
+    b, _, _ = oracle_mod.decode_expanded(d["cache"], d["block_table"], d["seq_lens"], 1,
+                                         f(d["q_nope"])[:, perm], f(d["q_rope"])[:, perm],
+                                         f(d["w_uk"])[perm], f(d["w_uv"])[perm], q_pos=d["q_pos"])
+    assert np.array_equal(a.reshape(2, 5, -1)[:, perm], b.reshape(2, 5, -1))
+    # and heads really differ
+    assert np.max(np.abs(a.reshape(2, 5, -1)[:, 0] - a.reshape(2, 5, -1)[:, 1])) > 1e-3
+
+
+def test_block_permutation_invariance(oracle_mod):
+    """The result depends only on the logical token order, not on where the
+    blocks sit physically."""
+    base = W.MLAConfig("t", B=3, s=1, H=2, L=0, paged=True, seed=31, d_model=64, seq_lens=(200, 65, 1))
+    d1 = W.make_decode_inputs(base)
+    d2 = W.make_decode_inputs(base.with_(paged=False))
+    assert not np.array_equal(d1["block_table"], d2["block_table"])
+    q_abs = oracle_mod.bf16_to_f64(W.make_q_abs(base))
+    l1, s1 = oracle_mod.decode_latent(d1["cache"], d1["block_table"], d1["seq_lens"], 1, q_abs)
+    l2, s2 = oracle_mod.decode_latent(d2["cache"], d2["block_table"], d2["seq_lens"], 1, q_abs)
+    assert np.array_equal(l1, l2) and np.array_equal(s1, s2)
+
+
+def test_nan_tail_slots_never_read(oracle_mod):
+    cfg = W.MLAConfig("t", B=2, s=2, H=2, L=0, paged=True, seed=41, d_model=64, seq_lens=(67, 3))
+    d = W.make_decode_inputs(cfg)
+    assert np.isnan(W.bf16_bits_to_f32(d["cache"])).any()
+    lat, lse = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 2,
+                                        oracle_mod.bf16_to_f64(W.make_q_abs(cfg)))
+    assert np.isfinite(lat).all() and np.isfinite(lse).all()
+
+
+def test_causal_mask_two_queries(oracle_mod):
+    """With s=2, query 0 of a length-L sequence sees exactly what a single
+    query sees in the same sequence cut to length L-1."""
+    cfg = W.MLAConfig("t", B=1, s=2, H=3, L=50, paged=True, seed=51, d_model=64)
+    d = W.make_decode_inputs(cfg)
+    q_abs = oracle_mod.bf16_to_f64(W.make_q_abs(cfg))
+    lat2, lse2 = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 2, q_abs)
+    lat1, lse1 = oracle_mod.decode_latent(d["cache"], d["block_table"], np.array([49], np.int32), 1,
+                                          q_abs[0:1])
+    assert np.array_equal(lat2[:3], lat1) and np.array_equal(lse2[:3], lse1)
+
+
+def test_empty_row(oracle_mod):
+    cfg = W.MLAConfig("t", B=2, s=1, H=2, L=0, paged=True, seed=61, d_model=64, seq_lens=(0, 4))
+    d = W.make_decode_inputs(cfg)
+    lat, lse = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], 1,
+                                        oracle_mod.bf16_to_f64(W.make_q_abs(cfg)))
+    assert np.all(lat[:2] == 0) and np.all(np.isneginf(lse[:2])) and np.isfinite(lse[2:]).all()
+
+
+def test_bad_block_table_is_rejected(oracle_mod):
+    cfg = W.MLAConfig("t", B=1, s=1, H=1, L=10, paged=True, seed=71, d_model=64)
+    d = W.make_decode_inputs(cfg)
+    bt = d["block_table"].copy(); bt[0, 0] = 5
+    with pytest.raises(ValueError):
+        oracle_mod.decode_latent(d["cache"], bt, d["seq_lens"], 1, np.zeros((1, 1, 576)))
+
+
+def test_kv_project_matches_library_and_identity(oracle_mod):
+    rng = np.random.default_rng(8)
+    T, d = 6, 96
+    h = bits(rng.standard_normal((T, d)))
+    wd = bits(rng.standard_normal((512, d)) / 10)
+    wr = bits(rng.standard_normal((64, d)) / 10)
+    pos = np.array([0, 1, 7, 100, 4095, 131071], np.int32)
+    c, kr = oracle_mod.kv_project(h, wd, wr, pos)
+    hf, wdf, wrf = (oracle_mod.bf16_to_f64(x) for x in (h, wd, wr))
+    np.testing.assert_allclose(c, hf @ wdf.T, rtol=1e-12, atol=1e-12)
+    raw = hf @ wrf.T
+    np.testing.assert_allclose(kr[0], raw[0], atol=1e-12)               # RoPE at 0 is the identity
+    np.testing.assert_allclose(np.linalg.norm(kr, axis=1), np.linalg.norm(raw, axis=1), rtol=1e-12)
+    # identity projection reproduces the input exactly
+    hh = bits(rng.standard_normal((3, 576)))
+    eye_c = bits(np.eye(576)[:512]); eye_r = bits(np.eye(576)[512:])
+    c2, kr2 = oracle_mod.kv_project(hh, eye_c, eye_r, np.zeros(3, np.int32))
+    assert np.array_equal(c2, oracle_mod.bf16_to_f64(hh)[:, :512])
+    assert np.array_equal(kr2, oracle_mod.bf16_to_f64(hh)[:, 512:])
+
+
+def test_up_v_and_out_proj_match_library(oracle_mod):
+    rng = np.random.default_rng(9)
+    lat = rng.standard_normal((4, 3, 512)); U = rng.standard_normal((3, 128, 512))
+    o = oracle_mod.up_v(lat, U)
+    np.testing.assert_allclose(o, np.einsum("hkm,thm->thk", U, lat), rtol=1e-12, atol=1e-11)
+    Wo = rng.standard_normal((40, 3 * 128))
+    u = oracle_mod.out_proj(o, Wo)
+    np.testing.assert_allclose(u, o.reshape(4, -1) @ Wo.T, rtol=1e-12, atol=1e-10)
+
+
+def test_generator_bf16_rounding_matches_torch():
+    import torch
+    x = np.random.default_rng(0).standard_normal(100000).astype(np.float32)
+    mine = W.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(mine, ref)
+
+
+def test_generator_is_deterministic_and_paged():
+    cfg = W.MLAConfig("t", B=3, s=2, H=2, L=(10, 200), paged=True, seed=99, d_model=64)
+    a, b = W.make_decode_inputs(cfg), W.make_decode_inputs(cfg)
+    for k in ("cache", "block_table", "q_nope", "w_uk", "seq_lens"):
+        assert np.array_equal(a[k], b[k])
+    bt = a["block_table"]
+    used = bt[bt >= 0]
+    assert sorted(used.tolist()) == list(range(a["num_blocks"]))
+    for bb in range(3):
+        n = (a["seq_lens"][bb] + 63) // 64
+        assert np.all(bt[bb, :n] >= 0) and np.all(bt[bb, n:] == -1)
+
+
+# ------------------------------------------------------ planted mistakes
+MUTATIONS = {
+    "drop_rope_term": ("for (int m = 0; m < d_r; ++m) dot += qr[m] * kr[m];", ""),
+    "rope_sign": ("y[2 * k] = x0 * c - x1 * s;", "y[2 * k] = x0 * c + x1 * s;"),
+    "transposed_uk": ("acc += Uk[(size_t)k * d_c + m] * c[m];", "acc += Uk[(size_t)(m % d_h) * d_c + k] * c[m];"),
+    "latent_scale": ("const double scale = 1.0 / sqrt((double)(d_h + d_r));\n    int bad = 0;\n    (void)B;\n#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)\n    for (int p = 0; p < n_pairs; ++p) {\n        const int row = pair_row[p], i = pair_head[p];\n        const int b = row / s, t = row % s;\n        const int L",
+                     "const double scale = 1.0 / sqrt((double)(d_c + d_r));\n    int bad = 0;\n    (void)B;\n#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)\n    for (int p = 0; p < n_pairs; ++p) {\n        const int row = pair_row[p], i = pair_head[p];\n        const int b = row / s, t = row % s;\n        const int L"),
+    "mask_off_by_one": ("const int n_vis = L - s + t + 1;", "const int n_vis = L - s + t;"),
+    "key_position": ("mla_oracle_rope(kr_raw, d_r, (double)j, rope_base, kr);\n            for (int k = 0; k < d_h; ++k) {",
+                     "mla_oracle_rope(kr_raw, d_r, (double)(j + 1), rope_base, kr);\n            for (int k = 0; k < d_h; ++k) {"),
+    "no_max_subtract_den": ("lse[p] = mx + log(den);\n        /* o = sum", "lse[p] = log(den);\n        /* o = sum"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistakes_are_caught(oracle_mod, tmp_path, name):
+    """Plant one plausible mistake in a copy of the oracle source and check
+    that the brute-force pin rejects the mutant."""
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle_mod.__file__), "mla_oracle.c")).read()
+    old, new = MUTATIONS[name]
+    assert src.count(old) >= 1, name
+    mutant = tmp_path / "m.c"
+    mutant.write_text(src.replace(old, new, 1))
+    so = tmp_path / "m.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(mutant), "-lm"],
+                   check=True)
+    saved = oracle_mod._LIB
+    oracle_mod._LIB = oracle_mod.load(str(so))
+    try:
+        caught = False
+        for seed, s, lens in ((0, 1, (3, 2)), (1, 2, (3, 4)), (4, 2, (5, 6))):
+            c = tiny_case(np.random.default_rng(seed), B=2, s=s, lens=lens, ints=False)
+            try:
+                check_brute(oracle_mod, c, tol=1e-9)
+            except AssertionError:
+                caught = True
+                break
+        assert caught, f"mutation {name} was not caught"
+    finally:
+        oracle_mod._LIB = saved
