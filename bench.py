@@ -1,0 +1,369 @@
+"""Benchmark: one MLA decode step of the whole hot path on synthetic inputs.
+
+A step = append the newest latent of every sequence from its hidden state
+(mla_append_cache) -> absorb U^K into the queries (mla_absorb_q) -> attention
+over the paged latent cache with split-KV combine (mla_decode) -> U^V
+up-projection (mla_up_v).  Default workload: the DeepSeek-V2-shaped decode
+batch (B=128 sequences, 1 query token each, H=128 heads, L=4096, d_c=512,
+d_r=64, 64-token paged cache with a random block table), bf16 storage with
+fp32 accumulation.  Every rank (one per GPU) runs its own copy of the batch:
+sequences are independent, so there is no collective (weak scaling).
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the host cores instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), tc=float(d["bf16_tflops"]),
+                    tc_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, source="fallback")
+
+
+def algorithmic(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
+    """Bytes and FLOPs one mla_decode call must move and compute.
+    Bytes: visible cache rows (1152 B/token, read once for all heads), the
+    absorbed queries, the latent outputs and lse, the block table and lengths.
+    FLOPs: 2*(576 + 512) per (head, query, visible key)."""
+    s = cfg.s
+    vis = sum(max(0, int(L) - s + t + 1) for L in seq_lens for t in range(s))
+    # a sequence's cache rows are read once even with several queries
+    rows_read = int(np.sum(seq_lens))
+    D = cfg.d_c + cfg.d_r
+    byts = rows_read * D * 2 + cfg.T * cfg.H * D * 2 + cfg.T * cfg.H * (cfg.d_c * 2 + 4) \
+        + cfg.B * max_blocks * 4 + cfg.B * 4
+    flops = 2 * (D + cfg.d_c) * cfg.H * vis
+    return byts, flops, rows_read
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# -------------------------------------------------------------- our arm
+class Step:
+    """Device-resident workload plus the four library calls of one step."""
+
+    def __init__(self, cfg: W.MLAConfig, dev: int, flags: int):
+        import torch
+        import head_latent_attention_10_b200 as M
+        self.M, self.torch, self.cfg, self.flags = M, torch, cfg, flags
+        M.load_library()
+        torch.cuda.set_device(dev)
+        d = W.make_decode_inputs(cfg, with_cache_pages=False)
+        self.seq_lens_np = d["seq_lens"]
+        self.max_blocks = d["block_table"].shape[1]
+        cu = lambda a, dt=None: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+        self.dims = M.dims(cfg.H)
+        self.block_table = cu(d["block_table"])
+        self.seq_lens = cu(d["seq_lens"])
+        D = cfg.d_c + cfg.d_r
+        self.cache = torch.full((d["num_blocks"], cfg.block_size, D), float("nan"),
+                                dtype=torch.bfloat16, device="cuda")
+        N, chunk = d["tok_seq"].size, 1 << 20
+        for a in range(0, N, chunk):
+            b = min(N, a + chunk)
+            M.mla_append_latent(self.dims, bf(d["c_kv"][a:b]), bf(d["k_rope"][a:b]), cu(d["tok_seq"][a:b]),
+                                cu(d["tok_pos"][a:b]), self.block_table, self.cache)
+        del d["c_kv"], d["k_rope"]
+        self.w_uk, self.w_uv = bf(d["w_uk"]), bf(d["w_uv"])
+        a = W.make_append_inputs(cfg, cfg.T)
+        self.w_dkv, self.w_kr = bf(a["w_dkv"]), bf(a["w_kr"])
+        # per-step inputs: new hidden states, their slots (the newest s
+        # positions of each sequence), and the queries
+        T = cfg.T
+        t = np.tile(np.arange(cfg.s), cfg.B)
+        app_pos = (np.repeat(d["seq_lens"], cfg.s) - cfg.s + t).astype(np.int32)
+        self.host = dict(h=a["h"], q_nope=d["q_nope"], q_rope=d["q_rope"], q_pos=d["q_pos"],
+                         app_seq=np.repeat(np.arange(cfg.B, dtype=np.int32), cfg.s), app_pos=app_pos)
+        self.dev = {k: (bf(v) if v.dtype == np.uint16 else cu(v)) for k, v in self.host.items()}
+        self.q_abs = torch.empty(T, cfg.H, D, dtype=torch.bfloat16, device="cuda")
+        self.lat = torch.empty(T, cfg.H, cfg.d_c, dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty(T, cfg.H, dtype=torch.float32, device="cuda")
+        self.out = torch.empty(T, cfg.H, cfg.d_h, dtype=torch.bfloat16, device="cuda")
+        self.ws = torch.empty(M.mla_decode_workspace_size(self.dims, cfg.B, cfg.s, self.max_blocks * 64),
+                              dtype=torch.uint8, device="cuda")
+        self.stream = torch.cuda.current_stream()
+        torch.cuda.synchronize()
+
+    def run(self, inp=None, dec_events=None):
+        M, x = self.M, (inp if inp is not None else self.dev)
+        M.mla_append_cache(self.dims, x["h"], self.w_dkv, self.w_kr, x["app_seq"], x["app_pos"],
+                           self.block_table, self.cache)
+        M.mla_absorb_q(self.dims, x["q_nope"], x["q_rope"], x["q_pos"], self.w_uk, self.q_abs)
+        if dec_events is not None:
+            dec_events[0].record(self.stream)
+        M.mla_decode(self.dims, self.q_abs, self.cache, self.block_table, self.seq_lens, self.cfg.s,
+                     self.lat, self.lse, self.ws, flags=self.flags)
+        if dec_events is not None:
+            dec_events[1].record(self.stream)
+        M.mla_up_v(self.dims, self.lat, self.w_uv, self.out)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    cfg = W.CONFIGS[args.config]
+    import head_latent_attention_10_b200 as M
+    st = Step(cfg, local, flags=(M.MLA_FORCE_SIMPLE if args.simple else 0))
+    E = torch.cuda.Event
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # --- device-resident timing (inputs already in HBM)
+    for _ in range(args.warmup):
+        st.run()
+    barrier()
+    dec = [(E(enable_timing=True), E(enable_timing=True)) for _ in range(args.steps)]
+    clock = ClockSampler(local)
+    clock.start()
+    time.sleep(0.3)
+    barrier()
+    l0 = M.mla_kernel_launches()
+    t0, t1 = E(enable_timing=True), E(enable_timing=True)
+    t0.record()
+    for k in range(args.steps):
+        st.run(dec_events=dec[k])
+    t1.record()
+    barrier()
+    launches = M.mla_kernel_launches() - l0
+    clocks = clock.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec]))
+    if world > 1:
+        v = torch.tensor([ms, dec_ms], device="cuda")
+        dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(v[0]), float(v[1])
+
+    # --- end to end: pinned host inputs copied in and the output copied out
+    pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else v)
+           .pin_memory() for k, v in st.host.items()}
+    out_host = torch.empty(st.out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = out_host.numel() * out_host.element_size()
+    stage = {k: torch.empty_like(v) for k, v in st.dev.items()}
+
+    def e2e_step():
+        for k, v in pin.items():
+            dst = stage[k]
+            dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(v, non_blocking=True)
+        st.run(stage)
+        out_host.copy_(st.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0, e1 = E(enable_timing=True), E(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        v = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        e2e_ms = float(v[0])
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    tok = cfg.T * world
+    byts, flops, rows = algorithmic(cfg, st.seq_lens_np, st.max_blocks)
+    pk = peaks()
+    hbm_t, tc_t = byts / (pk["hbm"] * 1e9), flops / (pk["tc"] * 1e12)
+    bound = "hbm" if hbm_t >= tc_t else "tensor"
+    dec_s = dec_ms / 1e3
+    if bound == "hbm":
+        achieved, peak, unit = byts / dec_s / 1e9, pk["hbm"], "GB/s"
+    else:
+        achieved, peak, unit = flops / dec_s / 1e12, pk["tc"], "TFLOP/s"
+    line = {
+        "metric": "MLA decode tokens/s, latent-cache GB/s & TFLOP/s (H=128,B=128,L=4K) vs roofline",
+        "value": tok / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, N(0,1) latents/queries, "
+        "N(0,1/512) up-projections, random block table)",
+        "config": {"workload": cfg.describe, "B": cfg.B, "s": cfg.s, "H": cfg.H,
+                   "L": cfg.L if not isinstance(cfg.L, tuple) else list(cfg.L),
+                   "d_c": cfg.d_c, "d_r": cfg.d_r, "d_h": cfg.d_h, "block_size": cfg.block_size,
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                   "l2": "inputs larger than L2 (%.0f MB of cache read per step)" % (rows * 1152 / 1e6),
+                   "decode_path": "simple" if args.simple else "default"},
+        "decode": {"ms": dec_ms, "cache_gbs": rows * 1152 / dec_s / 1e9, "bytes": byts,
+                   "gbs": byts / dec_s / 1e9, "flops": flops, "tflops": flops / dec_s / 1e12,
+                   "roofline_us": max(hbm_t, tc_t) * 1e6,
+                   "roofline_frac": max(hbm_t, tc_t) / dec_s},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": pk["source"] + (" burst" if bound == "tensor" else "")},
+        "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------- CPU oracle (baseline)
+def cpu_baseline(cfg: W.MLAConfig, budget_s: float = 10.0):
+    """The fp64 expanded-form oracle, as it stands, on a bounded sample of the
+    workload: (row 0, heads 0..k-1) at full context, k grown until the run
+    takes about `budget_s`; tokens/s = 1 / (time per query row of H heads)."""
+    import oracle
+    d = W.make_decode_inputs(cfg.with_(B=1), with_cache_pages=True)
+    f = oracle.bf16_to_f64
+    args = (d["cache"], d["block_table"], d["seq_lens"], cfg.s, f(d["q_nope"]), f(d["q_rope"]),
+            f(d["w_uk"]), f(d["w_uv"]))
+    k = max(1, min(cfg.H, oracle.num_threads()))
+    while True:
+        t = time.perf_counter()
+        oracle.decode_expanded(*args, q_pos=d["q_pos"], rows=np.zeros(k, np.int32),
+                               heads=np.arange(k, dtype=np.int32))
+        el = time.perf_counter() - t
+        if el >= budget_s / 3 or k >= cfg.H:
+            break
+        k = min(cfg.H, k * 2)
+    per_row = el * cfg.H / k
+    return {"value": 1.0 / per_row, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"expanded-form fp64 oracle on {k} of {cfg.H} heads of one query row at full "
+                      f"context L={int(d['seq_lens'][0])}: {el:.2f} s, scaled to one row of all heads"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = W.CONFIGS[args.config]
+    import oracle
+    oracle._lib()
+    d = W.make_decode_inputs(cfg.with_(B=1), with_cache_pages=True)
+    f = oracle.bf16_to_f64
+    a = (d["cache"], d["block_table"], d["seq_lens"], cfg.s, f(d["q_nope"]), f(d["q_rope"]),
+         f(d["w_uk"]), f(d["w_uv"]))
+    k = max(1, min(cfg.H, oracle.num_threads()))
+    step = lambda: oracle.decode_expanded(*a, q_pos=d["q_pos"], rows=np.zeros(k, np.int32),
+                                          heads=np.arange(k, dtype=np.int32))
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = (time.perf_counter() - t) / args.steps
+    v = k / cfg.H / el
+    sample = (f"each step: expanded-form fp64 oracle on {k} of {cfg.H} heads of one query row at full "
+              f"context L={int(d['seq_lens'][0])}; tokens/s = rows of all heads per second")
+    print(json.dumps({
+        "impl": "reference", "metric": "MLA decode tokens/s, latent-cache GB/s & TFLOP/s (H=128,B=128,L=4K) vs roofline",
+        "value": v, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": cfg.describe, "B": cfg.B, "s": cfg.s, "H": cfg.H},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="v2", choices=sorted(W.CONFIGS))
+    ap.add_argument("--simple", action="store_true", help="force the CUDA-core decode kernel")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

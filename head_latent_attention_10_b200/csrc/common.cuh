@@ -1,0 +1,53 @@
+// common.cuh -- shared device helpers of the MLA decode library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// Kernels launched by the library in this process (see mla_kernel_launches).
+extern unsigned long long g_launches;
+inline void count_launch(unsigned n = 1) { __atomic_fetch_add(&g_launches, n, __ATOMIC_RELAXED); }
+
+typedef __nv_bfloat16 bf16;
+
+constexpr int kDc = 512;      // latent width d_c
+constexpr int kDr = 64;       // RoPE width d_r
+constexpr int kDh = 128;      // per-head content width d_h
+constexpr int kRow = kDc + kDr;  // 576 values per cached token
+constexpr int kBlock = 64;    // tokens per cache block
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits)
+{
+    if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ float bf2f(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ bf16 f2bf(float v) { return __float2bfloat16_rn(v); }
+
+// RoPE of one pair (x0, x1) = (x[2k], x[2k+1]) at position pos: turn by
+// pos * base^(-2k/d_r).  The angle is formed in double precision: at
+// positions up to 2^17 an fp32 angle would be off by ~1e-2 rad.
+__device__ __forceinline__ void rope_pair(float x0, float x1, int pos, int k, int d_r,
+                                          double base, float *y0, float *y1)
+{
+    const double theta = pow(base, -2.0 * (double)k / (double)d_r);
+    const double ang = (double)pos * theta;
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    *y0 = (float)((double)x0 * cs - (double)x1 * sn);
+    *y1 = (float)((double)x0 * sn + (double)x1 * cs);
+}
+
+// 16-byte vector of 8 bf16
+struct __align__(16) bf16x8 {
+    __nv_bfloat162 v[4];
+};
+
+}  // namespace mla

@@ -1,0 +1,206 @@
+/*
+ * mla.h -- C ABI of the absorbed Multi-head Latent Attention (MLA) decode
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V2; pages cited by title and section):
+ *   - the KV cache keeps, per token, only the joint latent c^KV = W^DKV h
+ *     (d_c = 512 values) and one decoupled RoPE key k^R = RoPE(W^KR h)
+ *     (d_r = 64 values) shared by all heads
+ *       [DeepSeek-V3 report summary (xyznot.com), Method 1 (MLA);
+ *        DeepSeek-V2 paper review (jiphyeonjeon.kr), sections 2-3];
+ *   - each head's content query is absorbed into the latent space,
+ *     q~_i = (U^K_i)^T q^C_i, so the score against token j is
+ *     (q~_i . c^KV_j + q^R_i . k^R_j) / sqrt(d_h + d_r)
+ *       [DeepSeek-V2 paper review, section 2 (absorption identity) and
+ *        section 3 (score and its 1/sqrt(128+64) scale)];
+ *   - the attention-weighted latents are summed and U^V_i (then O_i) is
+ *     applied once afterwards: o_i = U^V_i sum_j a_ij c^KV_j,
+ *     u = sum_i O_i o_i   [DeepSeek-V2 paper review, section 2].
+ *
+ * Conventions shared by every call:
+ *   - bf16 tensors are passed as pointers to 16-bit storage (IEEE bfloat16
+ *     bit patterns), row-major, contiguous, 16-byte aligned.
+ *   - Every pointer is caller-owned DEVICE memory unless stated otherwise.
+ *     The library allocates no device memory; scratch comes from the
+ *     caller's workspace.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Inputs are never modified,
+ *     except the cache by the append calls.
+ *   - Argument errors are returned synchronously and launch nothing.  A
+ *     failed launch returns MLA_ERR_CUDA.  Errors only the device can see
+ *     (bad block-table entries, sequence lengths out of range, a bounded
+ *     wait that gave up) set bits of a device error word (MLA_DEVERR_*);
+ *     the offending access is skipped, never performed.
+ *   - Supported shapes: d_c = 512, d_rope = 64, d_head = 128,
+ *     block_size = 64, num_heads a multiple of 16 in [16, 128].  Anything
+ *     else returns MLA_ERR_UNSUPPORTED.
+ *
+ * Paged latent cache layout (one model layer):
+ *   cache[num_blocks][block_size][d_c + d_rope] bf16; a row is
+ *   [c^KV (512) | k^R (64), already rotated] = 1152 bytes.  Logical position
+ *   p of sequence b lives in block block_table[b * max_blocks + p / 64],
+ *   slot p % 64.  The RoPE position of the token at logical position p is p.
+ */
+#ifndef MLA_H
+#define MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer */
+    MLA_ERR_UNSUPPORTED = 2, /* shape outside the supported set */
+    MLA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    MLA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+    MLA_ERR_DEVICE = 5       /* device error word non-zero (MLA_SYNC_CHECK) */
+} mla_status_t;
+
+/* Bits of the device error word. */
+#define MLA_DEVERR_BLOCK_ID 0x1u /* block-table entry outside [0, num_blocks) */
+#define MLA_DEVERR_SEQ_LEN  0x2u /* seq_len > max_blocks*block_size, or a query
+                                    with no visible key (seq_len < s), or a
+                                    position / sequence index out of range */
+#define MLA_DEVERR_TIMEOUT  0x4u /* a bounded device-side wait gave up */
+
+/* mla_decode flags */
+#define MLA_SYNC_CHECK   0x1u  /* synchronize the stream after the call and
+                                  return MLA_ERR_DEVICE if the error word is
+                                  non-zero */
+#define MLA_FORCE_SIMPLE 0x2u  /* run the CUDA-core decode kernel instead of
+                                  the tensor-core one (same results within
+                                  rounding; used to cross-check) */
+
+typedef struct {
+    int32_t num_heads;   /* H */
+    int32_t d_c;         /* latent width, 512 */
+    int32_t d_rope;      /* RoPE key / query width, 64 */
+    int32_t d_head;      /* per-head content width, 128 */
+    int32_t block_size;  /* tokens per cache block, 64 */
+    float softmax_scale; /* <= 0 selects 1/sqrt(d_head + d_rope) */
+    float rope_base;     /* RoPE base; <= 0 selects 10000 */
+} mla_dims_t;
+
+/* Human-readable name of a status code (static storage). */
+const char *mla_status_string(mla_status_t status);
+
+/*
+ * mla_append_cache -- step a1: project new tokens into the latent cache.
+ *   c^KV_t = W^DKV h_t,  k^R_t = RoPE(W^KR h_t, pos[t])
+ *   [DeepSeek-V2 paper review, section 2 (c^KV = W^DKV h);
+ *    DeepSeek-V3 report summary, Method 1 (k^R = RoPE(W^KR h), cache only
+ *    c^KV and k^R)]
+ * and writes row [c^KV | k^R] (rounded to bf16, fp32 accumulation) to the
+ * slot of (seq_idx[t], pos[t]).
+ *   h            [T][d_model] bf16
+ *   w_dkv        [d_c][d_model] bf16      (W^DKV)
+ *   w_kr         [d_rope][d_model] bf16   (W^KR)
+ *   seq_idx, pos [T] int32                (device)
+ *   block_table  [num_seqs][max_blocks] int32 (device)
+ *   cache        [num_blocks][block_size][d_c+d_rope] bf16, written in place
+ *   err_word     optional device uint32; bits MLA_DEVERR_* are OR-ed in for
+ *                tokens whose slot is invalid (those tokens are not written)
+ * d_model must be a positive multiple of 64.  T = 0 is a no-op.
+ */
+mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int d_model,
+                              const void *w_dkv, const void *w_kr,
+                              const int32_t *seq_idx, const int32_t *pos,
+                              const int32_t *block_table, int num_seqs, int max_blocks,
+                              void *cache, int num_blocks, uint32_t *err_word, void *stream);
+
+/*
+ * mla_append_latent -- the RoPE-and-scatter half of step a1, for callers that
+ * already hold the latent: writes [c_kv[t] | RoPE(k_rope[t], pos[t])] to the
+ * slot of (seq_idx[t], pos[t]).  Same sources as mla_append_cache.
+ *   c_kv   [T][d_c] bf16, copied bit for bit
+ *   k_rope [T][d_rope] bf16, the raw (unrotated) RoPE key W^KR h
+ * Other arguments as for mla_append_cache.
+ */
+mla_status_t mla_append_latent(const mla_dims_t *dims, const void *c_kv, const void *k_rope,
+                               int T, const int32_t *seq_idx, const int32_t *pos,
+                               const int32_t *block_table, int num_seqs, int max_blocks,
+                               void *cache, int num_blocks, uint32_t *err_word, void *stream);
+
+/*
+ * mla_absorb_q -- step a2: absorb U^K into the query.
+ *   q_abs[t][i][0:d_c]    = (U^K_i)^T q^C_{t,i}     (fp32 accumulation -> bf16)
+ *   q_abs[t][i][d_c:]     = RoPE(q^R_{t,i}, q_pos[t]), or q^R copied if
+ *                           q_pos == NULL (already rotated)
+ *   [DeepSeek-V2 paper review, section 2: (q^C)^T U^K c = ((U^K)^T q^C)^T c;
+ *    section 3: per-head RoPE query of 64 dims]
+ *   q_nope [T][H][d_head] bf16, q_rope [T][H][d_rope] bf16,
+ *   q_pos  [T] int32 or NULL, w_uk [H][d_head][d_c] bf16 (U^K_i),
+ *   q_abs  [T][H][d_c+d_rope] bf16 (output).
+ */
+mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void *q_rope,
+                          const int32_t *q_pos, const void *w_uk, int T, void *q_abs,
+                          void *stream);
+
+/*
+ * mla_decode_workspace_size -- bytes of device workspace mla_decode needs for
+ * B sequences of s query tokens whose lengths are at most max_seq_len.
+ */
+size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s, int max_seq_len);
+
+/*
+ * mla_decode -- steps a3-a6: absorbed attention over the paged latent cache,
+ * with split-KV partials merged by log-sum-exp.
+ *   l_ij = softmax_scale * (q_abs[i] . cache_row_j)      (576-d dot product)
+ *   out_latent[i] = sum_j softmax_j(l_ij) c^KV_j           (U^V not applied)
+ *   [DeepSeek-V2 paper review, section 3 (score, scale, softmax over j) and
+ *    section 2 (U^V pulled out of the weighted sum)]
+ * Query t in [0,s) of sequence b sees the positions j <= seq_lens[b] - s + t.
+ *   q_abs       [B*s][H][d_c+d_rope] bf16 (row = b*s + t)
+ *   cache, num_blocks, block_table [B][max_blocks] int32, seq_lens [B] int32
+ *   out_latent  [B*s][H][d_c] bf16
+ *   out_lse     [B*s][H] fp32 natural-log softmax denominator of the scaled
+ *               logits, or NULL.  A query with no visible key gets a zero
+ *               latent and lse = -inf (and MLA_DEVERR_SEQ_LEN).
+ *   workspace   device buffer of ws_bytes >= mla_decode_workspace_size();
+ *               its first 4 bytes are the device error word (cleared by the
+ *               call); the rest holds the split plan and partial results.
+ *   flags       MLA_SYNC_CHECK, MLA_FORCE_SIMPLE.
+ * Sequences are independent; calls that share a workspace must not overlap
+ * on the GPU.  B = 0 is a no-op.
+ */
+mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *cache,
+                        int num_blocks, const int32_t *block_table, int max_blocks,
+                        const int32_t *seq_lens, int B, int s, void *out_latent,
+                        float *out_lse, void *workspace, size_t ws_bytes, uint32_t flags,
+                        void *stream);
+
+/*
+ * mla_decode_error -- copy the device error word of a workspace into
+ * *err_host (blocking on `stream`), optionally clearing it.
+ */
+mla_status_t mla_decode_error(const void *workspace, uint32_t *err_host, int clear, void *stream);
+
+/*
+ * mla_up_v -- step a7: apply U^V (and optionally O) after the weighted sum.
+ *   out_heads[t][i] = U^V_i latent[t][i]                 (bf16, fp32 accum.)
+ *   out_model[t]    = sum_i O_i out_heads[t][i]          (if w_o != NULL)
+ *   [DeepSeek-V2 paper review, section 2: u_t = sum_i O_i U^V_i (sum_j a_ij c_j)]
+ *   latent    [T][H][d_c] bf16, w_uv [H][d_head][d_c] bf16 (U^V_i),
+ *   w_o       [d_model][H*d_head] bf16 (column block i is O_i) or NULL,
+ *   out_heads [T][H][d_head] bf16 (required), out_model [T][d_model] bf16.
+ */
+mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const void *w_uv,
+                      const void *w_o, int d_model, void *out_heads, void *out_model,
+                      void *stream);
+
+/*
+ * mla_kernel_launches -- number of CUDA kernels this library has launched in
+ * the calling process (all devices, all entry points).  A measurement aid:
+ * the difference across a region counts the library's launches in it.
+ */
+uint64_t mla_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H */

@@ -41,6 +41,7 @@ def load(path: str):
     lib = ctypes.CDLL(path)
     lib.mla_oracle_num_threads.restype = ctypes.c_int
     lib.mla_oracle_rope.argtypes = [_f64p, ctypes.c_int, ctypes.c_double, ctypes.c_double, _f64p]
+    lib.mla_oracle_rope_rows.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _i32p, ctypes.c_double, _f64p]
     lib.mla_oracle_kv_project.argtypes = [ctypes.c_int] * 4 + [_u16p, _u16p, _u16p, _i32p,
                                                              ctypes.c_double, _f64p, _f64p]
     lib.mla_oracle_absorb_q.argtypes = [ctypes.c_int] * 5 + [_f64p, _f64p, _i32p, _f64p,
@@ -110,6 +111,15 @@ def rope(x, pos: float, base: float = 10000.0) -> np.ndarray:
     x = _f64(x)
     y = np.empty_like(x)
     _lib().mla_oracle_rope(_p(x, _f64p), x.shape[-1], float(pos), float(base), _p(y, _f64p))
+    return y
+
+
+def rope_rows(x, pos, base: float = 10000.0) -> np.ndarray:
+    """RoPE of each row x[n] at position pos[n]."""
+    x, pos = _f64(x), _i32(pos)
+    y = np.empty_like(x)
+    _lib().mla_oracle_rope_rows(x.shape[0], x.shape[1], _p(x, _f64p), _p(pos, _i32p), float(base),
+                                _p(y, _f64p))
     return y
 
 

@@ -85,6 +85,15 @@ void mla_oracle_rope(const double *x, int d_r, double pos, double base, double *
     }
 }
 
+/* RoPE of N rows x [N][d_r] at positions pos[N] (the cache's k^R part). */
+void mla_oracle_rope_rows(int N, int d_r, const double *x, const int32_t *pos, double base,
+                          double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n)
+        mla_oracle_rope(x + (size_t)n * d_r, d_r, (double)pos[n], base, y + (size_t)n * d_r);
+}
+
 /* Append projection (step a1): for each of T tokens,
  *   c^KV = W^DKV h           (W^DKV: [d_c][d] row-major)
  *   k^R  = RoPE(W^KR h, pos) (W^KR : [d_r][d] row-major)

@@ -1,0 +1,114 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol
+include/mla.h declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    from head_latent_attention_10_b200 import build
+    build.build()
+    import head_latent_attention_10_b200 as M
+    M.load_library()
+    return M
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "mla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(M):
+    decl = declared_symbols()
+    assert len(decl) >= 8
+    lib = M.load_library()
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert set(decl) == set(M.EXPORTED)
+
+
+def test_library_has_no_libcuda_or_torch_dependency():
+    import subprocess
+    from head_latent_attention_10_b200 import LIB_PATH
+    out = subprocess.run(["ldd", LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda" not in out and "torch" not in out and "libcudart" not in out
+
+
+def test_status_strings(M):
+    for code in range(6):
+        assert M.mla_status_string(code).startswith("MLA_")
+    assert "unknown" in M.mla_status_string(99)
+
+
+def _raw(M):
+    return M.load_library()
+
+
+def test_unsupported_shapes_are_rejected(M):
+    lib = _raw(M)
+    p = ctypes.c_void_p(16)
+    for bad in (M.dims(8), M.dims(136), M.dims(24), M.dims(128, d_c=256), M.dims(128, block_size=32)):
+        st = lib.mla_decode(ctypes.byref(bad), p, p, 1, p, 1, p, 1, 1, p, None, p, 1 << 30, 0, None)
+        assert st == M.MLA_ERR_UNSUPPORTED
+        assert lib.mla_decode_workspace_size(ctypes.byref(bad), 1, 1, 64) == 0
+
+
+def test_argument_errors(M):
+    lib = _raw(M)
+    d = M.dims(128)
+    p = ctypes.c_void_p(256)
+    assert lib.mla_decode(None, p, p, 1, p, 1, p, 1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode(ctypes.byref(d), None, p, 1, p, 1, p, 1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode(ctypes.byref(d), p, p, 1, p, 1, p, -1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode(ctypes.byref(d), p, p, 1, p, 1, p, 1, 0, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    # misaligned
+    q = ctypes.c_void_p(258)
+    assert lib.mla_decode(ctypes.byref(d), q, p, 1, p, 1, p, 1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    # workspace missing or too small
+    assert lib.mla_decode(ctypes.byref(d), p, p, 1, p, 1, p, 1, 1, p, None, None, 0, 0, None) == M.MLA_ERR_WORKSPACE
+    assert lib.mla_decode(ctypes.byref(d), p, p, 1, p, 1, p, 1, 1, p, None, p, 16, 0, None) == M.MLA_ERR_WORKSPACE
+    # empty batch is a no-op that succeeds without touching the GPU
+    assert lib.mla_decode(ctypes.byref(d), None, None, 0, None, 0, None, 0, 1, None, None, None, 0, 0, None) == M.MLA_OK
+    assert lib.mla_absorb_q(ctypes.byref(d), p, p, None, p, 0, p, None) == M.MLA_OK
+    assert lib.mla_absorb_q(ctypes.byref(d), None, p, None, p, 4, p, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_up_v(ctypes.byref(d), p, 4, p, p, 100, p, p, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_up_v(ctypes.byref(d), p, 4, None, None, 0, p, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_cache(ctypes.byref(d), p, 4, 100, p, p, p, p, p, 1, 1, p, 1, None, None) == M.MLA_ERR_UNSUPPORTED
+    assert lib.mla_append_latent(ctypes.byref(d), p, p, -1, p, p, p, 1, 1, p, 1, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_error(None, None, 0, None) == M.MLA_ERR_INVALID_ARG
+
+
+def test_workspace_size_grows_with_batch(M):
+    lib = _raw(M)
+    d = M.dims(128)
+    a = lib.mla_decode_workspace_size(ctypes.byref(d), 1, 1, 4096)
+    b = lib.mla_decode_workspace_size(ctypes.byref(d), 128, 1, 4096)
+    c = lib.mla_decode_workspace_size(ctypes.byref(d), 128, 2, 4096)
+    assert 0 < a < b <= c and a % 256 == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import head_latent_attention_10_b200 as M
+    saved = M._LIB
+    M._LIB = None
+    try:
+        with pytest.raises(RuntimeError):
+            M.load_library(str(tmp_path / "nope.so"))
+    finally:
+        M._LIB = saved
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "head_latent_attention_10_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "mla_oracle" not in text, f

@@ -1,0 +1,239 @@
+"""GPU parity: every library call against the fp64 oracle on seeded inputs.
+
+Sizes are ones the oracle finishes in seconds while still spanning several
+64-token blocks, several KV splits and ragged tails.  The bar (written in
+assert_parity): max-abs error <= 2e-2 and relative L2 error <= 1e-2 for
+floating point; bit-exact for the cache placement.
+"""
+import numpy as np
+import pytest
+
+import mla_workloads as W
+from _gpu_setup import GpuWorkload, assert_parity, host_bits, i32, rel_l2, torch_bits
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    W.MLAConfig("h16_ragged", B=3, s=1, H=16, L=0, paged=True, seed=201, d_model=2048,
+                seq_lens=(1000, 65, 1)),
+    W.MLAConfig("h128_ragged", B=3, s=1, H=128, L=0, paged=True, seed=202, d_model=5120,
+                seq_lens=(700, 129, 63)),
+    W.MLAConfig("h128_two_queries", B=3, s=2, H=128, L=0, paged=True, seed=203, d_model=5120,
+                seq_lens=(300, 2, 1500)),
+    W.MLAConfig("h64_many_splits", B=2, s=1, H=64, L=0, paged=True, seed=204, d_model=4096,
+                seq_lens=(2500, 1100)),
+    W.MLAConfig("h32_contiguous", B=2, s=1, H=32, L=0, paged=False, seed=205, d_model=2048,
+                seq_lens=(257, 64)),
+    W.CONFIGS["tiny"],
+]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import head_latent_attention_10_b200 as M
+    M.load_library()
+    return M
+
+
+def _oracle():
+    import oracle
+    return oracle
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_cache_writer_places_rows_bit_exactly(lib, cfg):
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    d = g.d
+    got = host_bits(g.cache)
+    # latent part: bit for bit at the slot the block table names; every
+    # slot no token maps to is still NaN
+    assert np.array_equal(got[..., :cfg.d_c], d["cache"][..., :cfg.d_c])
+    # RoPE part: the rotated raw key, within bf16 rounding of the fp64 rotation
+    bt = d["block_table"]
+    blk = bt[d["tok_seq"], d["tok_pos"] // 64]
+    slot = d["tok_pos"] % 64
+    kr_gpu = W.bf16_bits_to_f32(got[blk, slot, cfg.d_c:]).astype(np.float64)
+    kr_ref = o.rope_rows(o.bf16_to_f64(d["k_rope"]), d["tok_pos"])
+    assert np.max(np.abs(kr_gpu - kr_ref) / (np.abs(kr_ref) + 1e-2)) < 2 ** -7
+    mask = np.ones(got.shape[:2], bool)
+    mask[blk, slot] = False
+    assert np.all(got[mask] == d["cache"][mask])
+    assert int(g.err.item()) == 0
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_absorb_q(lib, cfg):
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    got = W.bf16_bits_to_f32(host_bits(g.absorb()))
+    ref = o.absorb_q(o.bf16_to_f64(g.d["q_nope"]), o.bf16_to_f64(g.d["q_rope"]),
+                     o.bf16_to_f64(g.d["w_uk"]), q_pos=g.d["q_pos"])
+    assert_parity(got, ref, what="absorb_q")
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+@pytest.mark.parametrize("flags", [0, 2], ids=["default", "simple"])
+def test_decode_latent(lib, cfg, flags):
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    q_abs_bits = W.make_q_abs(cfg)
+    lat, lse = g.decode(torch_bits(q_abs_bits), flags=flags)
+    ref, rlse = o.decode_latent(g.d["cache"], g.d["block_table"], g.d["seq_lens"], cfg.s,
+                                o.bf16_to_f64(q_abs_bits))
+    got = W.bf16_bits_to_f32(host_bits(lat)).reshape(ref.shape)
+    assert_parity(got, ref, what="latent")
+    # lse moves with the logits: the cache holds the rotated k^R rounded to
+    # bf16 (relative 2^-9 per element), so a logit can move by up to
+    # scale * sum_m |q^R_m| |k^R_m| 2^-9 ~ 1e-2 for N(0,1) data.
+    np.testing.assert_allclose(lse.cpu().numpy().ravel(), rlse, atol=1e-2, rtol=0)
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_full_path_against_expanded_oracle(lib, cfg):
+    """absorb -> decode -> up_v on the GPU against the textbook expanded form."""
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    out = g.up_v(g.decode(g.absorb())[0])
+    got = W.bf16_bits_to_f32(host_bits(out)).astype(np.float64)
+    rng = np.random.default_rng(cfg.seed)
+    heads = np.sort(rng.choice(cfg.H, size=min(cfg.H, 16), replace=False))
+    rows = np.repeat(np.arange(cfg.T), heads.size)
+    hh = np.tile(heads, cfg.T)
+    f = o.bf16_to_f64
+    ref, _, _ = o.decode_expanded(g.d["cache"], g.d["block_table"], g.d["seq_lens"], cfg.s,
+                                  f(g.d["q_nope"]), f(g.d["q_rope"]), f(g.d["w_uk"]), f(g.d["w_uv"]),
+                                  q_pos=g.d["q_pos"], rows=rows, heads=hh)
+    assert_parity(got[rows, hh], ref, what="o")
+
+
+@pytest.mark.parametrize("cfg", SMALL[:3], ids=lambda c: c.name)
+def test_up_v_and_out_proj(lib, cfg):
+    import torch
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    lat_bits = W.make_latent(cfg)
+    w_o = W.make_w_o(cfg)
+    out_h = torch.empty(cfg.T, cfg.H, cfg.d_h, dtype=torch.bfloat16, device="cuda")
+    out_m = torch.empty(cfg.T, cfg.d_model, dtype=torch.bfloat16, device="cuda")
+    lib.mla_up_v(g.dims, torch_bits(lat_bits), g.w_uv, out_h, w_o=torch_bits(w_o), out_model=out_m)
+    ref_h = o.up_v(o.bf16_to_f64(lat_bits), o.bf16_to_f64(g.d["w_uv"]))
+    assert_parity(W.bf16_bits_to_f32(host_bits(out_h)), ref_h, what="heads")
+    ref_m = o.out_proj(ref_h, o.bf16_to_f64(w_o))
+    assert_parity(W.bf16_bits_to_f32(host_bits(out_m)), ref_m, what="model")
+
+
+@pytest.mark.parametrize("cfg", SMALL[:2], ids=lambda c: c.name)
+def test_append_cache_projection(lib, cfg):
+    import torch
+    o = _oracle()
+    g = GpuWorkload(cfg)
+    T = 37
+    a = W.make_append_inputs(cfg, T)
+    rng = np.random.default_rng(3)
+    seq = rng.integers(0, cfg.B, T).astype(np.int32)
+    maxpos = g.d["block_table"].shape[1] * 64
+    pos = np.array([rng.integers(0, min(maxpos, int(g.d["seq_lens"][b]) + 1)) if g.d["seq_lens"][b] > 0
+                    else 0 for b in seq], np.int32)
+    # one token per slot so that the writes do not collide
+    _, uniq = np.unique(seq.astype(np.int64) * maxpos + pos, return_index=True)
+    seq, pos = seq[np.sort(uniq)], pos[np.sort(uniq)]
+    h = a["h"][: seq.size]
+    cache0 = host_bits(g.cache)
+    lib.mla_append_cache(g.dims, torch_bits(h), torch_bits(a["w_dkv"]), torch_bits(a["w_kr"]),
+                         i32(seq), i32(pos), g.block_table, g.cache, err_word=g.err)
+    got = host_bits(g.cache)
+    c_ref, kr_ref = o.kv_project(h, a["w_dkv"], a["w_kr"], pos)
+    bt = g.d["block_table"]
+    blk, slot = bt[seq, pos // 64], pos % 64
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, :512]), c_ref, what="c_kv")
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, 512:]), kr_ref, what="k_rope")
+    mask = np.ones(got.shape[:2], bool); mask[blk, slot] = False
+    assert np.array_equal(got[mask], cache0[mask])
+
+
+def test_append_cache_identity_weights_are_bit_exact(lib):
+    """W^DKV = [I 0], W^KR = [0 I] at position 0 copies h bit for bit
+    (projection by I is exact in fp32; RoPE at 0 is the identity)."""
+    import torch
+    cfg = W.MLAConfig("ident", B=2, s=1, H=16, L=0, paged=True, seed=301, d_model=576,
+                      seq_lens=(5, 70))
+    g = GpuWorkload(cfg)
+    h = W.f32_to_bf16_bits(np.random.default_rng(1).standard_normal((2, 576)).astype(np.float32))
+    eye = np.eye(576, dtype=np.float32)
+    wd, wr = W.f32_to_bf16_bits(eye[:512]), W.f32_to_bf16_bits(eye[512:])
+    seq = np.array([0, 1], np.int32); pos = np.array([0, 0], np.int32)
+    lib.mla_append_cache(g.dims, torch_bits(h), torch_bits(wd), torch_bits(wr), i32(seq), i32(pos),
+                         g.block_table, g.cache)
+    got = host_bits(g.cache)
+    bt = g.d["block_table"]
+    assert np.array_equal(got[bt[0, 0], 0], h[0]) and np.array_equal(got[bt[1, 0], 0], h[1])
+
+
+def test_block_permutation_gives_bitwise_identical_outputs(lib):
+    cfg = W.MLAConfig("perm", B=4, s=2, H=128, L=0, paged=True, seed=401, d_model=5120,
+                      seq_lens=(900, 64, 65, 333))
+    q = torch_bits(W.make_q_abs(cfg))
+    a = GpuWorkload(cfg).decode(q)
+    b = GpuWorkload(cfg.with_(paged=False)).decode(q)
+    assert np.array_equal(host_bits(a[0]), host_bits(b[0]))
+    assert np.array_equal(a[1].cpu().numpy(), b[1].cpu().numpy())
+
+
+def test_heads_with_distinct_queries_get_distinct_outputs(lib):
+    cfg = W.MLAConfig("heads", B=1, s=1, H=16, L=300, paged=True, seed=402, d_model=2048)
+    g = GpuWorkload(cfg)
+    lat, _ = g.decode(torch_bits(W.make_q_abs(cfg)))
+    x = W.bf16_bits_to_f32(host_bits(lat))[0]
+    assert min(np.max(np.abs(x[i] - x[j])) for i in range(16) for j in range(i)) > 1e-3
+
+
+def test_single_token_returns_the_latent_exactly(lib):
+    cfg = W.MLAConfig("one", B=3, s=1, H=128, L=1, paged=True, seed=403, d_model=5120)
+    g = GpuWorkload(cfg)
+    lat, lse = g.decode(torch_bits(W.make_q_abs(cfg)))
+    got = host_bits(lat)
+    for b in range(3):
+        assert np.all(got[b] == g.d["c_kv"][b][None, :])
+
+
+def test_bad_block_table_entry_sets_device_error(lib):
+    import torch
+    cfg = W.MLAConfig("bad", B=2, s=1, H=16, L=0, paged=True, seed=404, d_model=2048, seq_lens=(130, 40))
+    g = GpuWorkload(cfg)
+    g.block_table[0, 1] = g.cache.shape[0] + 5
+    with pytest.raises(lib.MLAError) as e:
+        g.decode(torch_bits(W.make_q_abs(cfg)), flags=lib.MLA_SYNC_CHECK)
+    assert e.value.status == lib.MLA_ERR_DEVICE
+    assert lib.mla_decode_error(g.ws) & lib.MLA_DEVERR_BLOCK_ID
+    torch.cuda.synchronize()
+    # the other sequence is unaffected and the context still works
+    lat, _ = g.decode(torch_bits(W.make_q_abs(cfg)))
+    assert np.isfinite(W.bf16_bits_to_f32(host_bits(lat))[1]).all()
+
+
+def test_seq_len_beyond_table_and_short_rows(lib):
+    import torch
+    cfg = W.MLAConfig("short", B=2, s=2, H=16, L=0, paged=True, seed=405, d_model=2048, seq_lens=(1, 50))
+    g = GpuWorkload(cfg)
+    lat, lse = g.decode(torch_bits(W.make_q_abs(cfg)))
+    err = lib.mla_decode_error(g.ws, clear=True)
+    assert err & lib.MLA_DEVERR_SEQ_LEN
+    x = W.bf16_bits_to_f32(host_bits(lat))
+    assert np.all(x[0] == 0) and np.all(np.isneginf(lse[0].cpu().numpy()))
+    assert np.isfinite(x[1:]).all()
+    g.seq_lens[1] = g.block_table.shape[1] * 64 + 1
+    with pytest.raises(lib.MLAError):
+        g.decode(torch_bits(W.make_q_abs(cfg)), flags=lib.MLA_SYNC_CHECK)
+    torch.cuda.synchronize()
+
+
+def test_empty_batch_is_a_no_op(lib):
+    import torch
+    d = lib.dims(128)
+    z = torch.empty(0, dtype=torch.int32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    q = torch.empty(0, 128, 576, dtype=torch.bfloat16, device="cuda")
+    cache = torch.empty(1, 64, 576, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(0, 128, 512, dtype=torch.bfloat16, device="cuda")
+    lib.mla_decode(d, q, cache, z.view(0, 1), z, 1, out, None, ws)
