@@ -4,8 +4,13 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <stdlib.h>
+
 #include "common.cuh"
 #include "k_simple.cuh"
+#include "tc_decode.cuh"
+#include "tc_gemm.cuh"
+#include "tmap.cuh"
 
 using namespace mla;
 
@@ -41,6 +46,82 @@ inline double rope_base(const mla_dims_t *d)
 }
 
 inline mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// Bound of every device-side wait (ns).  MLA_DEBUG_WAIT_LIMIT_NS overrides it
+// so that tests can make a wait give up on purpose.
+unsigned long long wait_limit_ns()
+{
+    const char *e = getenv("MLA_DEBUG_WAIT_LIMIT_NS");
+    if (e && *e) {
+        const unsigned long long v = strtoull(e, nullptr, 10);
+        if (v > 0) return v;
+    }
+    return 2000000000ull;
+}
+
+// A bf16 tensor map over a row-major 2-D or batched 3-D operand.
+//   rows x inner elements per batch entry, row stride and batch stride in elements.
+bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t batch, uint64_t row_stride,
+          uint64_t batch_stride, uint32_t box_inner, uint32_t box_rows)
+{
+    const uint64_t s1 = row_stride * 2, s2 = (batch > 1 ? batch_stride : row_stride * rows) * 2;
+    return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
+}
+
+// Tensor-core decode workspace: [error word][plan][partial latents][partial lse2]
+struct TcWs {
+    size_t off_plan, off_o, off_lse, total;
+};
+
+TcWs tc_ws(int H, int T)
+{
+    TcWs w;
+    w.off_plan = kWsAlign;
+    w.off_o = align_up(w.off_plan + (size_t)(4 + T + 1) * sizeof(int32_t), kWsAlign);
+    const size_t slots = 2 * (size_t)kMaxClusters * H;
+    w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
+    w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
+    return w;
+}
+
+// Clusters of the decode kernel that fit on the device at once (cached per device).
+int decode_clusters()
+{
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] > 0) return cache[dev];
+    if (cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) != cudaSuccess)
+        return 0;
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = kDecSmem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void *)tc_decode_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sms / 2;
+    }
+    if (n > kMaxClusters) n = kMaxClusters;
+    cache[dev] = n;
+    return n;
+}
+
+template <int BN, bool kBmn, class Epi>
+cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
+                           uint32_t *err, cudaStream_t st)
+{
+    using S = GemmSmem<BN>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
+    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, wait_limit_ns());
+    count_launch();
+    return cudaGetLastError();
+}
 
 // Workspace of the decode: [error word | pad] [partial latents] [partial lse2]
 struct SimpleWs {
@@ -113,17 +194,20 @@ mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int 
     if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(cache))
         return MLA_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
+    CUtensorMap ma, mb1, mb2;
+    if (!tmap(&ma, h, d_model, T, 1, d_model, 0, 64, 128) ||
+        !tmap(&mb1, w_dkv, d_model, kDc, 1, d_model, 0, 64, 256) ||
+        !tmap(&mb2, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
+        return MLA_ERR_CUDA;
     // c^KV = W^DKV h  (columns 0..511 of the row)
-    GemmArgs g{T, kDc, d_model, (const bf16 *)h, 0, d_model, 1, (const bf16 *)w_dkv, 0, 1, d_model};
-    EpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, false,
-                rope_base(dims), err_word};
-    cudaError_t ce = launch_gemm_simple(g, 1, e, s);
-    if (ce != cudaSuccess) return MLA_ERR_CUDA;
+    TcEpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, 0,
+                  rope_base(dims), err_word};
+    if (launch_tc_gemm<256, false>(ma, mb1, T, kDc, d_model, 1, e, err_word, s) != cudaSuccess)
+        return MLA_ERR_CUDA;
     // k^R = RoPE(W^KR h)  (columns 512..575)
-    GemmArgs g2{T, kDr, d_model, (const bf16 *)h, 0, d_model, 1, (const bf16 *)w_kr, 0, 1, d_model};
-    EpiAppend e2{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, kDc, true,
-                 rope_base(dims), nullptr};
-    return cuda_status(launch_gemm_simple(g2, 1, e2, s));
+    TcEpiAppend e2{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, kDc, 1,
+                   rope_base(dims), nullptr};
+    return cuda_status(launch_tc_gemm<64, false>(ma, mb2, T, kDr, d_model, 1, e2, err_word, s));
 }
 
 mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void *q_rope,
@@ -139,11 +223,12 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
     const int H = dims->num_heads;
     cudaStream_t s = as_stream(stream);
     // per head i: q_abs[:, i, 0:512] = q_nope[:, i, :] (T x 128) . U^K_i (128 x 512)
-    GemmArgs g{T, kDc, kDh, (const bf16 *)q_nope, kDh, (long long)H * kDh, 1,
-               (const bf16 *)w_uk, (long long)kDh * kDc, kDc, 1};
-    EpiStoreBf16 e{(bf16 *)q_abs, kRow, (long long)H * kRow};
-    cudaError_t ce = launch_gemm_simple(g, H, e, s);
-    if (ce != cudaSuccess) return MLA_ERR_CUDA;
+    CUtensorMap ma, mb;
+    if (!tmap(&ma, q_nope, kDh, T, H, (uint64_t)H * kDh, kDh, 64, 128) ||
+        !tmap(&mb, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64))
+        return MLA_ERR_CUDA;
+    TcEpiStore e{(bf16 *)q_abs, kRow, (long long)H * kRow};
+    if (launch_tc_gemm<256, true>(ma, mb, T, kDc, kDh, H, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
     const int warps = T * H;
     rope_q_kernel<<<(warps + 7) / 8, 256, 0, s>>>((const bf16 *)q_rope, q_pos, T, H, (bf16 *)q_abs,
                                                   rope_base(dims));
@@ -154,7 +239,9 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
 size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s, int max_seq_len)
 {
     if (check_dims(dims) != MLA_OK || B < 0 || s <= 0 || max_seq_len < 0) return 0;
-    return simple_ws(dims->num_heads, B * s, max_seq_len).total;
+    const size_t a = simple_ws(dims->num_heads, B * s, max_seq_len).total;
+    const size_t b = tc_ws(dims->num_heads, B * s).total;
+    return a > b ? a : b;
 }
 
 mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *cache, int num_blocks,
@@ -170,29 +257,70 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
     if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(out_latent)) return MLA_ERR_INVALID_ARG;
     if (!workspace) return MLA_ERR_WORKSPACE;
     const int H = dims->num_heads, T = B * s;
-    const SimpleWs w = simple_ws(H, T, max_blocks * kBlock);
-    if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
     cudaStream_t strm = as_stream(stream);
     char *ws = (char *)workspace;
     uint32_t *err = (uint32_t *)ws;
-    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
     const float scale_log2 = softmax_scale(dims) * kLog2e;
-    float *po = (float *)(ws + w.off_o);
-    float *pl = (float *)(ws + w.off_lse);
-    dim3 grid(T, H / kSimpleHeads, w.nsplit);
-    if (cudaFuncSetAttribute(decode_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSimpleSmem) != cudaSuccess)
-        return MLA_ERR_CUDA;
-    decode_simple_kernel<<<grid, 256, kSimpleSmem, strm>>>((const bf16 *)q_abs, (const bf16 *)cache, num_blocks,
-                                                 block_table, max_blocks, seq_lens, s, H, scale_log2,
-                                                 po, pl, w.nsplit, err);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    combine_simple_kernel<<<dim3(T, H), 128, 0, strm>>>(po, pl, w.nsplit, kSimpleSplit, seq_lens,
-                                                        max_blocks, s, H, (bf16 *)out_latent, out_lse,
-                                                        err);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (flags & MLA_FORCE_SIMPLE) {
+        const SimpleWs w = simple_ws(H, T, max_blocks * kBlock);
+        if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+        if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
+        float *po = (float *)(ws + w.off_o);
+        float *pl = (float *)(ws + w.off_lse);
+        dim3 grid(T, H / kSimpleHeads, w.nsplit);
+        if (cudaFuncSetAttribute(decode_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSimpleSmem) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        decode_simple_kernel<<<grid, 256, kSimpleSmem, strm>>>((const bf16 *)q_abs, (const bf16 *)cache,
+                                                               num_blocks, block_table, max_blocks, seq_lens, s,
+                                                               H, scale_log2, po, pl, w.nsplit, err);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+        combine_simple_kernel<<<dim3(T, H), 128, 0, strm>>>(po, pl, w.nsplit, kSimpleSplit, seq_lens,
+                                                            max_blocks, s, H, (bf16 *)out_latent, out_lse, err);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    } else {
+        const TcWs w = tc_ws(H, T);
+        if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+        const int nc = decode_clusters();
+        if (nc <= 0) return MLA_ERR_CUDA;
+        CUtensorMap mq, mqr, mkv, mkvr;
+        const uint64_t rows = (uint64_t)num_blocks * kBlock;
+        if (!tmap(&mq, q_abs, kRow, H, T, kRow, (uint64_t)H * kRow, 64, 128) ||
+            !tmap(&mqr, q_abs, kRow, H, T, kRow, (uint64_t)H * kRow, 32, 128) ||
+            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, 64) ||
+            !tmap(&mkvr, cache, kRow, rows, 1, kRow, 0, 32, 64))
+            return MLA_ERR_CUDA;
+        if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
+        int32_t *plan = (int32_t *)(ws + w.off_plan);
+        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, nc, plan, err);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+        DecArgs da;
+        da.block_table = block_table;
+        da.seq_lens = seq_lens;
+        da.plan = plan;
+        da.out = (bf16 *)out_latent;
+        da.out_lse = out_lse;
+        da.part_o = (float *)(ws + w.off_o);
+        da.part_lse2 = (float *)(ws + w.off_lse);
+        da.err = err;
+        da.limit_ns = wait_limit_ns();
+        da.scale_log2 = scale_log2;
+        da.max_blocks = max_blocks;
+        da.num_blocks = num_blocks;
+        da.s = s;
+        da.H = H;
+        da.T = T;
+        tc_decode_kernel<<<2 * nc, kDecThreads, kDecSmem, strm>>>(mq, mqr, mkv, mkvr, da);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+        dec_combine_kernel<<<dim3(T, H), 128, 0, strm>>>(plan, da.part_o, da.part_lse2, H, (bf16 *)out_latent,
+                                                          out_lse);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
     if (flags & MLA_SYNC_CHECK) {
         uint32_t host = 0;
         if (cudaMemcpyAsync(&host, err, sizeof host, cudaMemcpyDeviceToHost, strm) != cudaSuccess)
@@ -224,19 +352,26 @@ mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const v
     if (T == 0) return MLA_OK;
     if (!latent || !w_uv || !out_heads) return MLA_ERR_INVALID_ARG;
     if (w_o && (!out_model || d_model <= 0 || d_model % 64 != 0)) return MLA_ERR_INVALID_ARG;
+    if (w_o && (!aligned16(w_o) || !aligned16(out_model))) return MLA_ERR_INVALID_ARG;
     if (!aligned16(latent) || !aligned16(w_uv) || !aligned16(out_heads)) return MLA_ERR_INVALID_ARG;
     const int H = dims->num_heads;
     cudaStream_t s = as_stream(stream);
     // per head i: out[:, i, :] = latent[:, i, :] (T x 512) . (U^V_i)^T (512 x 128)
-    GemmArgs g{T, kDh, kDc, (const bf16 *)latent, kDc, (long long)H * kDc, 1,
-               (const bf16 *)w_uv, (long long)kDh * kDc, 1, kDc};
-    EpiStoreBf16 e{(bf16 *)out_heads, kDh, (long long)H * kDh};
-    if (launch_gemm_simple(g, H, e, s) != cudaSuccess) return MLA_ERR_CUDA;
+    CUtensorMap ma, mb;
+    if (!tmap(&ma, latent, kDc, T, H, (uint64_t)H * kDc, kDc, 64, 128) ||
+        !tmap(&mb, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128))
+        return MLA_ERR_CUDA;
+    TcEpiStore e{(bf16 *)out_heads, kDh, (long long)H * kDh};
+    if (launch_tc_gemm<128, false>(ma, mb, T, kDh, kDc, H, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
     if (w_o) {
+        // out_model = out_heads (T x H*128) . W^O^T
         const int K = H * kDh;
-        GemmArgs g2{T, d_model, K, (const bf16 *)out_heads, 0, K, 1, (const bf16 *)w_o, 0, 1, K};
-        EpiStoreBf16 e2{(bf16 *)out_model, 0, d_model};
-        if (launch_gemm_simple(g2, 1, e2, s) != cudaSuccess) return MLA_ERR_CUDA;
+        CUtensorMap ma2, mb2;
+        if (!tmap(&ma2, out_heads, K, T, 1, K, 0, 64, 128) || !tmap(&mb2, w_o, K, d_model, 1, K, 0, 64, 256))
+            return MLA_ERR_CUDA;
+        TcEpiStore e2{(bf16 *)out_model, 0, d_model};
+        if (launch_tc_gemm<256, false>(ma2, mb2, T, d_model, K, 1, e2, nullptr, s) != cudaSuccess)
+            return MLA_ERR_CUDA;
     }
     return MLA_OK;
 }

@@ -1,0 +1,200 @@
+// tc_gemm.cuh -- tensor-core GEMM for the projections around the decode
+// (query absorption, U^V / O up-projection, the append projection):
+//   C[z][m][n] = sum_k A[z][m][k] * B[z][k][n],  bf16 in, fp32 accumulate.
+//
+// One CTA computes a 128 x BN tile.  Warp 0 streams 64-wide K slices of A
+// and B into a 4-stage shared-memory ring with TMA (128-byte swizzle), warp 1
+// issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator and frees
+// each stage with tcgen05.commit, and warps 2-5 read the accumulator back
+// with tcgen05.ld (one TMEM lane = one output row per thread) and hand 16
+// columns at a time to the epilogue functor.
+//
+// A is K-major (rows of K contiguous).  B is either K-major (B^T stored
+// row-major, e.g. a weight [N][K]) or MN-major (B stored [K][N]).
+// Tensor maps are 3-D: A {K, M, Z}, B K-major {K, N, Z}, B MN-major {N, K, Z}.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace mla {
+
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmSmem {
+    static constexpr int A = 128 * 64 * 2;
+    static constexpr int B = BN * 64 * 2;
+    static constexpr int STAGE = A + B;
+    static constexpr int BAR = kGemmStages * STAGE;
+    static constexpr int BYTES = BAR + 256 + 1024;  // + barriers + alignment slack
+    static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+};
+
+template <int BN, bool kBmn, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, int M,
+               int N, int K, Epi epi, uint32_t *err, unsigned long long limit_ns)
+{
+    using S = GemmSmem<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::BAR);
+    uint64_t *empty = full + kGemmStages;
+    uint64_t *done = empty + kGemmStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * 128, z = blockIdx.z;
+    const int nk = K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            sm100::mbar_init(&full[s], 1);
+            sm100::mbar_init(&empty[s], 1);
+        }
+        sm100::mbar_init(done, 1);
+        *abort_flag = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tensormap(&mapA);
+        sm100::prefetch_tensormap(&mapB);
+    }
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, S::TMEM_COLS);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const unsigned long long drain_ns = limit_ns > 200000000ull ? limit_ns : 200000000ull;
+    if (warp == 0) {
+        if (sm100::elect_one()) {
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % kGemmStages;
+                const uint32_t use = kb / kGemmStages;
+                if (use > 0 && !sm100::mbar_wait(&empty[s], (use - 1) & 1, abort_flag, err, limit_ns)) break;
+                issued = kb + 1;
+                uint8_t *a = smem + s * S::STAGE;
+                uint8_t *b = a + S::A;
+                sm100::mbar_arrive_expect_tx(&full[s], S::STAGE);
+                sm100::tma_load_3d(&mapA, &full[s], a, kb * 64, m0, z);
+                if (kBmn) {
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        sm100::tma_load_3d(&mapB, &full[s], b + j * 8192, n0 + 64 * j, kb * 64, z);
+                } else {
+                    sm100::tma_load_3d(&mapB, &full[s], b, kb * 64, n0, z);
+                }
+            }
+            if (*abort_flag) {
+                // never leave a copy in flight into shared memory: wait for the
+                // last load issued on every stage
+                volatile int no_abort = 0;
+                for (int kb = issued - kGemmStages < 0 ? 0 : issued - kGemmStages; kb < issued; ++kb)
+                    sm100::mbar_wait(&full[kb % kGemmStages], (kb / kGemmStages) & 1, &no_abort, err, drain_ns);
+            }
+        }
+    } else if (warp == 1) {
+        if (sm100::elect_one()) {
+            const uint32_t idesc = sm100::idesc_bf16(128, BN, 0, kBmn ? 1 : 0);
+            bool ok = true;
+            for (int kb = 0; kb < nk && ok; ++kb) {
+                const int s = kb % kGemmStages;
+                ok = sm100::mbar_wait(&full[s], (kb / kGemmStages) & 1, abort_flag, err, limit_ns);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                const uint32_t a = sm100::smem_u32(smem + s * S::STAGE);
+                const uint32_t b = a + S::A;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = sm100::desc_kmajor(a + kk * 32, 128, sm100::kSw128);
+                    const uint64_t bd = kBmn ? sm100::desc_mnmajor_sw128(b + kk * 16 * 128, 8192)
+                                             : sm100::desc_kmajor(b + kk * 32, 128, sm100::kSw128);
+                    sm100::umma_ss(tmem, ad, bd, idesc, (kb | kk) != 0);
+                }
+                sm100::umma_commit(&empty[s]);
+            }
+            sm100::umma_commit(done);
+        }
+    } else {
+        // epilogue: warps 2..5 cover TMEM lane quarters 2,3,0,1
+        const int q = warp & 3;
+        const bool ok = sm100::mbar_wait(done, 0, abort_flag, err, limit_ns);
+        sm100::tc_fence_after();
+        const int m = m0 + q * 32 + lane;
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                uint32_t r[16];
+                sm100::tmem_ld16(sm100::tmem_addr(tmem, q * 32, c), r);
+                sm100::tmem_wait_ld();
+                if (m < M && n0 + c < N) epi(z, m, n0 + c, reinterpret_cast<const float *>(r));
+            }
+        }
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        if (*abort_flag) {  // every issued MMA has retired before TMEM is freed
+            volatile int no_abort = 0;
+            sm100::mbar_wait(done, 0, &no_abort, err, drain_ns);
+        }
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, S::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- epilogues
+// 16 consecutive outputs -> bf16 at base + z*bs + m*rs + n (32-byte aligned).
+struct TcEpiStore {
+    bf16 *base;
+    long long bs, rs;
+    __device__ void operator()(int z, int m, int n, const float *v) const
+    {
+        uint4 pk[2];
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(pk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        uint4 *p = reinterpret_cast<uint4 *>(base + z * bs + m * rs + n);
+        p[0] = pk[0];
+        p[1] = pk[1];
+    }
+};
+
+// Append: token m's projected columns go to its cache slot; with `rope` the
+// 16 columns are RoPE dims n..n+15 (8 pairs) and are turned first.
+struct TcEpiAppend {
+    bf16 *cache;
+    const int32_t *seq_idx, *pos, *block_table;
+    int num_seqs, max_blocks, num_blocks, col0;
+    int rope;
+    double base;
+    uint32_t *err;
+    __device__ void operator()(int, int m, int n, const float *v) const
+    {
+        const int p = pos[m];
+        const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks, seq_idx[m], p,
+                                          n == 0 ? err : nullptr);
+        if (slot < 0) return;
+        float o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = v[i];
+        if (rope) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rope_pair(v[2 * i], v[2 * i + 1], p, n / 2 + i, kDr, base, &o[2 * i], &o[2 * i + 1]);
+        }
+        uint4 pk[2];
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(pk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+        uint4 *dst = reinterpret_cast<uint4 *>(cache + slot * kRow + col0 + n);
+        dst[0] = pk[0];
+        dst[1] = pk[1];
+    }
+};
+
+}  // namespace mla
