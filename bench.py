@@ -179,6 +179,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     cfg = W.CONFIGS[args.config]
+    if args.batch:
+        cfg = cfg.with_(B=args.batch, describe=cfg.describe + f" (batch cut to {args.batch})")
     import head_latent_attention_10_b200 as M
     st = Step(cfg, local, flags=(M.MLA_FORCE_SIMPLE if args.simple else 0))
     E = torch.cuda.Event
@@ -268,7 +270,8 @@ def run_ours(args):
                    "d_c": cfg.d_c, "d_r": cfg.d_r, "d_h": cfg.d_h, "block_size": cfg.block_size,
                    "parallelism": f"replicas x{world} (independent sequences, no collective)",
                    "l2": "inputs larger than L2 (%.0f MB of cache read per step)" % (rows * 1152 / 1e6),
-                   "decode_path": "simple" if args.simple else "default"},
+                   "decode_path": "simple" if args.simple else "default",
+                   "decode_ctas": M.mla_decode_ctas(st.dims, cfg.s)},
         "decode": {"ms": dec_ms, "cache_gbs": rows * 1152 / dec_s / 1e9, "bytes": byts,
                    "gbs": byts / dec_s / 1e9, "flops": flops, "tflops": flops / dec_s / 1e12,
                    "roofline_us": max(hbm_t, tc_t) * 1e6,
@@ -354,6 +357,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="v2", choices=sorted(W.CONFIGS))
     ap.add_argument("--simple", action="store_true", help="force the CUDA-core decode kernel")
+    ap.add_argument("--batch", type=int, default=0, help="override the number of sequences (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

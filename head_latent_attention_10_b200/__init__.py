@@ -22,7 +22,7 @@ MLA_SYNC_CHECK, MLA_FORCE_SIMPLE = 0x1, 0x2
 
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",
-            "mla_kernel_launches")
+            "mla_kernel_launches", "mla_decode_ctas")
 
 
 class MLAError(RuntimeError):
@@ -67,10 +67,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                ctypes.c_uint32, _vp]
     lib.mla_decode_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32), _i, _vp]
     lib.mla_up_v.argtypes = [D, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]
+    lib.mla_decode_ctas.argtypes = [D, _i]
+    lib.mla_decode_ctas.restype = _i
     lib.mla_kernel_launches.argtypes = []
     lib.mla_kernel_launches.restype = ctypes.c_uint64
     for name in EXPORTED:
-        if name not in ("mla_status_string", "mla_decode_workspace_size", "mla_kernel_launches"):
+        if name not in ("mla_status_string", "mla_decode_workspace_size", "mla_kernel_launches",
+                        "mla_decode_ctas"):
             getattr(lib, name).restype = _i
     _LIB = lib
     return lib
@@ -128,6 +131,11 @@ def mla_absorb_q(d, q_nope, q_rope, q_pos, w_uk, q_abs, stream=None):
 def mla_kernel_launches() -> int:
     """Kernels the library has launched in this process."""
     return int(load_library().mla_kernel_launches())
+
+
+def mla_decode_ctas(d, s: int = 1) -> int:
+    """CTAs of the tensor-core decode's persistent grid on the current device."""
+    return int(load_library().mla_decode_ctas(ctypes.byref(d), s))
 
 
 def mla_decode_workspace_size(d, B: int, s: int, max_seq_len: int) -> int:

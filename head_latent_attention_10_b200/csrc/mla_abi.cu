@@ -68,47 +68,6 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
     return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
 }
 
-// Tensor-core decode workspace: [error word][plan][partial latents][partial lse2]
-struct TcWs {
-    size_t off_plan, off_o, off_lse, total;
-};
-
-TcWs tc_ws(int H, int T)
-{
-    TcWs w;
-    w.off_plan = kWsAlign;
-    w.off_o = align_up(w.off_plan + (size_t)(4 + T + 1) * sizeof(int32_t), kWsAlign);
-    const size_t slots = 2 * (size_t)kMaxClusters * H;
-    w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
-    w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
-    return w;
-}
-
-// Clusters of the decode kernel that fit on the device at once (cached per device).
-int decode_clusters()
-{
-    static int cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cache[dev] > 0) return cache[dev];
-    if (cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) != cudaSuccess)
-        return 0;
-    int sms = 0;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
-    cfg.dynamicSmemBytes = kDecSmem;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, (void *)tc_decode_kernel, &cfg) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        n = sms / 2;
-    }
-    if (n > kMaxClusters) n = kMaxClusters;
-    cache[dev] = n;
-    return n;
-}
-
 template <int BN, bool kBmn, class Epi>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
                            uint32_t *err, cudaStream_t st)
@@ -141,9 +100,55 @@ SimpleWs simple_ws(int H, int T, int max_seq_len)
     return w;
 }
 
+// Tensor-core decode workspace: [error word][plan][partial latents][partial lse2]
+struct TcWs {
+    size_t off_plan, off_o, off_lse, total;
+};
+
+inline int dec_groups(int H, int s) { return (s * H + kGroupRows - 1) / kGroupRows; }
+
+TcWs tc_ws(int H, int s, int B)
+{
+    TcWs w;
+    const int ranges = kMaxRanges / dec_groups(H, s) > 0 ? kMaxRanges / dec_groups(H, s) : 1;
+    w.off_plan = kWsAlign;
+    w.off_o = align_up(w.off_plan + (size_t)(4 + B + 1) * sizeof(int32_t), kWsAlign);
+    const size_t slots = 2 * (size_t)ranges * s * H;
+    w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
+    w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
+    return w;
+}
+
+// Ranges (persistent CTAs per row group) of the decode on the current device.
+int decode_ranges(int groups)
+{
+    static int sms_cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (sms_cache[dev] <= 0) {
+        if (cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) !=
+            cudaSuccess)
+            return 0;
+        int sms = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        sms_cache[dev] = sms;
+    }
+    int r = sms_cache[dev] / groups;
+    const int cap = kMaxRanges / groups;
+    if (r > cap) r = cap;
+    return r > 0 ? r : 1;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mla_decode_ctas(const mla_dims_t *dims, int s)
+{
+    if (check_dims(dims) != MLA_OK || s <= 0) return 0;
+    const int g = dec_groups(dims->num_heads, s);
+    return decode_ranges(g) * g;
+}
 
 uint64_t mla_kernel_launches(void) { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
 
@@ -240,7 +245,7 @@ size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s, int max_s
 {
     if (check_dims(dims) != MLA_OK || B < 0 || s <= 0 || max_seq_len < 0) return 0;
     const size_t a = simple_ws(dims->num_heads, B * s, max_seq_len).total;
-    const size_t b = tc_ws(dims->num_heads, B * s).total;
+    const size_t b = tc_ws(dims->num_heads, s, B).total;
     return a > b ? a : b;
 }
 
@@ -281,20 +286,19 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     } else {
-        const TcWs w = tc_ws(H, T);
+        const TcWs w = tc_ws(H, s, B);
         if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
-        const int nc = decode_clusters();
-        if (nc <= 0) return MLA_ERR_CUDA;
-        CUtensorMap mq, mqr, mkv, mkvr;
+        const int groups = dec_groups(H, s);
+        const int ranges = decode_ranges(groups);
+        if (ranges <= 0) return MLA_ERR_CUDA;
+        CUtensorMap mq, mkv;
         const uint64_t rows = (uint64_t)num_blocks * kBlock;
-        if (!tmap(&mq, q_abs, kRow, H, T, kRow, (uint64_t)H * kRow, 64, 128) ||
-            !tmap(&mqr, q_abs, kRow, H, T, kRow, (uint64_t)H * kRow, 32, 128) ||
-            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, 64) ||
-            !tmap(&mkvr, cache, kRow, rows, 1, kRow, 0, 32, 64))
+        if (!tmap(&mq, q_abs, kRow, (uint64_t)T * H, 1, kRow, 0, 64, kGroupRows) ||
+            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kTN))
             return MLA_ERR_CUDA;
         if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
         int32_t *plan = (int32_t *)(ws + w.off_plan);
-        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, nc, plan, err);
+        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, plan, err);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
         DecArgs da;
@@ -312,12 +316,14 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.num_blocks = num_blocks;
         da.s = s;
         da.H = H;
-        da.T = T;
-        tc_decode_kernel<<<2 * nc, kDecThreads, kDecSmem, strm>>>(mq, mqr, mkv, mkvr, da);
+        da.B = B;
+        da.groups = groups;
+        tc_decode_kernel<<<ranges * groups, kDecThreads, kDecSmem, strm>>>(mq, mkv, da);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-        dec_combine_kernel<<<dim3(T, H), 128, 0, strm>>>(plan, da.part_o, da.part_lse2, H, (bf16 *)out_latent,
-                                                          out_lse);
+        const int ry = s * H < 128 ? s * H : 128;
+        dec_combine_kernel<<<dim3(B, ry), 128, 0, strm>>>(plan, da.part_o, da.part_lse2, seq_lens, max_blocks, s, H,
+                                                          (bf16 *)out_latent, out_lse);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }

@@ -113,6 +113,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, and
+// __syncwarp orders the other lanes' later accesses after lane 0's acquire.
+// Every lane of the warp must call it.
+template <bool kCluster = false>
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *err,
+                                          uint64_t limit_ns)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(bar, parity, abort, err, limit_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
 // --------------------------------------------------------------------- TMA
 // Tile loads into this CTA's shared memory, completing bytes on `bar`.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y)
@@ -140,6 +154,14 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *ba
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// Bring a tile into L2 ahead of its load (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+                 "r"(z)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first()

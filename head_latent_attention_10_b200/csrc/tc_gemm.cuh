@@ -109,13 +109,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 sm100::tc_fence_after();
                 const uint32_t a = sm100::smem_u32(smem + s * S::STAGE);
                 const uint32_t b = a + S::A;
+                const uint64_t ad = sm100::desc_kmajor(a, 128, sm100::kSw128);
+                const uint64_t bd = kBmn ? sm100::desc_mnmajor_sw128(b, 8192) : sm100::desc_kmajor(b, 128, sm100::kSw128);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = sm100::desc_kmajor(a + kk * 32, 128, sm100::kSw128);
-                    const uint64_t bd = kBmn ? sm100::desc_mnmajor_sw128(b + kk * 16 * 128, 8192)
-                                             : sm100::desc_kmajor(b + kk * 32, 128, sm100::kSw128);
-                    sm100::umma_ss(tmem, ad, bd, idesc, (kb | kk) != 0);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    sm100::umma_ss(tmem, ad + (uint64_t)((kk * 32) >> 4),
+                                   bd + (uint64_t)(((kBmn ? kk * 16 * 128 : kk * 32)) >> 4), idesc, (kb | kk) != 0);
                 sm100::umma_commit(&empty[s]);
             }
             sm100::umma_commit(done);
@@ -123,7 +122,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     } else {
         // epilogue: warps 2..5 cover TMEM lane quarters 2,3,0,1
         const int q = warp & 3;
-        const bool ok = sm100::mbar_wait(done, 0, abort_flag, err, limit_ns);
+        const bool ok = sm100::warp_wait(done, 0, abort_flag, err, limit_ns);
         sm100::tc_fence_after();
         const int m = m0 + q * 32 + lane;
         if (ok) {

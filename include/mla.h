@@ -193,6 +193,13 @@ mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const v
                       void *stream);
 
 /*
+ * mla_decode_ctas -- number of CTAs (the persistent grid) the tensor-core
+ * decode launches on the current device for these dims and s query tokens
+ * per sequence, or 0 if it cannot run.  A measurement aid.
+ */
+int mla_decode_ctas(const mla_dims_t *dims, int s);
+
+/*
  * mla_kernel_launches -- number of CUDA kernels this library has launched in
  * the calling process (all devices, all entry points).  A measurement aid:
  * the difference across a region counts the library's launches in it.
