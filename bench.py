@@ -107,6 +107,27 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------ replicas (N GPUs)
+def replica_config(cfg: W.MLAConfig, rank: int) -> W.MLAConfig:
+    """Rank r times its own batch of the same shape: independent sequences,
+    drawn from a seed of its own (rank 0 keeps the single-GPU workload)."""
+    if rank == 0:
+        return cfg
+    return cfg.with_(seed=cfg.seed + 7919 * rank)
+
+
+def max_over_ranks(vals, world: int, device: str):
+    """Every rank gets the element-wise max of `vals` over all ranks (a job
+    is as slow as its slowest replica).  One collective, same on every rank."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 # -------------------------------------------------------------- our arm
 class Step:
     """Device-resident workload plus the four library calls of one step."""
@@ -182,7 +203,7 @@ def run_ours(args):
     if args.batch:
         cfg = cfg.with_(B=args.batch, describe=cfg.describe + f" (batch cut to {args.batch})")
     import head_latent_attention_10_b200 as M
-    st = Step(cfg, local, flags=(M.MLA_FORCE_SIMPLE if args.simple else 0))
+    st = Step(replica_config(cfg, rank), local, flags=(M.MLA_FORCE_SIMPLE if args.simple else 0))
     E = torch.cuda.Event
 
     def barrier():
@@ -210,10 +231,7 @@ def run_ours(args):
     clocks = clock.stop()
     ms = t0.elapsed_time(t1) / args.steps
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec]))
-    if world > 1:
-        v = torch.tensor([ms, dec_ms], device="cuda")
-        dist.all_reduce(v, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(v[0]), float(v[1])
+    ms, dec_ms = max_over_ranks([ms, dec_ms], world, "cuda")
 
     # --- end to end: pinned host inputs copied in and the output copied out
     pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else v)
@@ -240,10 +258,8 @@ def run_ours(args):
     e1.record()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e_ms, = max_over_ranks([e2e_ms], world, "cuda")
     if world > 1:
-        v = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(v, op=dist.ReduceOp.MAX)
-        e2e_ms = float(v[0])
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
