@@ -22,7 +22,7 @@ MLA_SYNC_CHECK, MLA_FORCE_SIMPLE = 0x1, 0x2
 
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",
-            "mla_kernel_launches", "mla_decode_ctas")
+            "mla_kernel_launches", "mla_decode_ctas", "mla_decode_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -65,6 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_decode_workspace_size.restype = ctypes.c_size_t
     lib.mla_decode.argtypes = [D, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _vp, _vp, _vp, ctypes.c_size_t,
                                ctypes.c_uint32, _vp]
+    lib.mla_decode_noalloc.argtypes = [D, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _vp, _vp, ctypes.c_uint32, _vp]
     lib.mla_decode_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32), _i, _vp]
     lib.mla_up_v.argtypes = [D, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]
     lib.mla_decode_ctas.argtypes = [D, _i]
@@ -151,6 +152,19 @@ def mla_decode(d, q_abs, cache, block_table, seq_lens, s, out_latent, out_lse, w
         block_table.shape[1], _ptr(seq_lens), B, s, _ptr(out_latent), _ptr(out_lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), flags, _stream(stream)),
         "mla_decode")
+
+
+MLA_NOALLOC_SCRATCH_BYTES = 40 << 20
+
+
+def mla_decode_noalloc(d, q_abs, cache, block_table, seq_lens, s, out_latent, out_lse,
+                       flags: int = 0, stream=None):
+    """mla_decode on the library's own per-device scratch array (no workspace)."""
+    B = seq_lens.shape[0]
+    _check(load_library().mla_decode_noalloc(
+        ctypes.byref(d), _ptr(q_abs), _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), B, s, _ptr(out_latent), _ptr(out_lse), flags,
+        _stream(stream)), "mla_decode_noalloc")
 
 
 def mla_decode_error(workspace, clear: bool = False, stream=None) -> int:

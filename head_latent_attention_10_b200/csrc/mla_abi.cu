@@ -139,6 +139,26 @@ int decode_ranges(int groups)
     return r > 0 ? r : 1;
 }
 
+// Decode scratch for callers that pass no workspace: one array per device,
+// its address looked up once per device.
+__device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+void *noalloc_scratch()
+{
+    static void *addr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -335,6 +355,25 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         if (host) return MLA_ERR_DEVICE;
     }
     return MLA_OK;
+}
+
+mla_status_t mla_decode_noalloc(const mla_dims_t *dims, const void *q_abs, const void *cache,
+                                int num_blocks, const int32_t *block_table, int max_blocks,
+                                const int32_t *seq_lens, int B, int s, void *out_latent, float *out_lse,
+                                uint32_t flags, void *stream)
+{
+    const mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (B < 0 || s <= 0 || num_blocks < 0 || max_blocks < 0) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    const size_t need = (flags & MLA_FORCE_SIMPLE)
+                            ? simple_ws(dims->num_heads, B * s, max_blocks * kBlock).total
+                            : tc_ws(dims->num_heads, s, B).total;
+    if (need > (size_t)MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return MLA_ERR_CUDA;
+    return mla_decode(dims, q_abs, cache, num_blocks, block_table, max_blocks, seq_lens, B, s, out_latent,
+                      out_lse, scratch, MLA_NOALLOC_SCRATCH_BYTES, flags, stream);
 }
 
 mla_status_t mla_decode_error(const void *workspace, uint32_t *err_host, int clear, void *stream)

@@ -180,6 +180,41 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
 mla_status_t mla_decode_error(const void *workspace, uint32_t *err_host, int clear, void *stream);
 
 /*
+ * mla_decode_noalloc -- the same decode as mla_decode, for a caller that
+ * cannot hand over a workspace.  The pages have no counterpart: it is a
+ * packaging of the same computation, not a step of the method.
+ *
+ * Scratch: a file-scope device array of MLA_NOALLOC_SCRATCH_BYTES inside this
+ * library, one per device.  Nothing is allocated: no cudaMalloc/cudaFree and
+ * no allocating library call.  On the first call on a device (with that
+ * device current) the library looks up the array's address with
+ * cudaGetSymbolAddress and keeps it; make that first call before any stream
+ * capture.  Nothing in the array has to start at zero: every call clears the
+ * error word and rewrites the plan and the partials it reads.
+ *
+ * Arguments, layouts and the result are those of mla_decode without
+ * `workspace` and `ws_bytes`.
+ *
+ * Errors:
+ *   - MLA_ERR_WORKSPACE if the scratch this shape needs (the size
+ *     mla_decode_workspace_size would report for the path the flags choose)
+ *     exceeds MLA_NOALLOC_SCRATCH_BYTES.  This is checked before any device
+ *     work.
+ *   - MLA_ERR_CUDA if the address lookup fails.
+ *   - Device-side errors are reported only through MLA_SYNC_CHECK, because
+ *     the scratch is not visible to the caller.
+ *
+ * Concurrency: every call on a device shares the one array.  Calls ordered on
+ * one stream are safe.  Calls that may overlap (different streams, or
+ * different host threads without ordering) race on it.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (40u << 20)
+mla_status_t mla_decode_noalloc(const mla_dims_t *dims, const void *q_abs, const void *cache,
+                                int num_blocks, const int32_t *block_table, int max_blocks,
+                                const int32_t *seq_lens, int B, int s, void *out_latent,
+                                float *out_lse, uint32_t flags, void *stream);
+
+/*
  * mla_up_v -- step a7: apply U^V (and optionally O) after the weighted sum.
  *   out_heads[t][i] = U^V_i latent[t][i]                 (bf16, fp32 accum.)
  *   out_model[t]    = sum_i O_i out_heads[t][i]          (if w_o != NULL)

@@ -112,3 +112,16 @@ def test_product_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "mla_oracle" not in text, f
+
+
+def test_every_entry_point_has_a_full_ctypes_signature(M):
+    """A missing argtypes list makes ctypes pass 64-bit pointers as C ints."""
+    import re
+    lib = M.load_library()
+    header = open(os.path.join(ROOT, "include", "mla.h")).read()
+    for name in M.EXPORTED:
+        f = getattr(lib, name)
+        assert f.argtypes is not None, name
+        decl = re.search(r"\b" + name + r"\(([^)]*)\)", header).group(1).strip()
+        nargs = 0 if decl in ("", "void") else decl.count(",") + 1
+        assert len(f.argtypes) == nargs, (name, len(f.argtypes), nargs)
