@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "k_simple.cuh"
 #include "tc_decode.cuh"
+#include "tc_decode64.cuh"
 #include "tc_gemm.cuh"
 #include "tmap.cuh"
 
@@ -107,6 +108,13 @@ struct TcWs {
 
 inline int dec_groups(int H, int s) { return (s * H + kGroupRows - 1) / kGroupRows; }
 
+// 32-token tiles with one MMA-issuing warp instead of 64-token tiles with three (comparison aid).
+bool use_tile32()
+{
+    const char *e = getenv("MLA_DECODE_TILE32");
+    return e && e[0] == '1';
+}
+
 TcWs tc_ws(int H, int s, int B)
 {
     TcWs w;
@@ -127,7 +135,9 @@ int decode_ranges(int groups)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (sms_cache[dev] <= 0) {
         if (cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(tc_decode64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kD64Smem) !=
+                cudaSuccess)
             return 0;
         int sms = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -313,15 +323,18 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         if (ranges <= 0) return MLA_ERR_CUDA;
         CUtensorMap mq, mkv;
         const uint64_t rows = (uint64_t)num_blocks * kBlock;
+        const bool t32 = use_tile32();
+        const int tile = t32 ? kTN : kT64;
         if (!tmap(&mq, q_abs, kRow, (uint64_t)T * H, 1, kRow, 0, 64, kGroupRows) ||
-            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kTN))
+            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, tile))
             return MLA_ERR_CUDA;
         if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
         int32_t *plan = (int32_t *)(ws + w.off_plan);
-        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, plan, err);
+        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, tile, plan, err);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
         DecArgs da;
+        da.q_abs = (const bf16 *)q_abs;
         da.block_table = block_table;
         da.seq_lens = seq_lens;
         da.plan = plan;
@@ -338,7 +351,10 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.H = H;
         da.B = B;
         da.groups = groups;
-        tc_decode_kernel<<<ranges * groups, kDecThreads, kDecSmem, strm>>>(mq, mkv, da);
+        if (t32)
+            tc_decode_kernel<<<ranges * groups, kDecThreads, kDecSmem, strm>>>(mq, mkv, da);
+        else
+            tc_decode64_kernel<<<ranges * groups, kD64Threads, kD64Smem, strm>>>(mq, mkv, da);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
         const int ry = s * H < 128 ? s * H : 128;

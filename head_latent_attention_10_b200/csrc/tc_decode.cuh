@@ -61,6 +61,7 @@ constexpr int kMaxRanges = 148;                // ranges per group (= CTAs / gro
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct DecArgs {
+    const bf16 *q_abs;    // [B*s][H][576]
     const int32_t *block_table;
     const int32_t *seq_lens;
     const int32_t *plan;  // [0]=tiles per range, [1]=total tiles, [2]=ranges, [4..4+B] sequence tile starts
@@ -511,12 +512,12 @@ tc_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 }
 
 // -------------------------------------------------------------------- plan
-// One CTA: 32-token tiles of every sequence (its last query sees all L
+// One CTA: `tile`-token tiles of every sequence (its last query sees all L
 // tokens), their prefix sums, and the per-range quota.
 // plan[0] = tiles per range, plan[1] = total tiles, plan[2] = ranges,
 // plan[4 + b] = first tile of sequence b (b = 0..B).
 __global__ void __launch_bounds__(1024)
-dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges,
+dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int tile,
                 int32_t *__restrict__ plan, uint32_t *err)
 {
     __shared__ int part[1024];
@@ -530,7 +531,7 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
             L = L < 0 ? 0 : max_blocks * kBlock;
         }
         if (L < s) set_error(err, MLA_DEVERR_SEQ_LEN);  // some query sees no key
-        sum += (L + kTN - 1) / kTN;
+        sum += (L + tile - 1) / tile;
     }
     part[threadIdx.x] = sum;
     __syncthreads();
@@ -545,7 +546,7 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
         plan[4 + b] = run;
         int L = seq_lens[b];
         L = L < 0 ? 0 : min(L, max_blocks * kBlock);
-        run += (L + kTN - 1) / kTN;
+        run += (L + tile - 1) / tile;
     }
     if (threadIdx.x == 1023) {
         const int total = part[1023];

@@ -1,0 +1,456 @@
+// tc_decode64.cuh -- absorbed-MLA decode on tcgen05 tensor cores (sm_100a),
+// one 64-token cache page per tile, three MMA-issuing warps.
+//
+// What it computes (DeepSeek-V2 paper review, sections 2-3): for every query
+// row (query token t of sequence b, head i), softmax_j(scale * q_abs . row_j)
+// weighted sum of the latents c^KV_j, where row_j = [c^KV_j | k^R_j] is the
+// 576-value cache row and q_abs = [(U^K_i)^T q^C | RoPE(q^R)].  U^V is applied
+// later.
+//
+// Work unit: 64 rows of one sequence (its s*H (query, head) pairs, cut in
+// groups of 64; the MMA M dimension) against 64-token tiles of its cache.
+// Why this shape on B200: a tcgen05.mma costs a fixed ~30 ns to issue from one
+// thread whatever its size up to M=128, N=128, and M=64 runs at half rate.
+// With one issuing thread the 36 K-steps of the logits MMA (K=576) made the
+// kernel issue-bound.  Here the logits are split over K between two issuing
+// warps, each into its own accumulator, and a third warp issues the P.C MMA,
+// which brings the tensor pipe to its work-bound rate.
+//
+//   S_a = Q[:, 0:288]   C[:, 0:288]^T     M=64, N=64, K=288   (warp 1)
+//   S_b = Q[:, 288:576] C[:, 288:576]^T   M=64, N=64, K=288   (warp 2)
+//   O  += P C[:, 0:512]                   M=64, N=2 x 256, K=64   (warp 3)
+//
+// TMEM (512 columns): a 64-row operand occupies one half of each 32-lane
+// quarter (row m at lane 32*(m/16) + m%16, plus 16 for the upper half):
+//   lanes 0-15:  S_a (columns 0-63) | S_b (64-127) | Q (128-415, bf16 pairs)
+//   lanes 16-31: O (columns 0-511)
+// Q is the A operand of the logits MMAs, read from TMEM; an A operand in TMEM
+// must sit in the same lanes as its accumulator, hence S and Q share a half.
+// Keeping Q out of shared memory leaves room for a 3-stage ring of 64-token
+// tiles (73,728 B each; TMA loads one 64 x 64 box per chunk from the tile's
+// page).  P of a tile (64 x 64 bf16, 128-byte swizzle, 8 KB) is written over
+// the tile's RoPE chunk, which no MMA reads once the tile's logits are done,
+// so P has one buffer per stage and is freed with the stage.  Tiles three
+// ahead are prefetched into L2, so a freed stage refills from L2.
+//
+// Softmax: warps 4-7, one per TMEM quarter.  Lanes 0-15 read a row's logits
+// (S_a + S_b) from TMEM, free the logits buffer for S(k+1) at once, and hand
+// the row's upper 32 columns to lane +16, so all 32 lanes share the exp work;
+// lanes 16-31 also own the row's O.  At the start of each sequence the softmax
+// warps write its Q rows into TMEM (after the previous sequence's output has
+// been read out).  Online softmax in the log2 domain with lazy rescaling (O
+// and l are rescaled only when the running max grows by more than 8, a factor
+// 256).  A rescale rewrites whole TMEM columns (all 32 lanes; the logits and
+// Q lanes are stored back unchanged), so it first waits for S(k+1) to land;
+// S(k+2) cannot start before the next free.
+//
+// Work split and combine are those of tc_decode.cuh (ranges of the
+// (sequence, tile) list per group; pieces cut by range ends are merged by
+// dec_combine_kernel).  Every wait is bounded; a wait that gives up sets
+// MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own copies in flight and
+// frees its TMEM.
+#pragma once
+
+#include "tc_decode.cuh"
+
+namespace mla {
+
+constexpr int kT64 = 64;                          // tokens per tile (one page)
+constexpr int kD64Stages = 3;
+constexpr int kD64Threads = 256;
+constexpr int kD64Chunk = kT64 * 128;             // one 64-column chunk of a tile (8 KB)
+constexpr int kD64Stage = 9 * kD64Chunk;          // 73728
+constexpr int kD64OffStage = 0;
+constexpr int kD64OffBar = kD64OffStage + kD64Stages * kD64Stage;  // 221184
+constexpr int kD64PChunk = 8 * kD64Chunk;         // P of a tile goes where its RoPE chunk was
+constexpr int kD64Smem = kD64OffBar + 512 + 1024;                // + alignment slack
+constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-511
+constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
+constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
+
+__global__ void __launch_bounds__(kD64Threads, 1)
+tc_decode64_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                   const DecArgs a)
+{
+    extern __shared__ uint8_t d64_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(d64_smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kD64OffBar);
+    uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
+    uint64_t *kv_empty = bars + 21;  // [3] O MMA -> TMA
+    uint64_t *q_full = bars + 4;     // softmax (Q of a new sequence in TMEM) -> S issuers
+    uint64_t *s_full = bars + 6;     // both S issuers -> softmax
+    uint64_t *s_free = bars + 8;     // softmax -> S issuers
+    uint64_t *p_full = bars + 24;    // [3] softmax -> O issuer (per stage)
+    uint64_t *o_done = bars + 11;    // [2] O issuer -> softmax (O of tile k done)
+    uint64_t *o_free = bars + 13;    // softmax (epilogue read O) -> O issuer
+    uint64_t *mma_done = bars + 14;  // the three issuers at teardown
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int group = blockIdx.x % a.groups, rng = blockIdx.x / a.groups;
+    const int32_t *seq_start = a.plan + 4;
+    const int q_per = a.plan[0], total = a.plan[1];
+    const int lo = rng * q_per, hi = min(lo + q_per, total);
+    if (lo >= hi) return;
+    const int rows_per_seq = a.s * a.H;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kD64Stages; ++i) { sm100::mbar_init(&kv_full[i], 1); sm100::mbar_init(&kv_empty[i], 1); }
+        sm100::mbar_init(q_full, 4);
+        sm100::mbar_init(s_full, 2);
+        sm100::mbar_init(s_free, 4);
+        for (int i = 0; i < 2; ++i) sm100::mbar_init(&o_done[i], 1);
+        for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&p_full[i], 4);
+        sm100::mbar_init(o_free, 4);
+        sm100::mbar_init(mma_done, 3);
+        *abort_flag = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tensormap(&map_q);
+        sm100::prefetch_tensormap(&map_kv);
+    }
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, 512);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const unsigned long long lim = a.limit_ns;
+    const unsigned long long drain = lim > 200000000ull ? lim : 200000000ull;
+    uint8_t *stages = smem + kD64OffStage;
+
+    auto page_of = [&](const TileIter &t) -> int {
+        const int blk = a.block_table[(long long)t.seq * a.max_blocks + t.tt];
+        return (blk < 0 || blk >= a.num_blocks) ? -1 : blk;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            TileIter it, ahead;
+            it.init(seq_start, a.B, lo, hi);
+            ahead = it;
+            for (int i = 0; i < kD64Ahead && ahead.ok; ++i) ahead.advance();
+            int issued_k = 0;
+            bool ok = true;
+            while (ok && it.ok) {
+                const int k = it.k, st = k % kD64Stages;
+                if (ahead.ok) {
+                    // warm L2 with a tile further ahead while this stage waits to be freed
+                    const int pb = page_of(ahead);
+                    if (pb >= 0)
+                        for (int j = 0; j < 9; ++j) sm100::tma_prefetch_3d(&map_kv, 64 * j, pb * kBlock, 0);
+                    ahead.advance();
+                }
+                if (k >= kD64Stages)
+                    ok = sm100::mbar_wait(&kv_empty[st], ((k / kD64Stages) - 1) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+                int blk = page_of(it);
+                if (blk < 0) {
+                    // never read outside the cache: load block 0 instead; the
+                    // sequence's output is then unspecified and the error bit says so
+                    set_error(a.err, MLA_DEVERR_BLOCK_ID);
+                    blk = 0;
+                }
+                uint8_t *dst = stages + st * kD64Stage;
+                sm100::mbar_arrive_expect_tx(&kv_full[st], kD64Stage);
+                for (int j = 0; j < 9; ++j)
+                    sm100::tma_load_3d(&map_kv, &kv_full[st], dst + j * kD64Chunk, 64 * j, blk * kBlock, 0);
+                issued_k = k + 1;
+                it.advance();
+            }
+            if (*abort_flag) {  // wait for the copies still in flight
+                volatile int no_abort = 0;
+                for (int kk = issued_k - kD64Stages < 0 ? 0 : issued_k - kD64Stages; kk < issued_k; ++kk)
+                    sm100::mbar_wait(&kv_full[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
+            }
+        }
+    } else if (warp == 1 || warp == 2) {
+        // --------------------------------------------- logits MMAs (K halves)
+        const int half = warp - 1;                       // 0: K steps 0-17, 1: K steps 18-35
+        const uint32_t idesc_s = sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
+        TileIter is;
+        is.init(seq_start, a.B, lo, hi);
+        bool ok = true;
+        while (ok && is.ok) {
+            const int kk = is.k, st = kk % kD64Stages;
+            if (is.first()) {
+                // a new sequence: its Q rows are written into TMEM by the softmax warps
+                ok = sm100::warp_wait(q_full, is.seg & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+            }
+            ok = sm100::warp_wait(&kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
+            if (ok && kk >= 1) ok = sm100::warp_wait(s_free, (kk - 1) & 1, abort_flag, a.err, lim);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            if (lane == 0) {
+                const uint64_t kd = sm100::desc_kmajor(sm100::smem_u32(stages + st * kD64Stage), 128, sm100::kSw128);
+                const uint32_t d = tmem + half * 64;
+#pragma unroll
+                for (int j = 0; j < 18; ++j) {
+                    const int step = 18 * half + j;              // 16-column K step
+                    const uint32_t off = (step >> 2) * kD64Chunk + (step & 3) * 32;
+                    sm100::umma_ts(d, tmem + kD64TmQ + 8 * step, kd + (uint64_t)(off >> 4), idesc_s, j > 0);
+                }
+                sm100::umma_commit(s_full);
+            }
+            __syncwarp();
+            is.advance();
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------- P.C MMAs
+        const uint32_t idesc_o = sm100::idesc_bf16(kGroupRows, 256, 0, 1);
+        TileIter io;
+        io.init(seq_start, a.B, lo, hi);
+        int nseq = 0;
+        bool ok = true;
+        while (ok && io.ok) {
+            const int k = io.k;
+            ok = sm100::warp_wait(&p_full[k % kD64Stages], (k / kD64Stages) & 1, abort_flag, a.err, lim);
+            if (ok && io.first() && io.seg > 0) ok = sm100::warp_wait(o_free, (io.seg - 1) & 1, abort_flag, a.err, lim);
+            if (!ok) break;
+            if (io.first()) nseq = seq_len_clamped(a.seq_lens, io.seq, a.max_blocks);
+            // a ragged last tile: zero the latent rows past the sequence end so
+            // that 0 * (whatever the page holds there) stays 0
+            const int valid = min(kT64, nseq - io.tt * kT64);
+            uint8_t *kvp = stages + (k % kD64Stages) * kD64Stage;
+            if (valid < kT64) {
+                for (int e = lane; e < (kT64 - valid) * 8 * 8; e += 32) {
+                    const int rr = valid + (e >> 6), j = (e >> 3) & 7, c16 = e & 7;
+                    reinterpret_cast<uint4 *>(kvp + j * kD64Chunk + rr * 128)[c16] = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            sm100::tc_fence_after();
+            if (lane == 0) {
+                const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(kvp), kD64Chunk);
+                const uint64_t pd = sm100::desc_kmajor(sm100::smem_u32(kvp + kD64PChunk), 128, sm100::kSw128);
+                const uint32_t acc0 = io.first() ? 0u : 1u;
+#pragma unroll
+                for (int kq = 0; kq < kT64 / 16; ++kq)
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh)
+                        sm100::umma_ss(tmem + kD64TmO + 256 * jh, pd + (uint64_t)((kq * 32) >> 4),
+                                       vd + (uint64_t)((4 * jh * kD64Chunk + kq * 2048) >> 4), idesc_o,
+                                       kq > 0 ? 1u : acc0);
+                sm100::umma_commit(&kv_empty[k % kD64Stages]);
+                sm100::umma_commit(&o_done[k & 1]);
+            }
+            __syncwarp();
+            io.advance();
+        }
+    } else {
+        // -------------------------------------------------------- softmax
+        // warp q (0..3) owns group rows [16q, 16q+16): lane i holds row
+        // 16q+i's logits (TMEM lane 32q+i), lane 16+i the same row's O
+        // (lane 32q+16+i)
+        const int qd = warp & 3;
+        const bool srow = lane < 16;
+        const int r = 16 * qd + (lane & 15);
+        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+        const uint32_t p_row0 = sm100::smem_u32(stages + kD64PChunk) + r * 128;
+        const int grow_row = group * kGroupRows + r;  // index among the sequence's s*H rows
+        const bool row_ok = grow_row < rows_per_seq;
+        const int tq = row_ok ? grow_row / a.H : 0;   // query token of this row
+        const int head = row_ok ? grow_row % a.H : 0;
+        TileIter it;
+        it.init(seq_start, a.B, lo, hi);
+        float m_run = -INFINITY, l_run = 0.f;
+        int nvis = 0;
+        bool ok = true;
+        while (ok && it.ok) {
+            const int k = it.k;
+            if (it.first()) {
+                m_run = -INFINITY;
+                l_run = 0.f;
+                // query tq of a sequence of length L sees positions j <= L - s + tq
+                nvis = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks) - a.s + tq + 1;
+                // the sequence's Q rows into TMEM (lanes 0-15; the O lanes 16-31
+                // of these columns are dead here: the previous sequence's output
+                // has been read and the next P.C MMA starts from zero).  Every
+                // logits MMA of the previous sequence has retired: its last
+                // logits were read above.
+                const bf16 *qrow = a.q_abs + ((long long)it.seq * rows_per_seq + (row_ok ? grow_row : 0)) * kRow;
+                const uint4 *q4 = reinterpret_cast<const uint4 *>(qrow);
+#pragma unroll
+                for (int g = 0; g < 3; ++g) {  // 3 x 96 columns, loads batched per round
+                    uint4 v[24];
+#pragma unroll
+                    for (int e = 0; e < 24; ++e) v[e] = (srow && row_ok) ? __ldg(q4 + 24 * g + e) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int j = 0; j < 6; ++j)
+                        sm100::tmem_st16(lane_base + kD64TmQ + 96 * g + 16 * j, reinterpret_cast<const uint32_t *>(v + 4 * j));
+                }
+                // warm L2 with the next sequence's row, which a range moving on will read next
+                if (srow && row_ok && it.seq + 1 < a.B) {
+                    const char *nq = reinterpret_cast<const char *>(qrow + (long long)rows_per_seq * kRow);
+#pragma unroll
+                    for (int e = 0; e < 9; ++e) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * e));
+                }
+                sm100::tmem_wait_st();
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(q_full);
+            }
+            ok = sm100::warp_wait(s_full, k & 1, abort_flag, a.err, lim);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            // raw logits of row r, columns [32h, 32h+32): lanes 0-15 read the row
+            // (S_a + S_b) from TMEM and hand the upper 32 columns to lane +16
+            float x[32];
+            {
+                uint32_t sa[64], sbv[64];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    sm100::tmem_ld16(lane_base + 16 * c, sa + 16 * c);        // lanes 0-15: S_a
+                    sm100::tmem_ld16(lane_base + 64 + 16 * c, sbv + 16 * c);  // lanes 0-15: S_b
+                }
+                sm100::tmem_wait_ld();
+                // the logits buffer may take S(k+1) now; a rescale below waits for it
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(s_free);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float lo = __uint_as_float(sa[c]) + __uint_as_float(sbv[c]);
+                    const float hi = __uint_as_float(sa[32 + c]) + __uint_as_float(sbv[32 + c]);
+                    const float up = __shfl_up_sync(0xffffffffu, hi, 16);
+                    x[c] = srow ? lo : up;
+                }
+            }
+            const int tok0 = it.tt * kT64 + (srow ? 0 : 32);
+            if (tok0 + 32 > nvis) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    if (tok0 + c >= nvis) x[c] = -INFINITY;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) mx = fmaxf(mx, fmaxf(fmaxf(x[c], x[c + 1]), fmaxf(x[c + 2], x[c + 3])));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            // online softmax, log2 domain, lazy rescale (both lanes of a row take
+            // the same decisions: they hold the same max)
+            const float mt = mx * a.scale_log2;
+            const bool grow = (mt != -INFINITY) && (m_run == -INFINITY || mt > m_run + kRescaleThreshold);
+            const bool need_rescale = grow && m_run != -INFINITY;
+            const float m_new = grow ? mt : m_run;
+            const float corr = grow ? (m_run == -INFINITY ? 0.f : ex2(m_run - m_new)) : 1.f;
+            if (__any_sync(0xffffffffu, need_rescale)) {
+                // O holds this segment's tiles up to k-1: let them retire.  The
+                // rewrite below passes over all 32 lanes of each column (the
+                // logits and Q lanes are stored back unchanged), so S(k+1) must
+                // have landed; S(k+2) waits for the next free of the buffer.
+                const int kp = k - 1;
+                ok = sm100::warp_wait(&o_done[kp & 1], (kp >> 1) & 1, abort_flag, a.err, lim);
+                if (ok && k + 1 < hi - lo) ok = sm100::warp_wait(s_full, (k + 1) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                const float f = srow ? 1.f : (need_rescale ? corr : 1.f);
+                for (int c = 0; c < 512; c += 64) {
+                    uint32_t ov[64];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sm100::tmem_ld16(lane_base + c + 16 * j, ov + 16 * j);
+                    sm100::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sm100::tmem_st16(lane_base + c + 16 * j, ov + 16 * j);
+                }
+                sm100::tmem_wait_st();
+                sm100::tc_fence_before();
+            }
+            l_run *= corr;   // this lane's share of the row sum
+            m_run = m_new;
+            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+            uint32_t pw[16];
+            float lsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float p0 = ex2(fmaf(x[2 * c], a.scale_log2, -mu));
+                const float p1 = ex2(fmaf(x[2 * c + 1], a.scale_log2, -mu));
+                pw[c] = pack_bf162(p0, p1);
+                lsum += p0 + p1;
+            }
+            l_run += lsum;
+            {
+                // P row r: 128-byte row of 64 bf16, 16-byte chunk c at c ^ (r & 7)
+                // (128-byte swizzle); lanes 0-15 write chunks 0-3, lanes 16-31 chunks 4-7
+                const int c0 = srow ? 0 : 4;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    st_shared_v4(p_row0 + (k % kD64Stages) * kD64Stage + (((c0 + c) ^ (r & 7)) << 4),
+                                 make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&p_full[k % kD64Stages]);
+            if (it.last()) {
+                // epilogue of the sequence segment: lanes 16-31 write their O rows
+                ok = sm100::warp_wait(&o_done[k & 1], (k >> 1) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+                const float m_fin = m_run;
+                const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+                const float lse2 = l_tot > 0.f ? m_fin + __log2f(l_tot) : -INFINITY;
+                const long long orow = (long long)(it.seq * a.s + tq) * a.H + head;
+                const long long slot = 2LL * rng + (it.seg == 0 ? 0 : 1);
+                const bool writer = row_ok && !srow;
+                for (int c = 0; c < 512; c += 64) {
+                    uint32_t ov[64];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sm100::tmem_ld16(lane_base + c + 16 * j, ov + 16 * j);
+                    sm100::tmem_wait_ld();
+                    if (!writer) continue;
+                    if (it.complete) {
+                        uint4 *d = reinterpret_cast<uint4 *>(a.out + orow * kDc + c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            d[e] = make_uint4(pack_bf162(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
+                                              pack_bf162(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
+                                              pack_bf162(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
+                                              pack_bf162(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
+                    } else {
+                        float4 *d4 = reinterpret_cast<float4 *>(a.part_o + (slot * rows_per_seq + grow_row) * kDc + c);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                                __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+                    }
+                }
+                if (writer) {
+                    if (it.complete) {
+                        if (a.out_lse) a.out_lse[orow] = lse2 * kLn2;
+                    } else {
+                        a.part_lse2[slot * rows_per_seq + grow_row] = lse2;
+                    }
+                }
+                sm100::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sm100::mbar_arrive(o_free);
+            }
+            it.advance();
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp >= 1 && warp <= 3) {
+        // every MMA this CTA issued retires before its TMEM is released
+        if (lane == 0) sm100::umma_commit(mma_done);
+        __syncwarp();
+    }
+    if (warp == 1) {
+        volatile int no_abort = 0;
+        sm100::warp_wait(mma_done, 0, &no_abort, a.err, drain);
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace mla
