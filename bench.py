@@ -59,6 +59,13 @@ def algorithmic(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
     return byts, flops, rows_read
 
 
+# DRAM bytes (read + write) the current decode kernel moves per cache token,
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
+# tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (167.8 MB for
+# 131,072 tokens).  Set to None whenever the decode kernel changes.
+DECODE_DRAM_BYTES_PER_TOKEN = 167.8e6 / (32 * 4096)
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle samples while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -293,7 +300,10 @@ def run_ours(args):
                    "roofline_us": max(hbm_t, tc_t) * 1e6,
                    "roofline_frac": max(hbm_t, tc_t) / dec_s},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": (DECODE_DRAM_BYTES_PER_TOKEN * rows
+                                 if (cfg.name == "v2" and not args.simple and DECODE_DRAM_BYTES_PER_TOKEN)
+                                 else None),
                      "peak_source": pk["source"] + (" burst" if bound == "tensor" else "")},
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
