@@ -69,12 +69,12 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
     return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
 }
 
-template <int BN, bool kBmn, class Epi>
+template <int BN, bool kBmn, class Epi, bool kSplitK = false>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
                            uint32_t *err, cudaStream_t st)
 {
     using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kSplitK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
@@ -169,6 +169,38 @@ void *noalloc_scratch()
     return addr[dev];
 }
 
+// Split-K partial sums of the append projection: one array per device.
+constexpr size_t kAppendScratchFloats = 4u << 20;  // 16 MB
+__device__ __align__(256) float g_append_scratch[kAppendScratchFloats];
+
+float *append_scratch()
+{
+    static void *addr[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_append_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    return static_cast<float *>(addr[dev]);
+}
+
+// K slice of the split-K append projection: the narrowest 128 * 2^j that
+// divides d_model and whose partials fit the scratch; 0 when none does (or
+// when fewer than two slices would result).
+int append_kslice(int T, int d_model)
+{
+    for (int ks = 128; ks <= d_model / 2; ks *= 2) {
+        if (d_model % ks) continue;
+        if ((size_t)(d_model / ks) * (size_t)T * kRow <= kAppendScratchFloats) return ks;
+    }
+    return 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -234,6 +266,24 @@ mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int 
         !tmap(&mb1, w_dkv, d_model, kDc, 1, d_model, 0, 64, 256) ||
         !tmap(&mb2, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
         return MLA_ERR_CUDA;
+    const int ks = append_kslice(T, d_model);
+    if (ks > 0) {
+        // few tokens, long K: split K over CTAs, sum the slices in order
+        float *scr = append_scratch();
+        if (!scr) return MLA_ERR_CUDA;
+        const int S = d_model / ks;
+        const long long zs = (long long)T * kRow;
+        if (launch_tc_gemm<256, false, TcEpiPartial, true>(ma, mb1, T, kDc, ks, S, TcEpiPartial{scr, zs, kRow, 0},
+                                                          err_word, s) != cudaSuccess ||
+            launch_tc_gemm<64, false, TcEpiPartial, true>(ma, mb2, T, kDr, ks, S, TcEpiPartial{scr, zs, kRow, kDc},
+                                                         err_word, s) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        append_finish_kernel<<<(T * (kRow / 8) + 255) / 256, 256, 0, s>>>(
+            scr, S, zs, T, seq_idx, pos, block_table, num_seqs, max_blocks, (bf16 *)cache, num_blocks,
+            rope_base(dims), err_word);
+        count_launch();
+        return cuda_status(cudaGetLastError());
+    }
     // c^KV = W^DKV h  (columns 0..511 of the row)
     TcEpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, 0,
                   rope_base(dims), err_word};
@@ -264,7 +314,7 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
         return MLA_ERR_CUDA;
     TcEpiStore e{(bf16 *)q_abs, kRow, (long long)H * kRow};
     if (launch_tc_gemm<256, true>(ma, mb, T, kDc, kDh, H, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
-    const int warps = T * H;
+    const int warps = T * ((H + kRopeHeads - 1) / kRopeHeads);
     rope_q_kernel<<<(warps + 7) / 8, 256, 0, s>>>((const bf16 *)q_rope, q_pos, T, H, (bf16 *)q_abs,
                                                   rope_base(dims));
     count_launch();

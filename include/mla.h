@@ -105,6 +105,13 @@ const char *mla_status_string(mla_status_t status);
  *   err_word     optional device uint32; bits MLA_DEVERR_* are OR-ed in for
  *                tokens whose slot is invalid (those tokens are not written)
  * d_model must be a positive multiple of 64.  T = 0 is a no-op.
+ * For few tokens (T * d_model small enough) the projection splits K over
+ * many CTAs and keeps the fp32 partial sums in a 16 MB array inside the
+ * library (one per device); the slices are summed in a fixed order, so the
+ * result is deterministic.  Calls on one stream are ordered; calls that may
+ * overlap on one device (different streams, unordered host threads) race on
+ * that array.  The first call on a device looks up its address and should
+ * precede any stream capture.
  */
 mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int d_model,
                               const void *w_dkv, const void *w_kr,

@@ -152,22 +152,25 @@ def test_append_cache_projection(lib, cfg):
     assert np.array_equal(got[mask], cache0[mask])
 
 
-def test_append_cache_identity_weights_are_bit_exact(lib):
-    """W^DKV = [I 0], W^KR = [0 I] at position 0 copies h bit for bit
-    (projection by I is exact in fp32; RoPE at 0 is the identity)."""
+@pytest.mark.parametrize("d_model", [576, 1024], ids=["one_pass", "split_k"])
+def test_append_cache_identity_weights_are_bit_exact(lib, d_model):
+    """W^DKV = [I 0], W^KR = [0 I 0] at position 0 copies the first 576
+    columns of h bit for bit (projection by I is exact in fp32, also when
+    the K sum is split over CTAs; RoPE at 0 is the identity).  576 runs the
+    GEMM in one pass over K, 1024 the split-K path."""
     import torch
-    cfg = W.MLAConfig("ident", B=2, s=1, H=16, L=0, paged=True, seed=301, d_model=576,
+    cfg = W.MLAConfig("ident", B=2, s=1, H=16, L=0, paged=True, seed=301, d_model=d_model,
                       seq_lens=(5, 70))
     g = GpuWorkload(cfg)
-    h = W.f32_to_bf16_bits(np.random.default_rng(1).standard_normal((2, 576)).astype(np.float32))
-    eye = np.eye(576, dtype=np.float32)
+    h = W.f32_to_bf16_bits(np.random.default_rng(1).standard_normal((2, d_model)).astype(np.float32))
+    eye = np.eye(576, d_model, dtype=np.float32)
     wd, wr = W.f32_to_bf16_bits(eye[:512]), W.f32_to_bf16_bits(eye[512:])
     seq = np.array([0, 1], np.int32); pos = np.array([0, 0], np.int32)
     lib.mla_append_cache(g.dims, torch_bits(h), torch_bits(wd), torch_bits(wr), i32(seq), i32(pos),
                          g.block_table, g.cache)
     got = host_bits(g.cache)
     bt = g.d["block_table"]
-    assert np.array_equal(got[bt[0, 0], 0], h[0]) and np.array_equal(got[bt[1, 0], 0], h[1])
+    assert np.array_equal(got[bt[0, 0], 0], h[0, :576]) and np.array_equal(got[bt[1, 0], 0], h[1, :576])
 
 
 def test_block_permutation_gives_bitwise_identical_outputs(lib):
