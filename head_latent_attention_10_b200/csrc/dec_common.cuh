@@ -1,0 +1,206 @@
+// dec_common.cuh -- pieces shared by the decode kernels: the argument block,
+// the walk over a range of the (sequence, tile) list, small device helpers
+// and the plan kernel that cuts the batch's tiles into equal ranges.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace mla {
+
+constexpr int kGroupRows = 64;                // rows of one work unit (the MMA M dimension)
+constexpr int kMaxRanges = 148;               // ranges per row group at most (= CTAs / groups)
+constexpr float kRescaleThreshold = 8.0f;     // lazy rescale of the running max, log2 units
+
+struct DecArgs {
+    const bf16 *q_abs;    // [B*s][H][576]
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    const int32_t *plan;  // [0]=tiles per range, [1]=total tiles, [2]=ranges, [4..4+B] sequence tile starts
+    bf16 *out;
+    float *out_lse;
+    float *part_o;        // [2*ranges][s*H][512] fp32
+    float *part_lse2;     // [2*ranges][s*H]
+    uint32_t *err;
+    unsigned long long limit_ns;
+    float scale_log2;
+    int max_blocks, num_blocks, s, H, B, groups;
+};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ int seq_len_clamped(const int32_t *seq_lens, int b, int max_blocks)
+{
+    int L = seq_lens[b];
+    return L < 0 ? 0 : min(L, max_blocks * kBlock);
+}
+
+// Largest r in [0, n] with start[r] <= x.
+__device__ __forceinline__ int find_seq(const int32_t *start, int n, int x)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Walks a range of the (sequence, tile) list one tile at a time.
+struct TileIter {
+    const int32_t *rs;
+    int n, pos, hi, r;
+    int seq, t0, t1, seg, tt, k;
+    bool complete, ok;
+    __device__ bool next_seg()
+    {
+        while (pos < hi && r < n && rs[r + 1] <= pos) ++r;
+        if (pos >= hi || r >= n) return false;
+        const int a = rs[r], e = rs[r + 1];
+        const int end = min(hi, e);
+        seq = r; t0 = pos - a; t1 = end - a;
+        complete = (pos == a) && (end == e);
+        pos = end; ++r; ++seg;
+        return true;
+    }
+    __device__ void init(const int32_t *start, int n_, int lo, int hi_)
+    {
+        rs = start; n = n_; pos = lo; hi = hi_; seg = -1; k = 0;
+        r = find_seq(rs, n, lo);
+        ok = next_seg();
+        tt = t0;
+    }
+    __device__ bool first() const { return tt == t0; }
+    __device__ bool last() const { return tt + 1 == t1; }
+    __device__ void advance()
+    {
+        ++k;
+        if (++tt >= t1) {
+            ok = next_seg();
+            tt = t0;
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// -------------------------------------------------------------------- plan
+// One CTA: `tile`-token tiles of every sequence (its last query sees all L
+// tokens), their prefix sums, and the per-range quota.
+// plan[0] = tiles per range, plan[1] = total tiles, plan[2] = ranges,
+// plan[4 + b] = first tile of sequence b (b = 0..B).
+__global__ void __launch_bounds__(1024)
+dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int tile,
+                int32_t *__restrict__ plan, uint32_t *err)
+{
+    __shared__ int part[1024];
+    const int per = (B + 1023) / 1024;
+    const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) {
+        int L = seq_lens[b];
+        if (L < 0 || L > max_blocks * kBlock) {
+            set_error(err, MLA_DEVERR_SEQ_LEN);
+            L = L < 0 ? 0 : max_blocks * kBlock;
+        }
+        if (L < s) set_error(err, MLA_DEVERR_SEQ_LEN);  // some query sees no key
+        sum += (L + tile - 1) / tile;
+    }
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+        const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+        __syncthreads();
+        part[threadIdx.x] += v;
+        __syncthreads();
+    }
+    int run = part[threadIdx.x] - sum;
+    for (int b = b0; b < b1; ++b) {
+        plan[4 + b] = run;
+        int L = seq_lens[b];
+        L = L < 0 ? 0 : min(L, max_blocks * kBlock);
+        run += (L + tile - 1) / tile;
+    }
+    if (threadIdx.x == 1023) {
+        const int total = part[1023];
+        plan[4 + B] = total;
+        plan[1] = total;
+        plan[2] = ranges;
+        plan[0] = total > 0 ? (total + ranges - 1) / ranges : 1;
+    }
+}
+
+
+// ------------------------------------------------------------------ combine
+// grid (B, row blocks): sequences cut by range ends are merged by
+// log-sum-exp; sequences one range finished are already in place; queries
+// with no visible key get a zero latent and lse = -inf.
+__global__ void __launch_bounds__(128)
+dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
+                   const float *__restrict__ part_lse2, const int32_t *__restrict__ seq_lens, int max_blocks,
+                   int s, int H, bf16 *__restrict__ out, float *__restrict__ out_lse)
+{
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const int rows = s * H;
+    const int q = plan[0];
+    const int a0 = plan[4 + b], a1 = plan[4 + b + 1];
+    int L = seq_lens[b];
+    L = L < 0 ? 0 : min(L, max_blocks * kBlock);
+    const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
+    const bool split = a1 > a0 && c0 != c1;
+    if (!split && L >= s) return;
+    for (int rr = blockIdx.y; rr < rows; rr += gridDim.y) {
+        const int t = rr / H;
+        const long long orow = (long long)b * rows + rr;
+        if (L - s + t + 1 <= 0) {
+            reinterpret_cast<uint2 *>(out + orow * kDc)[tid] = make_uint2(0, 0);
+            if (tid == 0 && out_lse) out_lse[orow] = -INFINITY;
+            continue;
+        }
+        if (!split) continue;
+        float M = -INFINITY;
+        for (int c = c0; c <= c1; ++c) {
+            const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
+            M = fmaxf(M, part_lse2[(long long)slot * rows + rr]);
+        }
+        float den = 0.f;
+        float4 acc = make_float4(0, 0, 0, 0);
+        for (int c = c0; c <= c1; ++c) {
+            const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
+            const float l2 = part_lse2[(long long)slot * rows + rr];
+            const float w = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
+            den += w;
+            const float4 v = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc)[tid];
+            acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        uint2 pk;
+        pk.x = pack_bf162(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf162(acc.z * inv, acc.w * inv);
+        reinterpret_cast<uint2 *>(out + orow * kDc)[tid] = pk;
+        if (tid == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+    }
+}
+
+
+}  // namespace mla

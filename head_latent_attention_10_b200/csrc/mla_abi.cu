@@ -8,7 +8,6 @@
 
 #include "common.cuh"
 #include "k_simple.cuh"
-#include "tc_decode.cuh"
 #include "tc_decode64.cuh"
 #include "tc_gemm.cuh"
 #include "tmap.cuh"
@@ -108,17 +107,11 @@ struct TcWs {
 
 inline int dec_groups(int H, int s) { return (s * H + kGroupRows - 1) / kGroupRows; }
 
-// 32-token tiles with one MMA-issuing warp instead of 64-token tiles with three (comparison aid).
-bool use_tile32()
-{
-    const char *e = getenv("MLA_DECODE_TILE32");
-    return e && e[0] == '1';
-}
-
 TcWs tc_ws(int H, int s, int B)
 {
     TcWs w;
-    const int ranges = kMaxRanges / dec_groups(H, s) > 0 ? kMaxRanges / dec_groups(H, s) : 1;
+    const int groups = dec_groups(H, s);
+    const int ranges = kMaxRanges / groups > 0 ? kMaxRanges / groups : 1;
     w.off_plan = kWsAlign;
     w.off_o = align_up(w.off_plan + (size_t)(4 + B + 1) * sizeof(int32_t), kWsAlign);
     const size_t slots = 2 * (size_t)ranges * s * H;
@@ -134,10 +127,8 @@ int decode_ranges(int groups)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
     if (sms_cache[dev] <= 0) {
-        if (cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(tc_decode64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kD64Smem) !=
-                cudaSuccess)
+        if (cudaFuncSetAttribute(tc_decode64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kD64Smem) !=
+            cudaSuccess)
             return 0;
         int sms = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -371,16 +362,12 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         const int groups = dec_groups(H, s);
         const int ranges = decode_ranges(groups);
         if (ranges <= 0) return MLA_ERR_CUDA;
-        CUtensorMap mq, mkv;
+        CUtensorMap mkv;
         const uint64_t rows = (uint64_t)num_blocks * kBlock;
-        const bool t32 = use_tile32();
-        const int tile = t32 ? kTN : kT64;
-        if (!tmap(&mq, q_abs, kRow, (uint64_t)T * H, 1, kRow, 0, 64, kGroupRows) ||
-            !tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, tile))
-            return MLA_ERR_CUDA;
+        if (!tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
         if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
         int32_t *plan = (int32_t *)(ws + w.off_plan);
-        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, tile, plan, err);
+        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
         DecArgs da;
@@ -401,10 +388,7 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.H = H;
         da.B = B;
         da.groups = groups;
-        if (t32)
-            tc_decode_kernel<<<ranges * groups, kDecThreads, kDecSmem, strm>>>(mq, mkv, da);
-        else
-            tc_decode64_kernel<<<ranges * groups, kD64Threads, kD64Smem, strm>>>(mq, mkv, da);
+        tc_decode64_kernel<<<ranges * groups, kD64Threads, kD64Smem, strm>>>(mkv, da);
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
         const int ry = s * H < 128 ? s * H : 128;

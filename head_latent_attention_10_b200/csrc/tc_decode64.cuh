@@ -44,14 +44,16 @@
 // Q lanes are stored back unchanged), so it first waits for S(k+1) to land;
 // S(k+2) cannot start before the next free.
 //
-// Work split and combine are those of tc_decode.cuh (ranges of the
-// (sequence, tile) list per group; pieces cut by range ends are merged by
-// dec_combine_kernel).  Every wait is bounded; a wait that gives up sets
-// MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own copies in flight and
-// frees its TMEM.
+// Work split: the (sequence, tile) list of the batch is cut into equal
+// contiguous ranges per row group (dec_plan_kernel).  A sequence a range covers
+// completely is normalized and written straight to the output.  A sequence cut
+// by range ends leaves one fp32 partial per piece (normalized, with its
+// log2-sum-exp), merged by dec_combine_kernel.  Every wait is bounded; a wait
+// that gives up sets MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own
+// copies in flight and frees its TMEM.
 #pragma once
 
-#include "tc_decode.cuh"
+#include "dec_common.cuh"
 
 namespace mla {
 
@@ -69,8 +71,7 @@ constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-
 constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
 
 __global__ void __launch_bounds__(kD64Threads, 1)
-tc_decode64_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-                   const DecArgs a)
+tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
 {
     extern __shared__ uint8_t d64_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(d64_smem_raw) + 1023) &
@@ -107,7 +108,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         sm100::mbar_init(mma_done, 3);
         *abort_flag = 0;
         sm100::fence_mbar_init();
-        sm100::prefetch_tensormap(&map_q);
         sm100::prefetch_tensormap(&map_kv);
     }
     if (warp == 1) {
