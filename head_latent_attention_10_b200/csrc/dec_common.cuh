@@ -22,6 +22,7 @@ struct DecArgs {
     float *part_lse2;     // [2*ranges][s*H]
     uint32_t *err;
     unsigned long long limit_ns;
+    int stall_tile;       // test hook: the page load of this tile of every range is never issued (-1: none)
     float scale_log2;
     int max_blocks, num_blocks, s, H, B, groups;
 };

@@ -59,6 +59,14 @@ unsigned long long wait_limit_ns()
     return 2000000000ull;
 }
 
+// Test hook for failure detection: MLA_DEBUG_STALL_TILE=k makes every decode
+// CTA skip the page load of its k-th tile, so that a wait runs out.
+int stall_tile()
+{
+    const char *e = getenv("MLA_DEBUG_STALL_TILE");
+    return (e && *e) ? atoi(e) : -1;
+}
+
 // A bf16 tensor map over a row-major 2-D or batched 3-D operand.
 //   rows x inner elements per batch entry, row stride and batch stride in elements.
 bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t batch, uint64_t row_stride,
@@ -381,6 +389,7 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.part_lse2 = (float *)(ws + w.off_lse);
         da.err = err;
         da.limit_ns = wait_limit_ns();
+        da.stall_tile = stall_tile();
         da.scale_log2 = scale_log2;
         da.max_blocks = max_blocks;
         da.num_blocks = num_blocks;

@@ -156,6 +156,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     blk = 0;
                 }
                 uint8_t *dst = stages + st * kD64Stage;
+                if (k == a.stall_tile) {
+                    // test hook for failure detection: this page never arrives, so the
+                    // first wait on it runs out and the CTA unwinds
+                    it.advance();
+                    continue;
+                }
                 sm100::mbar_arrive_expect_tx(&kv_full[st], kD64Stage);
                 for (int j = 0; j < 9; ++j)
                     sm100::tma_load_3d(&map_kv, &kv_full[st], dst + j * kD64Chunk, 64 * j, blk * kBlock, 0);
@@ -165,7 +171,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             if (*abort_flag) {  // wait for the copies still in flight
                 volatile int no_abort = 0;
                 for (int kk = issued_k - kD64Stages < 0 ? 0 : issued_k - kD64Stages; kk < issued_k; ++kk)
-                    sm100::mbar_wait(&kv_full[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
+                    if (kk != a.stall_tile)
+                        sm100::mbar_wait(&kv_full[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
             }
         }
     } else if (warp == 1 || warp == 2) {
