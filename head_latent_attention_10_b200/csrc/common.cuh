@@ -29,7 +29,6 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits)
 }
 
 __device__ __forceinline__ float bf2f(bf16 v) { return __bfloat162float(v); }
-__device__ __forceinline__ bf16 f2bf(float v) { return __float2bfloat16_rn(v); }
 
 // RoPE of one pair (x0, x1) = (x[2k], x[2k+1]) at position pos: turn by
 // pos * base^(-2k/d_r).  The angle is formed in double precision: at

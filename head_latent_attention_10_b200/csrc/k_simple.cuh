@@ -1,7 +1,7 @@
-// k_simple.cuh -- CUDA-core kernels: the cache writers, a small tiled GEMM
-// used by the projections, and a straightforward split-KV decode with its
-// log-sum-exp combine.  The decode here is the cross-check for the
-// tensor-core kernels and the path for shapes they do not cover.
+// k_simple.cuh -- CUDA-core kernels: the cache writers (from latents, and the
+// split-K finish of the append projection), the query RoPE, and a
+// straightforward split-KV decode with its log-sum-exp combine
+// (MLA_FORCE_SIMPLE), a cross-check for the tensor-core decode.
 #pragma once
 
 #include "common.cuh"
@@ -128,111 +128,6 @@ rope_q_kernel(const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos
         }
         reinterpret_cast<__nv_bfloat162 *>(q_abs + row * kRow + kDc)[lane] = y;
     }
-}
-
-// ---------------------------------------------------------------- tiled GEMM
-// C[z][m][n] = sum_k A[z][m][k] * B[z][k][n] with arbitrary element strides,
-// fp32 accumulation; a 64x64 tile per CTA, 4x4 outputs per thread, handed to
-// the epilogue four consecutive columns at a time (N is a multiple of 4).
-struct GemmArgs {
-    int M, N, K;
-    const bf16 *A;
-    long long a_bs, a_rs, a_cs;  // batch, m, k strides
-    const bf16 *B;
-    long long b_bs, b_rs, b_cs;  // batch, k, n strides
-};
-
-template <class Epi>
-__global__ void __launch_bounds__(256) gemm_simple_kernel(GemmArgs g, Epi epi)
-{
-    __shared__ float As[32][65];
-    __shared__ float Bs[32][65];
-    const int z = blockIdx.z, m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const bf16 *A = g.A + z * g.a_bs;
-    const bf16 *B = g.B + z * g.b_bs;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < g.K; k0 += 32) {
-        for (int e = threadIdx.x; e < 64 * 32; e += 256) {
-            const int mm = e >> 5, kk = e & 31;
-            const int m = m0 + mm, k = k0 + kk;
-            As[kk][mm] = (m < g.M && k < g.K) ? bf2f(A[m * g.a_rs + k * g.a_cs]) : 0.f;
-        }
-        for (int e = threadIdx.x; e < 64 * 32; e += 256) {
-            const int kk = e >> 6, nn = e & 63;
-            const int k = k0 + kk, n = n0 + nn;
-            Bs[kk][nn] = (k < g.K && n < g.N) ? bf2f(B[k * g.b_rs + n * g.b_cs]) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < 32; ++kk) {
-            float a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-    const int n = n0 + tx * 4;
-    if (n >= g.N) return;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int m = m0 + ty * 4 + i;
-        if (m < g.M) epi(z, m, n, acc[i]);
-    }
-}
-
-// Store four bf16 values at base + z*bs + m*rs + n.
-struct EpiStoreBf16 {
-    bf16 *base;
-    long long bs, rs;
-    __device__ void operator()(int z, int m, int n, const float *v) const
-    {
-        bf16 *p = base + z * bs + m * rs + n;
-        reinterpret_cast<__nv_bfloat162 *>(p)[0] = __floats2bfloat162_rn(v[0], v[1]);
-        reinterpret_cast<__nv_bfloat162 *>(p)[1] = __floats2bfloat162_rn(v[2], v[3]);
-    }
-};
-
-// Append epilogue: column n of the projection of token m goes to its cache
-// slot; RoPE pairs are turned first when `rope` is set (columns are then the
-// 64 RoPE dims, written after the 512 latent dims).
-struct EpiAppend {
-    bf16 *cache;
-    const int32_t *seq_idx, *pos, *block_table;
-    int num_seqs, max_blocks, num_blocks, col0;
-    bool rope;
-    double base;
-    uint32_t *err;
-    __device__ void operator()(int, int m, int n, const float *v) const
-    {
-        const int p = pos[m];
-        const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks, seq_idx[m],
-                                          p, n == 0 ? err : nullptr);
-        if (slot < 0) return;
-        float o[4] = {v[0], v[1], v[2], v[3]};
-        if (rope) {
-            rope_pair(v[0], v[1], p, n / 2, kDr, base, &o[0], &o[1]);
-            rope_pair(v[2], v[3], p, n / 2 + 1, kDr, base, &o[2], &o[3]);
-        }
-        bf16 *dst = cache + slot * kRow + col0 + n;
-        reinterpret_cast<__nv_bfloat162 *>(dst)[0] = __floats2bfloat162_rn(o[0], o[1]);
-        reinterpret_cast<__nv_bfloat162 *>(dst)[1] = __floats2bfloat162_rn(o[2], o[3]);
-    }
-};
-
-template <class Epi>
-static cudaError_t launch_gemm_simple(const GemmArgs &g, int batch, const Epi &epi, cudaStream_t st)
-{
-    dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, batch);
-    gemm_simple_kernel<Epi><<<grid, 256, 0, st>>>(g, epi);
-    count_launch();
-    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------- simple decode

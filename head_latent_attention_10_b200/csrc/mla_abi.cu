@@ -82,8 +82,17 @@ cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, in
 {
     using S = GemmSmem<BN>;
     auto kern = tc_gemm_kernel<BN, kBmn, Epi, kSplitK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+    // the shared-memory opt-in once per device, so that later launches can be
+    // captured into a graph
+    static bool attr_set[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
     dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
     kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, wait_limit_ns());
     count_launch();

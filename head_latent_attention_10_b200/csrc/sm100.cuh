@@ -1,7 +1,7 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features
-// the kernels use: mbarriers with time-bounded waits, TMA tile loads,
-// tcgen05 tensor-memory allocation / MMA / loads / stores, UMMA shared-memory
-// and instruction descriptors, and cluster (DSMEM) helpers.
+// the kernels use: mbarriers with time-bounded waits, TMA tile loads and L2
+// prefetches, tcgen05 tensor-memory allocation / MMA / loads / stores, and
+// UMMA shared-memory and instruction descriptors.
 //
 // Every wait here is bounded by wall-clock time (%globaltimer); a wait that
 // gives up raises MLA_DEVERR_TIMEOUT in the caller's error word and reports
@@ -27,8 +27,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
 __device__ __forceinline__ bool elect_one()
 {
@@ -76,32 +74,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar_addr, uint32_t parity)
     return ok != 0;
 }
 
-// Same, with cluster-scope acquire: for barriers a peer CTA completes.
-__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar_addr, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar_addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Bounded wait for phase `parity` of a barrier.  Gives up when *abort is set
 // (another warp already timed out) or after `limit_ns`; then ORs
 // MLA_DEVERR_TIMEOUT into *err, sets *abort and returns false.
-template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint32_t *err, uint64_t limit_ns)
 {
     const uint32_t a = smem_u32(bar);
-    if (kCluster ? mbar_test_cluster(a, parity) : mbar_test(a, parity)) return true;
+    if (mbar_test(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (kCluster ? mbar_test_cluster(a, parity) : mbar_test(a, parity)) return true;
+        if (mbar_test(a, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
@@ -116,37 +99,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, and
 // __syncwarp orders the other lanes' later accesses after lane 0's acquire.
 // Every lane of the warp must call it.
-template <bool kCluster = false>
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *err,
                                           uint64_t limit_ns)
 {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(bar, parity, abort, err, limit_ns) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, limit_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;
 }
 
 // --------------------------------------------------------------------- TMA
-// Tile loads into this CTA's shared memory, completing bytes on `bar`.
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d_hint(const CUtensorMap *map, uint64_t *bar, void *dst, int x,
-                                                 int y, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *bar, void *dst, int x, int y,
                                             int z)
 {
@@ -162,13 +125,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, i
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
                  "r"(z)
                  : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
@@ -245,12 +201,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r)
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
-{
-    tmem_ld16(taddr, r);
-    tmem_ld16(taddr + 16, r + 16);
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r)
 {
     asm volatile(
@@ -309,58 +259,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
            | ((uint32_t)b_mn_major << 16)  // B major
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16
-}
-
-// ------------------------------------------------------------------ cluster
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_id_x()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t nclusters_x()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Shared-memory address of the same variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-// 16-byte store into a peer CTA's shared memory that completes 16 bytes of
-// transaction count on the peer's barrier.
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint32_t remote_bar)
-{
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-            remote_addr),
-        "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
-        : "memory");
-}
-
-// Arrive on a barrier of a peer CTA (release at cluster scope).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
 }  // namespace sm100
