@@ -78,12 +78,11 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kD64OffBar);
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
-    uint64_t *kv_empty = bars + 21;  // [3] O MMA -> TMA
+    uint64_t *kv_empty = bars + 21;  // [3] O MMA -> TMA (and softmax: O of tile k done)
     uint64_t *q_full = bars + 4;     // softmax (Q of a new sequence in TMEM) -> S issuers
     uint64_t *s_full = bars + 6;     // both S issuers -> softmax
     uint64_t *s_free = bars + 8;     // softmax -> S issuers
     uint64_t *p_full = bars + 24;    // [3] softmax -> O issuer (per stage)
-    uint64_t *o_done = bars + 11;    // [2] O issuer -> softmax (O of tile k done)
     uint64_t *o_free = bars + 13;    // softmax (epilogue read O) -> O issuer
     uint64_t *mma_done = bars + 14;  // the three issuers at teardown
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
@@ -102,7 +101,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         sm100::mbar_init(q_full, 4);
         sm100::mbar_init(s_full, 2);
         sm100::mbar_init(s_free, 4);
-        for (int i = 0; i < 2; ++i) sm100::mbar_init(&o_done[i], 1);
         for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&p_full[i], 4);
         sm100::mbar_init(o_free, 4);
         sm100::mbar_init(mma_done, 3);
@@ -245,7 +243,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                        vd + (uint64_t)((4 * jh * kD64Chunk + kq * 2048) >> 4), idesc_o,
                                        kq > 0 ? 1u : acc0);
                 sm100::umma_commit(&kv_empty[k % kD64Stages]);
-                sm100::umma_commit(&o_done[k & 1]);
             }
             __syncwarp();
             io.advance();
@@ -352,8 +349,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 // logits and Q lanes are stored back unchanged), so S(k+1) must
                 // have landed; S(k+2) waits for the next free of the buffer.
                 const int kp = k - 1;
-                ok = sm100::warp_wait(&o_done[kp & 1], (kp >> 1) & 1, abort_flag, a.err, lim);
-                if (ok && k + 1 < hi - lo) ok = sm100::warp_wait(s_full, (k + 1) & 1, abort_flag, a.err, lim);
+                ok = sm100::warp_wait(&kv_empty[kp % kD64Stages], (kp / kD64Stages) & 1, abort_flag, a.err, lim);
+                if (ok && !it.last()) ok = sm100::warp_wait(s_full, (k + 1) & 1, abort_flag, a.err, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
                 const float f = srow ? 1.f : (need_rescale ? corr : 1.f);
@@ -397,7 +394,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             if (lane == 0) sm100::mbar_arrive(&p_full[k % kD64Stages]);
             if (it.last()) {
                 // epilogue of the sequence segment: lanes 16-31 write their O rows
-                ok = sm100::warp_wait(&o_done[k & 1], (k >> 1) & 1, abort_flag, a.err, lim);
+                ok = sm100::warp_wait(&kv_empty[k % kD64Stages], (k / kD64Stages) & 1, abort_flag, a.err, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
                 const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);

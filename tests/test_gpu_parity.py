@@ -215,6 +215,38 @@ def test_bad_block_table_entry_sets_device_error(lib):
     assert np.isfinite(W.bf16_bits_to_f32(host_bits(lat))[1]).all()
 
 
+def test_max_jump_on_the_last_tile_of_each_sequence(lib):
+    """Each sequence ends in two tokens that score far above the rest, so the
+    running max jumps (and O is rescaled) on a sequence's last tile, while
+    further sequences follow in the same CTA's range: short sequences, s*H =
+    256 rows (four row groups, so few ranges, each spanning several
+    sequences)."""
+    o = _oracle()
+    rng = np.random.default_rng(406)
+    lens = tuple(int(x) for x in rng.integers(40, 200, 64))
+    cfg = W.MLAConfig("late_max", B=64, s=2, H=128, L=0, paged=True, seed=406, d_model=5120,
+                      seq_lens=lens)
+    d = W.make_decode_inputs(cfg, with_cache_pages=False)
+    # heads share a per-sequence direction v, so one row can outscore all others
+    v = rng.standard_normal((cfg.B, 1, 1, cfg.d_c + cfg.d_r)).astype(np.float32) * 0.5
+    q = v + 0.25 * W.bf16_bits_to_f32(W.make_q_abs(cfg)).reshape(cfg.B, cfg.s, cfg.H, -1)
+    q_bits = W.f32_to_bf16_bits(q.reshape(cfg.T, cfg.H, -1))
+    sl = d["seq_lens"]
+    spike = d["tok_pos"] >= sl[d["tok_seq"]] - 2          # the last two tokens
+    d["c_kv"][spike] = W.f32_to_bf16_bits(2.0 * v[d["tok_seq"][spike], 0, 0, :cfg.d_c])
+    d["k_rope"][spike] = 0
+    d["cache"] = W.scatter_to_pages(cfg, d["block_table"], d["num_blocks"], d["tok_seq"], d["tok_pos"],
+                                    np.concatenate([d["c_kv"], d["k_rope"]], axis=1))
+    g = GpuWorkload(cfg, d=d)
+    lat, lse = g.decode(torch_bits(q_bits), flags=lib.MLA_SYNC_CHECK)
+    ref, rlse = o.decode_latent(d["cache"], d["block_table"], sl, cfg.s, o.bf16_to_f64(q_bits))
+    got = W.bf16_bits_to_f32(host_bits(lat)).reshape(ref.shape)
+    assert_parity(got, ref, what="latent")
+    np.testing.assert_allclose(lse.cpu().numpy().ravel(), rlse, atol=1e-2, rtol=0)
+    # the spike dominates: lse sits far above that of the N(0,1) rows
+    assert np.min(rlse) > 10.0
+
+
 def test_seq_len_beyond_table_and_short_rows(lib):
     import torch
     cfg = W.MLAConfig("short", B=2, s=2, H=16, L=0, paged=True, seed=405, d_model=2048, seq_lens=(1, 50))
