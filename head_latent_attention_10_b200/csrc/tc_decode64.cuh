@@ -9,23 +9,28 @@
 //
 // Work unit: 64 rows of one sequence (its s*H (query, head) pairs, cut in
 // groups of 64; the MMA M dimension) against 64-token tiles of its cache.
-// Why this shape on B200: a tcgen05.mma costs a fixed ~30 ns to issue from one
-// thread whatever its size up to M=128, N=128, and M=64 runs at half rate.
-// With one issuing thread the 36 K-steps of the logits MMA (K=576) made the
-// kernel issue-bound.  Here the logits are split over K between two issuing
-// warps, each into its own accumulator, and a third warp issues the P.C MMA,
-// which brings the tensor pipe to its work-bound rate.
+// Why this shape on B200: a tcgen05.mma costs a fixed ~34 ns to issue from one
+// thread whatever its size up to M=128, N=128, and M=64 runs at half rate, so
+// the 36 K-steps of one tile's logits take ~1.2 us to issue from one thread.
+// Two warps issue the logits of alternate tiles, each into its own buffer,
+// and a third warp issues the P.C MMAs:
 //
-//   S_a = Q[:, 0:288]   C[:, 0:288]^T     M=64, N=64, K=288   (warp 1)
-//   S_b = Q[:, 288:576] C[:, 288:576]^T   M=64, N=64, K=288   (warp 2)
-//   O  += P C[:, 0:512]                   M=64, N=2 x 256, K=64   (warp 3)
+//   S(k)  = Q C_k^T            M=64, N=64, K=576 (36 steps)   (warp 1 + (k & 1))
+//   O    += P(k) C_k[:, 0:512]  M=64, N=2 x 256, K=64          (warp 3)
+//
+// Each accumulator has a single issuer, so every sum is taken in a fixed
+// order and the output does not depend on timing.
 //
 // TMEM (512 columns): a 64-row operand occupies one half of each 32-lane
 // quarter (row m at lane 32*(m/16) + m%16, plus 16 for the upper half):
-//   lanes 0-15:  S_a (columns 0-63) | S_b (64-127) | Q (128-415, bf16 pairs)
+//   lanes 0-15:  S(even k) (columns 0-63) | S(odd k) (64-127) | Q (128-415, bf16 pairs)
 //   lanes 16-31: O (columns 0-511)
 // Q is the A operand of the logits MMAs, read from TMEM; an A operand in TMEM
 // must sit in the same lanes as its accumulator, hence S and Q share a half.
+// The softmax warps touch TMEM only with 16-lane accesses (tcgen05.ld/st
+// .16x32bx2), so the logits/Q half and the O half are used independently: a
+// rescale of O does not wait for the logits MMAs, and the next sequence's Q
+// is written while this sequence's O is still being read out.
 // Keeping Q out of shared memory leaves room for a 3-stage ring of 64-token
 // tiles (73,728 B each; TMA loads one 64 x 64 box per chunk from the tile's
 // page).  P of a tile (64 x 64 bf16, 128-byte swizzle, 8 KB) is written over
@@ -33,16 +38,11 @@
 // so P has one buffer per stage and is freed with the stage.  Tiles three
 // ahead are prefetched into L2, so a freed stage refills from L2.
 //
-// Softmax: warps 4-7, one per TMEM quarter.  Lanes 0-15 read a row's logits
-// (S_a + S_b) from TMEM, free the logits buffer for S(k+1) at once, and hand
-// the row's upper 32 columns to lane +16, so all 32 lanes share the exp work;
-// lanes 16-31 also own the row's O.  At the start of each sequence the softmax
-// warps write its Q rows into TMEM (after the previous sequence's output has
-// been read out).  Online softmax in the log2 domain with lazy rescaling (O
-// and l are rescaled only when the running max grows by more than 8, a factor
-// 256).  A rescale rewrites whole TMEM columns (all 32 lanes; the logits and
-// Q lanes are stored back unchanged), so it first waits for S(k+1) to land;
-// S(k+2) cannot start before the next free.
+// Softmax: warps 4-7, one per TMEM quarter.  Threads i and 16+i of a warp
+// share row 16q+i: each reads half of the row's 64 logits, frees the buffer
+// for S(k+2), and does half of the exp work and half of the row's epilogue.
+// Online softmax in the log2 domain with lazy rescaling (O and l are rescaled
+// only when the running max grows by more than 8, a factor 256).
 //
 // Work split: the (sequence, tile) list of the batch is cut into equal
 // contiguous ranges per row group (dec_plan_kernel).  A sequence a range covers
@@ -80,8 +80,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
     uint64_t *kv_empty = bars + 21;  // [3] O MMA -> TMA (and softmax: O of tile k done)
     uint64_t *q_full = bars + 4;     // softmax (Q of a new sequence in TMEM) -> S issuers
-    uint64_t *s_full = bars + 6;     // both S issuers -> softmax
-    uint64_t *s_free = bars + 8;     // softmax -> S issuers
+    uint64_t *s_full = bars + 6;     // [2] S issuer -> softmax (logits buffer b)
+    uint64_t *s_free = bars + 8;     // [2] softmax (buffer b read) -> S issuer
     uint64_t *p_full = bars + 24;    // [3] softmax -> O issuer (per stage)
     uint64_t *o_free = bars + 13;    // softmax (epilogue read O) -> O issuer
     uint64_t *mma_done = bars + 14;  // the three issuers at teardown
@@ -99,8 +99,10 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kD64Stages; ++i) { sm100::mbar_init(&kv_full[i], 1); sm100::mbar_init(&kv_empty[i], 1); }
         sm100::mbar_init(q_full, 4);
-        sm100::mbar_init(s_full, 2);
-        sm100::mbar_init(s_free, 4);
+        for (int i = 0; i < 2; ++i) {
+            sm100::mbar_init(&s_full[i], 1);
+            sm100::mbar_init(&s_free[i], 4);
+        }
         for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&p_full[i], 4);
         sm100::mbar_init(o_free, 4);
         sm100::mbar_init(mma_done, 3);
@@ -174,33 +176,43 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             }
         }
     } else if (warp == 1 || warp == 2) {
-        // --------------------------------------------- logits MMAs (K halves)
-        const int half = warp - 1;                       // 0: K steps 0-17, 1: K steps 18-35
+        // --------------------------------------------------- logits MMAs
+        // warp 1 takes the even tiles and warp 2 the odd ones, each into its
+        // own logits buffer (columns 64b, b = k & 1), all 36 K steps
+        const int b = warp - 1;
         const uint32_t idesc_s = sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
         is.init(seq_start, a.B, lo, hi);
+        int q_seg = -1;
         bool ok = true;
         while (ok && is.ok) {
             const int kk = is.k, st = kk % kD64Stages;
-            if (is.first()) {
-                // a new sequence: its Q rows are written into TMEM by the softmax warps
-                ok = sm100::warp_wait(q_full, is.seg & 1, abort_flag, a.err, lim);
-                if (!ok) break;
+            if ((kk & 1) != b) {
+                is.advance();
+                continue;
             }
+            // the Q rows of this tile's sequence are written into TMEM by the
+            // softmax warps; q_full completes once per segment, and its phases
+            // are taken in order, including segments whose tiles all went to
+            // the other warp (a parity wait must not skip a phase)
+            while (ok && q_seg < is.seg) {
+                ++q_seg;
+                ok = sm100::warp_wait(q_full, q_seg & 1, abort_flag, a.err, lim);
+            }
+            if (!ok) break;
             ok = sm100::warp_wait(&kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
-            if (ok && kk >= 1) ok = sm100::warp_wait(s_free, (kk - 1) & 1, abort_flag, a.err, lim);
+            if (ok && kk >= 2) ok = sm100::warp_wait(&s_free[b], ((kk >> 1) - 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
             if (lane == 0) {
                 const uint64_t kd = sm100::desc_kmajor(sm100::smem_u32(stages + st * kD64Stage), 128, sm100::kSw128);
-                const uint32_t d = tmem + half * 64;
+                const uint32_t d = tmem + b * 64;
 #pragma unroll
-                for (int j = 0; j < 18; ++j) {
-                    const int step = 18 * half + j;              // 16-column K step
+                for (int step = 0; step < 36; ++step) {          // 16-column K steps
                     const uint32_t off = (step >> 2) * kD64Chunk + (step & 3) * 32;
-                    sm100::umma_ts(d, tmem + kD64TmQ + 8 * step, kd + (uint64_t)(off >> 4), idesc_s, j > 0);
+                    sm100::umma_ts(d, tmem + kD64TmQ + 8 * step, kd + (uint64_t)(off >> 4), idesc_s, step > 0);
                 }
-                sm100::umma_commit(s_full);
+                sm100::umma_commit(&s_full[b]);
             }
             __syncwarp();
             is.advance();
@@ -249,23 +261,56 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         }
     } else {
         // -------------------------------------------------------- softmax
-        // warp q (0..3) owns group rows [16q, 16q+16): lane i holds row
-        // 16q+i's logits (TMEM lane 32q+i), lane 16+i the same row's O
-        // (lane 32q+16+i)
+        // warp q (0..3) owns group rows [16q, 16q+16): row 16q+i's logits and
+        // Q sit at TMEM lane 32q+i, its O at lane 32q+16+i; threads i and 16+i
+        // each take half of the row's columns in both
         const int qd = warp & 3;
         const bool srow = lane < 16;
         const int r = 16 * qd + (lane & 15);
-        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);        // logits and Q lanes
+        const uint32_t o_base = tmem + ((uint32_t)(qd * 32 + 16) << 16);      // O lanes
         const uint32_t p_row0 = sm100::smem_u32(stages + kD64PChunk) + r * 128;
         const int grow_row = group * kGroupRows + r;  // index among the sequence's s*H rows
         const bool row_ok = grow_row < rows_per_seq;
         const int tq = row_ok ? grow_row / a.H : 0;   // query token of this row
         const int head = row_ok ? grow_row % a.H : 0;
+        // Q rows of sequence `seq` into TMEM (16-lane stores: lanes 0-15 only, so
+        // the O lanes are untouched and the previous sequence's epilogue can
+        // still be running).  Thread i and thread 16+i each hold half of row r:
+        // 32-column block j, columns 16 each.
+        auto write_q = [&](int seq) {
+            const uint4 *q4 = reinterpret_cast<const uint4 *>(
+                a.q_abs + ((long long)seq * rows_per_seq + (row_ok ? grow_row : 0)) * kRow) + (srow ? 0 : 4);
+#pragma unroll
+            for (int g = 0; g < 3; ++g) {  // 3 rounds of 3 blocks, loads batched per round
+                uint4 v[12];
+#pragma unroll
+                for (int e = 0; e < 12; ++e)
+                    v[e] = row_ok ? __ldg(q4 + 8 * (3 * g + (e >> 2)) + (e & 3)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    sm100::tmem_st16x2_16(lane_base + kD64TmQ + 32 * (3 * g + j), reinterpret_cast<const uint32_t *>(v + 4 * j));
+            }
+            // warm L2 with the following sequence's row, the next one a range moving on reads
+            if (row_ok && seq + 1 < a.B) {
+                // the row's nine 128-byte lines: five by thread i, four by thread 16+i
+                const char *nq = reinterpret_cast<const char *>(
+                    a.q_abs + ((long long)(seq + 1) * rows_per_seq + grow_row) * kRow);
+#pragma unroll
+                for (int e = 0; e < 5; ++e)
+                    if (srow || e < 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * (srow ? e : 5 + e)));
+            }
+            sm100::tmem_wait_st();
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(q_full);
+        };
         TileIter it;
         it.init(seq_start, a.B, lo, hi);
         float m_run = -INFINITY, l_run = 0.f;
         int nvis = 0;
         bool ok = true;
+        if (it.ok) write_q(it.seq);
         while (ok && it.ok) {
             const int k = it.k;
             if (it.first()) {
@@ -273,58 +318,23 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 l_run = 0.f;
                 // query tq of a sequence of length L sees positions j <= L - s + tq
                 nvis = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks) - a.s + tq + 1;
-                // the sequence's Q rows into TMEM (lanes 0-15; the O lanes 16-31
-                // of these columns are dead here: the previous sequence's output
-                // has been read and the next P.C MMA starts from zero).  Every
-                // logits MMA of the previous sequence has retired: its last
-                // logits were read above.
-                const bf16 *qrow = a.q_abs + ((long long)it.seq * rows_per_seq + (row_ok ? grow_row : 0)) * kRow;
-                const uint4 *q4 = reinterpret_cast<const uint4 *>(qrow);
-#pragma unroll
-                for (int g = 0; g < 3; ++g) {  // 3 x 96 columns, loads batched per round
-                    uint4 v[24];
-#pragma unroll
-                    for (int e = 0; e < 24; ++e) v[e] = (srow && row_ok) ? __ldg(q4 + 24 * g + e) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                    for (int j = 0; j < 6; ++j)
-                        sm100::tmem_st16(lane_base + kD64TmQ + 96 * g + 16 * j, reinterpret_cast<const uint32_t *>(v + 4 * j));
-                }
-                // warm L2 with the next sequence's row, which a range moving on will read next
-                if (srow && row_ok && it.seq + 1 < a.B) {
-                    const char *nq = reinterpret_cast<const char *>(qrow + (long long)rows_per_seq * kRow);
-#pragma unroll
-                    for (int e = 0; e < 9; ++e) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * e));
-                }
-                sm100::tmem_wait_st();
-                sm100::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(q_full);
             }
-            ok = sm100::warp_wait(s_full, k & 1, abort_flag, a.err, lim);
+            const int sb = k & 1;
+            ok = sm100::warp_wait(&s_full[sb], (k >> 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
-            // raw logits of row r, columns [32h, 32h+32): lanes 0-15 read the row
-            // (S_a + S_b) from TMEM and hand the upper 32 columns to lane +16
+            // raw logits of row r, columns [32h, 32h+32) (h = 0 for threads 0-15);
+            // then the buffer is handed back for S(k+2)
             float x[32];
             {
-                uint32_t sa[64], sbv[64];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    sm100::tmem_ld16(lane_base + 16 * c, sa + 16 * c);        // lanes 0-15: S_a
-                    sm100::tmem_ld16(lane_base + 64 + 16 * c, sbv + 16 * c);  // lanes 0-15: S_b
-                }
+                uint32_t sv[32];
+                sm100::tmem_ld16x2_32(lane_base + 64 * sb, sv);
                 sm100::tmem_wait_ld();
-                // the logits buffer may take S(k+1) now; a rescale below waits for it
+#pragma unroll
+                for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sv[c]);
                 sm100::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(s_free);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float lo = __uint_as_float(sa[c]) + __uint_as_float(sbv[c]);
-                    const float hi = __uint_as_float(sa[32 + c]) + __uint_as_float(sbv[32 + c]);
-                    const float up = __shfl_up_sync(0xffffffffu, hi, 16);
-                    x[c] = srow ? lo : up;
-                }
+                if (lane == 0) sm100::mbar_arrive(&s_free[sb]);
             }
             const int tok0 = it.tt * kT64 + (srow ? 0 : 32);
             if (tok0 + 32 > nvis) {
@@ -344,25 +354,21 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             const float m_new = grow ? mt : m_run;
             const float corr = grow ? (m_run == -INFINITY ? 0.f : ex2(m_run - m_new)) : 1.f;
             if (__any_sync(0xffffffffu, need_rescale)) {
-                // O holds this segment's tiles up to k-1: let them retire.  The
-                // rewrite below passes over all 32 lanes of each column (the
-                // logits and Q lanes are stored back unchanged), so S(k+1) must
-                // have landed; S(k+2) waits for the next free of the buffer.
+                // O holds this segment's tiles up to k-1: let them retire, then
+                // scale the O lanes (16-lane accesses: the logits and Q lanes,
+                // which S(k+1) may be using, are not touched)
                 const int kp = k - 1;
                 ok = sm100::warp_wait(&kv_empty[kp % kD64Stages], (kp / kD64Stages) & 1, abort_flag, a.err, lim);
-                if (ok && !it.last()) ok = sm100::warp_wait(s_full, (k + 1) & 1, abort_flag, a.err, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                const float f = srow ? 1.f : (need_rescale ? corr : 1.f);
+                const float f = need_rescale ? corr : 1.f;
                 for (int c = 0; c < 512; c += 64) {
-                    uint32_t ov[64];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) sm100::tmem_ld16(lane_base + c + 16 * j, ov + 16 * j);
+                    uint32_t ov[32];
+                    sm100::tmem_ld16x2_32(o_base + c, ov);
                     sm100::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) sm100::tmem_st16(lane_base + c + 16 * j, ov + 16 * j);
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+                    sm100::tmem_st16x2_32(o_base + c, ov);
                 }
                 sm100::tmem_wait_st();
                 sm100::tc_fence_before();
@@ -393,7 +399,13 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             __syncwarp();
             if (lane == 0) sm100::mbar_arrive(&p_full[k % kD64Stages]);
             if (it.last()) {
-                // epilogue of the sequence segment: lanes 16-31 write their O rows
+                // every logits MMA of this segment has been read: the next
+                // sequence's Q goes in now, so its logits overlap this epilogue
+                TileIter nx = it;
+                nx.advance();
+                if (nx.ok) write_q(nx.seq);
+                // epilogue of the sequence segment: threads i and 16+i write the
+                // two halves of O row r
                 ok = sm100::warp_wait(&kv_empty[k % kD64Stages], (k / kD64Stages) & 1, abort_flag, a.err, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
@@ -403,30 +415,29 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 const float lse2 = l_tot > 0.f ? m_fin + __log2f(l_tot) : -INFINITY;
                 const long long orow = (long long)(it.seq * a.s + tq) * a.H + head;
                 const long long slot = 2LL * rng + (it.seg == 0 ? 0 : 1);
-                const bool writer = row_ok && !srow;
+                const int hc = srow ? 0 : 32;
                 for (int c = 0; c < 512; c += 64) {
-                    uint32_t ov[64];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) sm100::tmem_ld16(lane_base + c + 16 * j, ov + 16 * j);
+                    uint32_t ov[32];
+                    sm100::tmem_ld16x2_32(o_base + c, ov);
                     sm100::tmem_wait_ld();
-                    if (!writer) continue;
+                    if (!row_ok) continue;
                     if (it.complete) {
-                        uint4 *d = reinterpret_cast<uint4 *>(a.out + orow * kDc + c);
+                        uint4 *d = reinterpret_cast<uint4 *>(a.out + orow * kDc + c + hc);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
+                        for (int e = 0; e < 4; ++e)
                             d[e] = make_uint4(pack_bf162(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
                                               pack_bf162(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
                                               pack_bf162(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
                                               pack_bf162(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
                     } else {
-                        float4 *d4 = reinterpret_cast<float4 *>(a.part_o + (slot * rows_per_seq + grow_row) * kDc + c);
+                        float4 *d4 = reinterpret_cast<float4 *>(a.part_o + (slot * rows_per_seq + grow_row) * kDc + c + hc);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
+                        for (int e = 0; e < 8; ++e)
                             d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
                                                 __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
                     }
                 }
-                if (writer) {
+                if (row_ok && srow) {
                     if (it.complete) {
                         if (a.out_lse) a.out_lse[orow] = lse2 * kLn2;
                     } else {
