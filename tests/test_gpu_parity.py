@@ -247,6 +247,27 @@ def test_max_jump_on_the_last_tile_of_each_sequence(lib):
     assert np.min(rlse) > 10.0
 
 
+@pytest.mark.parametrize("flags", [0, 2], ids=["default", "simple"])
+def test_empty_sequences_get_zero_rows(lib, flags):
+    """Sequences with no cache token have no tile, so no decode CTA visits
+    them: their rows must still come out as a zero latent with lse = -inf
+    (the oracle's empty softmax), between sequences that are split across
+    several CTAs."""
+    o = _oracle()
+    cfg = W.MLAConfig("empty", B=5, s=1, H=16, L=0, paged=True, seed=407, d_model=2048,
+                      seq_lens=(0, 3000, 0, 70, 0))
+    g = GpuWorkload(cfg)
+    q = W.make_q_abs(cfg)
+    lat, lse = g.decode(torch_bits(q), flags=flags)
+    ref, rlse = o.decode_latent(g.d["cache"], g.d["block_table"], g.d["seq_lens"], cfg.s, o.bf16_to_f64(q))
+    got = W.bf16_bits_to_f32(host_bits(lat)).reshape(ref.shape)
+    assert_parity(got, ref, what="latent")
+    lse = lse.cpu().numpy().ravel()
+    empty = np.repeat(np.asarray(cfg.seq_lens) == 0, cfg.H)
+    assert np.all(got[empty] == 0) and np.all(np.isneginf(lse[empty]))
+    np.testing.assert_allclose(lse[~empty], rlse[~empty], atol=1e-2, rtol=0)
+
+
 def test_seq_len_beyond_table_and_short_rows(lib):
     import torch
     cfg = W.MLAConfig("short", B=2, s=2, H=16, L=0, paged=True, seed=405, d_model=2048, seq_lens=(1, 50))
