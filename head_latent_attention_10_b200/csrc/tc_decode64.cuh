@@ -1,5 +1,5 @@
 // tc_decode64.cuh -- absorbed-MLA decode on tcgen05 tensor cores (sm_100a),
-// one 64-token cache page per tile, three MMA-issuing warps.
+// one 64-token cache page per tile, two logits-issuing warps.
 //
 // What it computes (DeepSeek-V2 paper review, sections 2-3): for every query
 // row (query token t of sequence b, head i), softmax_j(scale * q_abs . row_j)
@@ -12,14 +12,17 @@
 // Why this shape on B200: a tcgen05.mma costs a fixed ~34 ns to issue from one
 // thread whatever its size up to M=128, N=128, and M=64 runs at half rate, so
 // the 36 K-steps of one tile's logits take ~1.2 us to issue from one thread.
-// Two warps issue the logits of alternate tiles, each into its own buffer,
-// and a third warp issues the P.C MMAs:
+// Two warps issue the logits of alternate tiles, each into its own buffer;
+// the P.C MMAs of a tile are issued by the softmax warp that completes its P
+// (no hand-off to another warp):
 //
 //   S(k)  = Q C_k^T            M=64, N=64, K=576 (36 steps)   (warp 1 + (k & 1))
-//   O    += P(k) C_k[:, 0:512]  M=64, N=2 x 256, K=64          (warp 3)
+//   O    += P(k) C_k[:, 0:512]  M=64, N=2 x 256, K=64          (last softmax warp)
 //
-// Each accumulator has a single issuer, so every sum is taken in a fixed
-// order and the output does not depend on timing.
+// Each logits buffer has a single issuer and the P.C MMAs are issued in tile
+// order (each after all four warps' P, tcgen05 fences around a shared-memory
+// counter), so every sum is taken in a fixed order and the output does not
+// depend on timing.
 //
 // TMEM (512 columns): a 64-row operand occupies one half of each 32-lane
 // quarter (row m at lane 32*(m/16) + m%16, plus 16 for the upper half):
@@ -41,6 +44,8 @@
 // Softmax: warps 4-7, one per TMEM quarter.  Threads i and 16+i of a warp
 // share row 16q+i: each reads half of the row's 64 logits, frees the buffer
 // for S(k+2), and does half of the exp work and half of the row's epilogue.
+// Warp q also zeroes its quarter of a ragged tile's latent rows past the
+// sequence end.  Warp 3 has no role.
 // Online softmax in the log2 domain with lazy rescaling (O and l are rescaled
 // only when the running max grows by more than 8, a factor 256).
 //
@@ -78,13 +83,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kD64OffBar);
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
-    uint64_t *kv_empty = bars + 21;  // [3] O MMA -> TMA (and softmax: O of tile k done)
+    uint64_t *kv_empty = bars + 21;  // [3] P.C MMAs of the stage done -> TMA, softmax
     uint64_t *q_full = bars + 4;     // softmax (Q of a new sequence in TMEM) -> S issuers
     uint64_t *s_full = bars + 6;     // [2] S issuer -> softmax (logits buffer b)
     uint64_t *s_free = bars + 8;     // [2] softmax (buffer b read) -> S issuer
-    uint64_t *p_full = bars + 24;    // [3] softmax -> O issuer (per stage)
-    uint64_t *o_free = bars + 13;    // softmax (epilogue read O) -> O issuer
-    uint64_t *mma_done = bars + 14;  // the three issuers at teardown
+    int *p_cnt = reinterpret_cast<int *>(bars + 24);  // [3] softmax warps done with P of the stage
+    uint64_t *mma_done = bars + 14;  // every MMA-issuing thread at teardown
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
 
@@ -103,9 +107,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             sm100::mbar_init(&s_full[i], 1);
             sm100::mbar_init(&s_free[i], 4);
         }
-        for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&p_full[i], 4);
-        sm100::mbar_init(o_free, 4);
-        sm100::mbar_init(mma_done, 3);
+        for (int i = 0; i < kD64Stages; ++i) p_cnt[i] = 0;
+        sm100::mbar_init(mma_done, 6);
         *abort_flag = 0;
         sm100::fence_mbar_init();
         sm100::prefetch_tensormap(&map_kv);
@@ -218,47 +221,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             is.advance();
         }
     } else if (warp == 3) {
-        // ------------------------------------------------------- P.C MMAs
-        const uint32_t idesc_o = sm100::idesc_bf16(kGroupRows, 256, 0, 1);
-        TileIter io;
-        io.init(seq_start, a.B, lo, hi);
-        int nseq = 0;
-        bool ok = true;
-        while (ok && io.ok) {
-            const int k = io.k;
-            ok = sm100::warp_wait(&p_full[k % kD64Stages], (k / kD64Stages) & 1, abort_flag, a.err, lim);
-            if (ok && io.first() && io.seg > 0) ok = sm100::warp_wait(o_free, (io.seg - 1) & 1, abort_flag, a.err, lim);
-            if (!ok) break;
-            if (io.first()) nseq = seq_len_clamped(a.seq_lens, io.seq, a.max_blocks);
-            // a ragged last tile: zero the latent rows past the sequence end so
-            // that 0 * (whatever the page holds there) stays 0
-            const int valid = min(kT64, nseq - io.tt * kT64);
-            uint8_t *kvp = stages + (k % kD64Stages) * kD64Stage;
-            if (valid < kT64) {
-                for (int e = lane; e < (kT64 - valid) * 8 * 8; e += 32) {
-                    const int rr = valid + (e >> 6), j = (e >> 3) & 7, c16 = e & 7;
-                    reinterpret_cast<uint4 *>(kvp + j * kD64Chunk + rr * 128)[c16] = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            sm100::tc_fence_after();
-            if (lane == 0) {
-                const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(kvp), kD64Chunk);
-                const uint64_t pd = sm100::desc_kmajor(sm100::smem_u32(kvp + kD64PChunk), 128, sm100::kSw128);
-                const uint32_t acc0 = io.first() ? 0u : 1u;
-#pragma unroll
-                for (int kq = 0; kq < kT64 / 16; ++kq)
-#pragma unroll
-                    for (int jh = 0; jh < 2; ++jh)
-                        sm100::umma_ss(tmem + kD64TmO + 256 * jh, pd + (uint64_t)((kq * 32) >> 4),
-                                       vd + (uint64_t)((4 * jh * kD64Chunk + kq * 2048) >> 4), idesc_o,
-                                       kq > 0 ? 1u : acc0);
-                sm100::umma_commit(&kv_empty[k % kD64Stages]);
-            }
-            __syncwarp();
-            io.advance();
-        }
+        // idle: the P.C MMAs are issued by the softmax warp that finishes P last
     } else {
         // -------------------------------------------------------- softmax
         // warp q (0..3) owns group rows [16q, 16q+16): row 16q+i's logits and
@@ -308,7 +271,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         TileIter it;
         it.init(seq_start, a.B, lo, hi);
         float m_run = -INFINITY, l_run = 0.f;
-        int nvis = 0;
+        int nvis = 0, nseq = 0;
+        const uint32_t idesc_o = sm100::idesc_bf16(kGroupRows, 256, 0, 1);
         bool ok = true;
         if (it.ok) write_q(it.seq);
         while (ok && it.ok) {
@@ -317,7 +281,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 m_run = -INFINITY;
                 l_run = 0.f;
                 // query tq of a sequence of length L sees positions j <= L - s + tq
-                nvis = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks) - a.s + tq + 1;
+                nseq = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks);
+                nvis = nseq - a.s + tq + 1;
             }
             const int sb = k & 1;
             ok = sm100::warp_wait(&s_full[sb], (k >> 1) & 1, abort_flag, a.err, lim);
@@ -395,9 +360,50 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     st_shared_v4(p_row0 + (k % kD64Stages) * kD64Stage + (((c0 + c) ^ (r & 7)) << 4),
                                  make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]));
             }
+            {
+                // a ragged last tile: zero the latent rows past the sequence end so
+                // that 0 * (whatever the page holds there) stays 0 (warp q: chunks 2q, 2q+1)
+                const int valid = min(kT64, nseq - it.tt * kT64);
+                uint8_t *kvp = stages + (k % kD64Stages) * kD64Stage;
+                for (int e = lane; e < (kT64 - valid) * 16; e += 32) {
+                    const int rr = valid + (e >> 4), j = 2 * qd + ((e >> 3) & 1), c16 = e & 7;
+                    reinterpret_cast<uint4 *>(kvp + j * kD64Chunk + rr * 128)[c16] = make_uint4(0, 0, 0, 0);
+                }
+            }
             fence_proxy_async_smem();
+            sm100::tc_fence_before();
             __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&p_full[k % kD64Stages]);
+            {
+                // the warp that completes P(k) issues O += P(k) C_k (the MMAs of
+                // O are thereby issued in tile order, each after every warp's P,
+                // V zeroing and previous read of O)
+                const int st = k % kD64Stages;
+                int last = 0;
+                if (lane == 0) {
+                    sm100::tc_fence_before();
+                    __threadfence_block();
+                    last = atomicAdd(&p_cnt[st], 1) == 3;
+                    __threadfence_block();
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last && lane == 0) {
+                    atomicExch(&p_cnt[st], 0);
+                    sm100::tc_fence_after();
+                    uint8_t *kvp = stages + st * kD64Stage;
+                    const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(kvp), kD64Chunk);
+                    const uint64_t pd = sm100::desc_kmajor(sm100::smem_u32(kvp + kD64PChunk), 128, sm100::kSw128);
+                    const uint32_t acc0 = it.first() ? 0u : 1u;
+#pragma unroll
+                    for (int kq = 0; kq < kT64 / 16; ++kq)
+#pragma unroll
+                        for (int jh = 0; jh < 2; ++jh)
+                            sm100::umma_ss(tmem + kD64TmO + 256 * jh, pd + (uint64_t)((kq * 32) >> 4),
+                                           vd + (uint64_t)((4 * jh * kD64Chunk + kq * 2048) >> 4), idesc_o,
+                                           kq > 0 ? 1u : acc0);
+                    sm100::umma_commit(&kv_empty[st]);
+                }
+                __syncwarp();
+            }
             if (it.last()) {
                 // every logits MMA of this segment has been read: the next
                 // sequence's Q goes in now, so its logits overlap this epilogue
@@ -444,9 +450,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                         a.part_lse2[slot * rows_per_seq + grow_row] = lse2;
                     }
                 }
-                sm100::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(o_free);
             }
             it.advance();
         }
@@ -455,7 +459,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     // ------------------------------------------------------------ teardown
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp >= 1 && warp <= 3) {
+    if (warp == 1 || warp == 2 || warp >= 4) {
         // every MMA this CTA issued retires before its TMEM is released
         if (lane == 0) sm100::umma_commit(mma_done);
         __syncwarp();
