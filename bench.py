@@ -182,7 +182,7 @@ class Step:
         self.stream = torch.cuda.current_stream()
         torch.cuda.synchronize()
 
-    def run(self, inp=None, dec_events=None):
+    def run(self, inp=None, dec_events=None, out=None):
         M, x = self.M, (inp if inp is not None else self.dev)
         M.mla_append_cache(self.dims, x["h"], self.w_dkv, self.w_kr, x["app_seq"], x["app_pos"],
                            self.block_table, self.cache)
@@ -193,7 +193,7 @@ class Step:
                      self.lat, self.lse, self.ws, flags=self.flags)
         if dec_events is not None:
             dec_events[1].record(self.stream)
-        M.mla_up_v(self.dims, self.lat, self.w_uv, self.out)
+        M.mla_up_v(self.dims, self.lat, self.w_uv, self.out if out is None else out)
 
 
 def run_ours(args):
@@ -269,28 +269,51 @@ def run_ours(args):
         del graph
         barrier()
 
-    # --- end to end: pinned host inputs copied in and the output copied out
+    # --- end to end: pinned host inputs copied in and the output copied out,
+    # every step.  Steps are pipelined over two input and two output buffers:
+    # step i+1's inputs cross PCIe (h2d stream) while step i computes, and step
+    # i's result comes back (d2h stream) while step i+1 computes.
     pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16) if v.dtype == np.uint16 else v)
            .pin_memory() for k, v in st.host.items()}
-    out_host = torch.empty(st.out.shape, dtype=torch.bfloat16).pin_memory()
+    out_host = [torch.empty(st.out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = out_host.numel() * out_host.element_size()
-    stage = {k: torch.empty_like(v) for k, v in st.dev.items()}
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    stage = [{k: torch.empty_like(v) for k, v in st.dev.items()} for _ in range(2)]
+    out_dev = [torch.empty_like(st.out) for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [E() for _ in range(2)]
+    ev_done = [E() for _ in range(2)]
+    ev_out = [E() for _ in range(2)]
 
-    def e2e_step():
-        for k, v in pin.items():
-            dst = stage[k]
-            dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(v, non_blocking=True)
-        st.run(stage)
-        out_host.copy_(st.out, non_blocking=True)
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev_done[b])      # step i-2 has read stage[b]
+            with torch.cuda.stream(s_in):
+                for k, v in pin.items():
+                    dst = stage[b][k]
+                    dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(v, non_blocking=True)
+                ev_in[b].record(s_in)
+            comp.wait_event(ev_in[b])
+            if i >= 2:
+                comp.wait_event(ev_out[b])       # step i-2's result has left out_dev[b]
+            st.run(stage[b], out=out_dev[b])
+            ev_done[b].record(comp)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        for b in range(min(n, 2)):
+            comp.wait_event(ev_out[b])
 
-    for _ in range(args.warmup):
-        e2e_step()
+    e2e_steps(args.warmup)
+    torch.cuda.synchronize()
     barrier()
     e0, e1 = E(enable_timing=True), E(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_steps(args.steps)
     e1.record()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
