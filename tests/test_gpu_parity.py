@@ -183,6 +183,23 @@ def test_block_permutation_gives_bitwise_identical_outputs(lib):
     assert np.array_equal(a[1].cpu().numpy(), b[1].cpu().numpy())
 
 
+def test_decode_is_bit_reproducible(lib):
+    """Every accumulator has one issuing thread and the P.C MMAs run in tile
+    order, so repeated calls on the same inputs give identical bits (latent
+    and lse), including sequences split across CTAs and merged by the
+    combine."""
+    cfg = W.MLAConfig("repro", B=6, s=2, H=128, L=0, paged=True, seed=408, d_model=5120,
+                      seq_lens=(2000, 70, 1500, 1, 900, 3100))
+    g = GpuWorkload(cfg)
+    q = torch_bits(W.make_q_abs(cfg))
+    first = g.decode(q)
+    ref_lat, ref_lse = host_bits(first[0]), first[1].cpu().numpy()
+    for _ in range(4):
+        lat, lse = g.decode(q)
+        assert np.array_equal(host_bits(lat), ref_lat)
+        assert np.array_equal(lse.cpu().numpy().view(np.uint32), ref_lse.view(np.uint32))
+
+
 def test_heads_with_distinct_queries_get_distinct_outputs(lib):
     cfg = W.MLAConfig("heads", B=1, s=1, H=16, L=300, paged=True, seed=402, d_model=2048)
     g = GpuWorkload(cfg)
