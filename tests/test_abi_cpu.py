@@ -84,6 +84,53 @@ def test_argument_errors(M):
     assert lib.mla_decode_error(None, None, 0, None) == M.MLA_ERR_INVALID_ARG
 
 
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mla.h"
+
+int main(void)
+{
+    mla_dims_t d;
+    memset(&d, 0, sizeof d);
+    d.num_heads = 128; d.d_c = 512; d.d_rope = 64; d.d_head = 128; d.block_size = 64;
+    d.softmax_scale = 0.f; d.rope_base = 0.f;
+    size_t ws = mla_decode_workspace_size(&d, 128, 1, 4096);
+    /* argument errors come back before any device work */
+    mla_status_t e1 = mla_decode(NULL, NULL, NULL, 0, NULL, 0, NULL, 1, 1, NULL, NULL, NULL, 0, 0u, NULL);
+    mla_status_t e2 = mla_decode(&d, (const void *)256, (const void *)256, 1, (const int32_t *)256, 1,
+                                 (const int32_t *)256, 1, 1, (void *)256, NULL, NULL, 0, MLA_SYNC_CHECK, NULL);
+    mla_status_t e3 = mla_decode(&d, NULL, NULL, 0, NULL, 0, NULL, 0, 1, NULL, NULL, NULL, 0, 0u, NULL);
+    printf("%zu %d %d %d %s\n", ws, (int)e1, (int)e2, (int)e3, mla_status_string(MLA_ERR_WORKSPACE));
+    return 0;
+}
+"""
+
+
+def test_plain_c_caller_builds_links_and_runs(M, tmp_path):
+    """A C11 program (no C++, no torch) compiles against include/mla.h, links
+    the library and gets its argument checks without a GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(M.LIB_PATH)
+    libname = os.path.basename(M.LIB_PATH)
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), os.path.join(libdir, libname), f"-Wl,-rpath,{libdir}"],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    lib = _raw(M)
+    d = M.dims(128)
+    assert int(out[0]) == lib.mla_decode_workspace_size(ctypes.byref(d), 128, 1, 4096) > 0
+    assert [int(x) for x in out[1:4]] == [M.MLA_ERR_INVALID_ARG, M.MLA_ERR_WORKSPACE, M.MLA_OK]
+    assert len(out[4]) > 0
+
+
 def test_workspace_size_grows_with_batch(M):
     lib = _raw(M)
     d = M.dims(128)
