@@ -393,6 +393,10 @@ def cpu_baseline(cfg: W.MLAConfig, budget_s: float = 10.0):
                       f"context L={int(d['seq_lens'][0])}: {el:.2f} s, scaled to one row of all heads"}
 
 
+# seconds the whole reference run (warm-up and timed steps) is sized to take
+REFERENCE_BUDGET_S = 60.0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -400,22 +404,43 @@ def run_reference(args):
     cfg = W.CONFIGS[args.config]
     import oracle
     oracle._lib()
-    d = W.make_decode_inputs(cfg.with_(B=1), with_cache_pages=True)
-    f = oracle.bf16_to_f64
-    a = (d["cache"], d["block_table"], d["seq_lens"], cfg.s, f(d["q_nope"]), f(d["q_rope"]),
-         f(d["w_uk"]), f(d["w_uv"]))
     k = max(1, min(cfg.H, oracle.num_threads()))
-    step = lambda: oracle.decode_expanded(*a, q_pos=d["q_pos"], rows=np.zeros(k, np.int32),
-                                          heads=np.arange(k, dtype=np.int32))
+    L_full = int(W.seq_lens_of(cfg.with_(B=1))[0])
+
+    def sample_step(L):
+        # the expanded-form oracle on k heads of one query row over a context of
+        # L tokens (its cost is linear in L: K/V expansion, scores, softmax, sum)
+        d = W.make_decode_inputs(cfg.with_(B=1, L=L, seq_lens=None), with_cache_pages=True)
+        f = oracle.bf16_to_f64
+        a = (d["cache"], d["block_table"], d["seq_lens"], cfg.s, f(d["q_nope"]), f(d["q_rope"]),
+             f(d["w_uk"]), f(d["w_uv"]))
+        return lambda: oracle.decode_expanded(*a, q_pos=d["q_pos"], rows=np.zeros(k, np.int32),
+                                              heads=np.arange(k, dtype=np.int32))
+
+    # each step is sized so that the whole --warmup W --steps K run takes about
+    # REFERENCE_BUDGET_S seconds: time a short context once, then pick the
+    # context of every step's sample (a multiple of 64 tokens, at most L_full)
+    per_step = REFERENCE_BUDGET_S / max(1, args.steps + args.warmup)
+    L_cal = min(L_full, 512)
+    cal = sample_step(L_cal)
+    cal()
+    t0 = time.perf_counter()
+    cal()
+    t_cal = max(time.perf_counter() - t0, 1e-6)
+    L_s = int(min(L_full, max(64, L_cal * per_step / t_cal))) // 64 * 64
+    L_s = max(64, min(L_full, L_s))
+    step = sample_step(L_s)
     for _ in range(args.warmup):
         step()
     t = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = (time.perf_counter() - t) / args.steps
-    v = k / cfg.H / el
-    sample = (f"each step: expanded-form fp64 oracle on {k} of {cfg.H} heads of one query row at full "
-              f"context L={int(d['seq_lens'][0])}; tokens/s = rows of all heads per second")
+    # rows of all H heads at the workload's full context per second
+    v = (k / cfg.H) * (L_s / L_full) / el
+    sample = (f"each step: expanded-form fp64 oracle on {k} of {cfg.H} heads of one query row over "
+              f"{L_s} of the workload's {L_full} context tokens; tokens/s = rows of all heads at full "
+              f"context per second (cost linear in context)")
     print(json.dumps({
         "impl": "reference", "metric": "MLA decode tokens/s, latent-cache GB/s & TFLOP/s (H=128,B=128,L=4K) vs roofline",
         "value": v, "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
