@@ -6,6 +6,9 @@
 
 #include <stdlib.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "k_simple.cuh"
 #include "tc_decode64.cuh"
@@ -47,24 +50,57 @@ inline double rope_base(const mla_dims_t *d)
 
 inline mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
-// Bound of every device-side wait (ns).  MLA_DEBUG_WAIT_LIMIT_NS overrides it
-// so that tests can make a wait give up on purpose.
-unsigned long long wait_limit_ns()
+// Bound of every device-side wait (ns).  With MLA_DEBUG_STALL (a test hook
+// for failure detection) waits give up after 20 ms instead.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr unsigned long long kStallWaitLimitNs = 20000000ull;
+
+// Per-device state that is filled once, on the first call that needs it:
+// lock-free reads, filled under one mutex, so that concurrent first calls
+// from several host threads are safe.
+std::mutex g_dev_mu;
+constexpr int kMaxDevices = 64;
+
+inline int current_device()
 {
-    const char *e = getenv("MLA_DEBUG_WAIT_LIMIT_NS");
-    if (e && *e) {
-        const unsigned long long v = strtoull(e, nullptr, 10);
-        if (v > 0) return v;
-    }
-    return 2000000000ull;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
 }
 
-// Test hook for failure detection: MLA_DEBUG_STALL_TILE=k makes every decode
-// CTA skip the page load of its k-th tile, so that a wait runs out.
-int stall_tile()
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) of `kern` once per device,
+// so that later launches can be captured into a graph.
+template <class K>
+cudaError_t ensure_smem_attr(K kern, int bytes, std::atomic<bool> *done)
 {
-    const char *e = getenv("MLA_DEBUG_STALL_TILE");
-    return (e && *e) ? atoi(e) : -1;
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
+}
+
+// Device address of a file-scope __device__ array on the current device,
+// looked up once per device (host code only holds a stand-in for it).
+template <class T>
+void *symbol_address(const T &sym, std::atomic<void *> *addr)
+{
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    p = addr[dev].load(std::memory_order_relaxed);
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, sym) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    addr[dev].store(p, std::memory_order_release);
+    return p;
 }
 
 // A bf16 tensor map over a row-major 2-D or batched 3-D operand.
@@ -82,19 +118,11 @@ cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, in
 {
     using S = GemmSmem<BN>;
     auto kern = tc_gemm_kernel<BN, kBmn, Epi, kSplitK>;
-    // the shared-memory opt-in once per device, so that later launches can be
-    // captured into a graph
-    static bool attr_set[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
     dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
-    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, wait_limit_ns());
+    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, kWaitLimitNs);
     count_launch();
     return cudaGetLastError();
 }
@@ -140,18 +168,17 @@ TcWs tc_ws(int H, int s, int B)
 // Ranges (persistent CTAs per row group) of the decode on the current device.
 int decode_ranges(int groups)
 {
-    static int sms_cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (sms_cache[dev] <= 0) {
-        if (cudaFuncSetAttribute(tc_decode64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kD64Smem) !=
-            cudaSuccess)
-            return 0;
-        int sms = 0;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        sms_cache[dev] = sms;
+    static std::atomic<int> sms_cache[kMaxDevices];
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0) return 0;
+    if (ensure_smem_attr(tc_decode64_kernel, kD64Smem, attr_set) != cudaSuccess) return 0;
+    int sms = sms_cache[dev].load(std::memory_order_acquire);
+    if (sms <= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 0;
+        sms_cache[dev].store(sms, std::memory_order_release);
     }
-    int r = sms_cache[dev] / groups;
+    int r = sms / groups;
     const int cap = kMaxRanges / groups;
     if (r > cap) r = cap;
     return r > 0 ? r : 1;
@@ -163,18 +190,8 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BY
 
 void *noalloc_scratch()
 {
-    static void *addr[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
-    return addr[dev];
+    static std::atomic<void *> addr[kMaxDevices];
+    return symbol_address(g_noalloc_scratch, addr);
 }
 
 // Split-K partial sums of the append projection: one array per device.
@@ -183,18 +200,8 @@ __device__ __align__(256) float g_append_scratch[kAppendScratchFloats];
 
 float *append_scratch()
 {
-    static void *addr[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_append_scratch) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        addr[dev] = p;
-    }
-    return static_cast<float *>(addr[dev]);
+    static std::atomic<void *> addr[kMaxDevices];
+    return static_cast<float *>(symbol_address(g_append_scratch, addr));
 }
 
 // K slice of the split-K append projection: the narrowest 128 * 2^j that
@@ -346,6 +353,7 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
     if (st != MLA_OK) return st;
     if (B < 0 || s <= 0 || num_blocks < 0 || max_blocks < 0) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
+    if (num_blocks == 0 || max_blocks == 0) return MLA_ERR_INVALID_ARG;
     if (!q_abs || !cache || !block_table || !seq_lens || !out_latent) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q_abs) || !aligned16(cache) || !aligned16(out_latent)) return MLA_ERR_INVALID_ARG;
     if (!workspace) return MLA_ERR_WORKSPACE;
@@ -361,9 +369,8 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         float *po = (float *)(ws + w.off_o);
         float *pl = (float *)(ws + w.off_lse);
         dim3 grid(T, H / kSimpleHeads, w.nsplit);
-        if (cudaFuncSetAttribute(decode_simple_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSimpleSmem) != cudaSuccess)
-            return MLA_ERR_CUDA;
+        static std::atomic<bool> attr_set[kMaxDevices];
+        if (ensure_smem_attr(decode_simple_kernel, kSimpleSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
         decode_simple_kernel<<<grid, 256, kSimpleSmem, strm>>>((const bf16 *)q_abs, (const bf16 *)cache,
                                                                num_blocks, block_table, max_blocks, seq_lens, s,
                                                                H, scale_log2, po, pl, w.nsplit, err);
@@ -397,8 +404,8 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.part_o = (float *)(ws + w.off_o);
         da.part_lse2 = (float *)(ws + w.off_lse);
         da.err = err;
-        da.limit_ns = wait_limit_ns();
-        da.stall_tile = stall_tile();
+        da.limit_ns = (flags & MLA_DEBUG_STALL) ? kStallWaitLimitNs : kWaitLimitNs;
+        da.stall_tile = (flags & MLA_DEBUG_STALL) ? 0 : -1;
         da.scale_log2 = scale_log2;
         da.max_blocks = max_blocks;
         da.num_blocks = num_blocks;

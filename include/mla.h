@@ -21,8 +21,14 @@
  *   - bf16 tensors are passed as pointers to 16-bit storage (IEEE bfloat16
  *     bit patterns), row-major, contiguous, 16-byte aligned.
  *   - Every pointer is caller-owned DEVICE memory unless stated otherwise.
- *     The library allocates no device memory; scratch comes from the
- *     caller's workspace.
+ *     No call allocates device memory (no cudaMalloc, no allocating library
+ *     routine).  mla_decode keeps its scratch in the caller's workspace;
+ *     mla_absorb_q, mla_append_latent and mla_up_v need none.  Two calls use
+ *     a fixed file-scope device array inside the library instead, one per
+ *     device, held until the process exits: mla_append_cache (16 MB of
+ *     split-K partial sums) and mla_decode_noalloc (MLA_NOALLOC_SCRATCH_BYTES).
+ *     Calls of either kind that may overlap on one device race on that
+ *     array (see their notes); calls ordered on one stream are safe.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream).  Inputs are never modified,
  *     except the cache by the append calls.
@@ -74,6 +80,12 @@ typedef enum {
 #define MLA_FORCE_SIMPLE 0x2u  /* run the CUDA-core decode kernel instead of
                                   the tensor-core one (same results within
                                   rounding; used to cross-check) */
+#define MLA_DEBUG_STALL  0x100u /* test hook for failure detection: every
+                                  tensor-core decode CTA skips the page load
+                                  of its first tile and the device waits give
+                                  up after 20 ms, so the call records
+                                  MLA_DEVERR_TIMEOUT and unwinds; the output is
+                                  then unspecified.  Never set in production. */
 
 typedef struct {
     int32_t num_heads;   /* H */
@@ -170,9 +182,10 @@ size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s, int max_s
  *   workspace   device buffer of ws_bytes >= mla_decode_workspace_size();
  *               its first 4 bytes are the device error word (cleared by the
  *               call); the rest holds the split plan and partial results.
- *   flags       MLA_SYNC_CHECK, MLA_FORCE_SIMPLE.
+ *   flags       MLA_SYNC_CHECK, MLA_FORCE_SIMPLE (MLA_DEBUG_STALL: tests only).
  * Sequences are independent; calls that share a workspace must not overlap
- * on the GPU.  B = 0 is a no-op.
+ * on the GPU.  B = 0 is a no-op.  With B > 0, num_blocks and max_blocks must
+ * be at least 1 (MLA_ERR_INVALID_ARG otherwise).
  */
 mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *cache,
                         int num_blocks, const int32_t *block_table, int max_blocks,

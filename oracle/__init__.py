@@ -17,9 +17,22 @@ Sources the routines follow (page title, section):
   * DeepSeek-V3 report summary (xyznot.com), Method 1: k^R = RoPE(W^KR h),
     k_{t,i} = [k^C_{t,i}; k^R_t], only c^KV and k^R are cached.
 
-Parity status: every routine here is pinned by tests/test_oracle_pins.py
-(closed forms, invariants, brute force on tiny inputs, the pages' cache
-accounting figures); none is "parity unpinned".
+Parity status: every routine here has pins of its own in
+tests/test_oracle_pins.py, none is "parity unpinned":
+  * decode_expanded, decode_latent: brute force on tiny integer inputs, the
+    absorption identity between the two, softmax rows summing to 1, the
+    single-token, uniform-attention and one-hot closed forms, the scale guard,
+    causal masking, paging invariances;
+  * decode_latent_rows: bit-identical to decode_latent, plus the single-token
+    and uniform-attention closed forms;
+  * rope, rope_rows: the identity at position 0, closed forms for unit
+    vectors, norm preservation, relative-position invariance, and each row of
+    rope_rows equal to rope of that row;
+  * kv_project: identity weights at position 0, a NumPy matmul;
+  * absorb_q: a NumPy matmul, U^K = [I | 0] returning q^C exactly;
+  * up_v, out_proj: a NumPy matmul, U^V = [I | 0] returning the first 128
+    latent columns exactly;
+  * the cache accounting figures the review prints (section 4).
 """
 from __future__ import annotations
 
@@ -55,6 +68,10 @@ def load(path: str):
         [ctypes.c_int] * 7 + [ctypes.c_double, _u16p, ctypes.c_int, _i32p, ctypes.c_int, _i32p,
                               _f64p, ctypes.c_int, _i32p, _i32p, _f64p, _f64p])
     lib.mla_oracle_decode_latent.restype = ctypes.c_int
+    lib.mla_oracle_decode_latent_rows.argtypes = (
+        [ctypes.c_int] * 7 + [ctypes.c_double, _u16p, ctypes.c_int, _i32p, ctypes.c_int, _i32p,
+                              _f64p, ctypes.c_int, _i32p, _f64p, _f64p])
+    lib.mla_oracle_decode_latent_rows.restype = ctypes.c_int
     lib.mla_oracle_up_v.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     lib.mla_oracle_out_proj.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     return lib
@@ -201,6 +218,29 @@ def decode_latent(cache, block_table, seq_lens, s, q_abs, rows=None, heads=None,
         B, s, H, d_c, d_r, d_h, block_size, float(base), _p(cache, _u16p), num_blocks,
         _p(bt, _i32p), max_blocks, _p(sl, _i32p), _p(q_abs, _f64p), n, _p(pr, _i32p),
         _p(ph, _i32p), _p(out, _f64p), _p(lse, _f64p))
+    if rc != 0:
+        raise ValueError("block table entry out of range")
+    return out, lse
+
+
+def decode_latent_rows(cache, block_table, seq_lens, s, q_abs, rows=None, block_size=64, d_r=64, d_h=128,
+                       base=10000.0):
+    """Absorbed-form decode of every head of the given rows (all rows if None):
+    (latent [n_rows][H][d_c], lse [n_rows][H]).  The same arithmetic, in the same
+    order, as decode_latent (bit-identical results); each key's RoPE part is
+    turned once per group of 16 heads, so whole batches stay affordable."""
+    cache, bt, sl = _bits(cache), _i32(block_table), _i32(seq_lens)
+    q_abs = _f64(q_abs)
+    T, H, D = q_abs.shape
+    d_c = D - d_r
+    B = sl.shape[0]
+    num_blocks = cache.size // (block_size * D)
+    max_blocks = bt.shape[-1] if bt.ndim > 1 else bt.size // max(B, 1)
+    rr = _i32(np.arange(T) if rows is None else rows)
+    out = np.zeros((rr.size, H, d_c)); lse = np.zeros((rr.size, H))
+    rc = _lib().mla_oracle_decode_latent_rows(
+        B, s, H, d_c, d_r, d_h, block_size, float(base), _p(cache, _u16p), num_blocks, _p(bt, _i32p),
+        max_blocks, _p(sl, _i32p), _p(q_abs, _f64p), rr.size, _p(rr, _i32p), _p(out, _f64p), _p(lse, _f64p))
     if rc != 0:
         raise ValueError("block table entry out of range")
     return out, lse

@@ -326,6 +326,92 @@ int mla_oracle_decode_latent(int B, int s, int H, int d_c, int d_r, int d_h,
     return bad ? -1 : 0;
 }
 
+/* The absorbed-form decode of mla_oracle_decode_latent for every head of a
+ * list of rows: out [n_rows][H][d_c], lse [n_rows][H].  Each output takes the
+ * same arithmetic in the same order as there (per key: the dot over the
+ * latent, then over the rotated RoPE key, times the scale; then the
+ * max-subtracted softmax over j ascending and the weighted latent sum over j
+ * ascending), so the two agree bit for bit.  Only the loop nest differs: the
+ * work is split over (row, group of up to 16 heads), and each key row is
+ * widened and its RoPE part turned once per group instead of once per head,
+ * which keeps whole batches affordable.  Returns 0, or -1 if a block table
+ * entry is out of range. */
+int mla_oracle_decode_latent_rows(int B, int s, int H, int d_c, int d_r, int d_h,
+                                  int block_size, double rope_base,
+                                  const uint16_t *cache, int num_blocks,
+                                  const int32_t *block_table, int max_blocks,
+                                  const int32_t *seq_lens, const double *q_abs,
+                                  int n_rows, const int32_t *rows,
+                                  double *out, double *lse)
+{
+    const int D = d_c + d_r;
+    const double scale = 1.0 / sqrt((double)(d_h + d_r));
+    const int G = 16;
+    const int n_grp = (H + G - 1) / G;
+    int bad = 0;
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int task = 0; task < n_rows * n_grp; ++task) {
+        const int ri = task / n_grp, h0 = (task % n_grp) * G;
+        const int h1 = h0 + G < H ? h0 + G : H, nh = h1 - h0;
+        const int row = rows[ri];
+        const int b = row / s, t = row % s;
+        const int n_vis = seq_lens[b] - s + t + 1;
+        for (int h = h0; h < h1; ++h) {
+            double *o = out + ((size_t)ri * H + h) * d_c;
+            for (int m = 0; m < d_c; ++m) o[m] = 0.0;
+            lse[(size_t)ri * H + h] = -INFINITY;
+        }
+        if (n_vis <= 0) continue;
+        double *score = (double *)malloc(sizeof(double) * (size_t)nh * (size_t)n_vis);
+        double *den = (double *)malloc(sizeof(double) * (size_t)nh);
+        double *c = (double *)malloc(sizeof(double) * (size_t)d_c);
+        double *kr_raw = (double *)malloc(sizeof(double) * (size_t)d_r);
+        double *kr = (double *)malloc(sizeof(double) * (size_t)d_r);
+        for (int j = 0; j < n_vis; ++j) {
+            const uint16_t *rowp = cache_row(cache, num_blocks, block_table, max_blocks,
+                                             block_size, D, b, j);
+            if (!rowp) {
+                bad = 1;
+                for (int h = 0; h < nh; ++h) score[(size_t)h * n_vis + j] = -INFINITY;
+                continue;
+            }
+            for (int m = 0; m < d_c; ++m) c[m] = bf16_bits_to_f64(rowp[m]);
+            for (int m = 0; m < d_r; ++m) kr_raw[m] = bf16_bits_to_f64(rowp[d_c + m]);
+            mla_oracle_rope(kr_raw, d_r, (double)j, rope_base, kr);
+            for (int h = 0; h < nh; ++h) {
+                const double *q = q_abs + ((size_t)row * H + h0 + h) * D;
+                double dot = 0.0;
+                for (int m = 0; m < d_c; ++m) dot += q[m] * c[m];
+                for (int m = 0; m < d_r; ++m) dot += q[d_c + m] * kr[m];
+                score[(size_t)h * n_vis + j] = dot * scale;
+            }
+        }
+        for (int h = 0; h < nh; ++h) {
+            double *sc = score + (size_t)h * n_vis;
+            double mx = -INFINITY;
+            for (int j = 0; j < n_vis; ++j) if (sc[j] > mx) mx = sc[j];
+            double dn = 0.0;
+            for (int j = 0; j < n_vis; ++j) { sc[j] = exp(sc[j] - mx); dn += sc[j]; }
+            den[h] = dn;
+            lse[(size_t)ri * H + h0 + h] = mx + log(dn);
+        }
+        for (int j = 0; j < n_vis; ++j) {
+            const uint16_t *rowp = cache_row(cache, num_blocks, block_table, max_blocks,
+                                             block_size, D, b, j);
+            if (!rowp) continue;
+            for (int m = 0; m < d_c; ++m) c[m] = bf16_bits_to_f64(rowp[m]);
+            for (int h = 0; h < nh; ++h) {
+                const double a = score[(size_t)h * n_vis + j] / den[h];
+                double *o = out + ((size_t)ri * H + h0 + h) * d_c;
+                for (int m = 0; m < d_c; ++m) o[m] += a * c[m];
+            }
+        }
+        free(score); free(den); free(c); free(kr_raw); free(kr);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Up-projection (step a7): out_heads[t][i] = U^V_i latent[t][i]
  * latent [T][H][d_c], w_uv [H][d_h][d_c] -> out_heads [T][H][d_h]. */
 void mla_oracle_up_v(int T, int H, int d_h, int d_c, const double *latent,

@@ -172,3 +172,32 @@ def test_every_entry_point_has_a_full_ctypes_signature(M):
         decl = re.search(r"\b" + name + r"\(([^)]*)\)", header).group(1).strip()
         nargs = 0 if decl in ("", "void") else decl.count(",") + 1
         assert len(f.argtypes) == nargs, (name, len(f.argtypes), nargs)
+
+
+def test_decode_rejects_an_empty_cache_for_a_non_empty_batch(M):
+    """B > 0 with no cache block (or no block-table column) is an argument
+    error, reported before any device work."""
+    lib = _raw(M)
+    d = M.dims(128)
+    p = ctypes.c_void_p(256)
+    n0 = lib.mla_kernel_launches()
+    assert lib.mla_decode(ctypes.byref(d), p, p, 0, p, 1, p, 1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode(ctypes.byref(d), p, p, 1, p, 0, p, 1, 1, p, None, p, 1 << 30, 0, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_kernel_launches() == n0
+
+
+@pytest.mark.parametrize("H,s", [(128, 200), (128, 96), (16, 900)])
+def test_noalloc_rejects_tensor_core_shapes_beyond_its_scratch(M, H, s):
+    """The tensor-core decode keeps two fp32 partial slots of s*H latent rows
+    per range; once s*H outgrows the fixed scratch the call must fail with
+    MLA_ERR_WORKSPACE before touching the device (no launch, no CUDA call:
+    this runs without a GPU)."""
+    lib = _raw(M)
+    d = M.dims(H)
+    p = ctypes.c_void_p(256)
+    n0 = lib.mla_kernel_launches()
+    st = lib.mla_decode_noalloc(ctypes.byref(d), p, p, 1, p, 1, p, 1, s, p, None, 0, None)
+    assert st == M.MLA_ERR_WORKSPACE
+    assert lib.mla_kernel_launches() == n0
+    # the size the call refused is indeed beyond the scratch
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, s, 64) > M.MLA_NOALLOC_SCRATCH_BYTES

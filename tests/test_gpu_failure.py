@@ -1,12 +1,10 @@
 """Failure detection without a GPU fault: every wait in the decode kernel is
-bounded.  The test hook MLA_DEBUG_STALL_TILE=0 makes each CTA skip the page
-load of its first tile (a barrier that nothing completes) and
-MLA_DEBUG_WAIT_LIMIT_NS cuts the bound to 20 ms.  The kernel must record
+bounded.  The test hook flag MLA_DEBUG_STALL makes each CTA skip the page
+load of its first tile (a barrier that nothing completes) and cuts the bound
+to 20 ms.  The kernel must record
 MLA_DEVERR_TIMEOUT in the workspace error word, unwind (its copies in flight
 drained, its TMEM freed) and leave the context usable: the next call,
 without the hook, must return the right answer."""
-import os
-
 import numpy as np
 import pytest
 
@@ -25,16 +23,10 @@ def test_wait_bound_reports_timeout_and_context_survives():
     M.load_library()
     g = GpuWorkload(CFG)
     q_abs = g.absorb()
-    os.environ["MLA_DEBUG_WAIT_LIMIT_NS"] = "20000000"
-    os.environ["MLA_DEBUG_STALL_TILE"] = "0"
-    try:
-        with pytest.raises(M.MLAError) as e:
-            g.decode(q_abs, flags=M.MLA_SYNC_CHECK)
-        assert e.value.status == M.MLA_ERR_DEVICE
-        assert M.mla_decode_error(g.ws, clear=True) & M.MLA_DEVERR_TIMEOUT
-    finally:
-        del os.environ["MLA_DEBUG_WAIT_LIMIT_NS"]
-        del os.environ["MLA_DEBUG_STALL_TILE"]
+    with pytest.raises(M.MLAError) as e:
+        g.decode(q_abs, flags=M.MLA_SYNC_CHECK | M.MLA_DEBUG_STALL)
+    assert e.value.status == M.MLA_ERR_DEVICE
+    assert M.mla_decode_error(g.ws, clear=True) & M.MLA_DEVERR_TIMEOUT
     lat, _ = g.decode(q_abs, flags=M.MLA_SYNC_CHECK)
     d = g.d
     want, _ = oracle.decode_latent(d["cache"], d["block_table"], d["seq_lens"], CFG.s,

@@ -504,3 +504,87 @@ def test_planted_mistakes_are_caught(oracle_mod, tmp_path, name):
         assert caught, f"mutation {name} was not caught"
     finally:
         oracle_mod._LIB = saved
+
+
+# ------------------------------------------------- pins added for the batch forms
+def test_rope_rows_equal_rope_of_each_row_and_closed_forms(oracle_mod):
+    """rope_rows is rope applied to each row at its own position: checked row
+    by row, and against the closed form of a unit vector (pair k turns by
+    pos * 10000^(-2k/64))."""
+    rng = np.random.default_rng(21)
+    pos = np.array([0, 1, 63, 64, 4095, 131071, 7, 7], np.int32)
+    x = rng.standard_normal((pos.size, 64))
+    y = oracle_mod.rope_rows(x, pos)
+    for n in range(pos.size):
+        assert np.array_equal(y[n], oracle_mod.rope(x[n], float(pos[n])))
+    assert np.array_equal(y[0], x[0])                       # position 0: identity
+    e = np.zeros((pos.size, 64)); k = 5
+    e[:, 2 * k] = 1.0
+    ye = oracle_mod.rope_rows(e, pos)
+    ang = pos.astype(np.float64) * 10000.0 ** (-2 * k / 64)
+    np.testing.assert_allclose(ye[:, 2 * k], np.cos(ang), atol=1e-12)
+    np.testing.assert_allclose(ye[:, 2 * k + 1], np.sin(ang), atol=1e-12)
+    assert np.count_nonzero(np.delete(ye, [2 * k, 2 * k + 1], axis=1)) == 0
+
+
+def test_up_v_identity_returns_the_latent_columns_exactly(oracle_mod):
+    """U^V_i = [I_128 | 0]: o_i is the first 128 latent columns, exactly."""
+    rng = np.random.default_rng(22)
+    lat = rng.standard_normal((5, 3, 512))
+    U = np.zeros((3, 128, 512)); U[:, :, :128] = np.eye(128)
+    assert np.array_equal(oracle_mod.up_v(lat, U), lat[:, :, :128])
+    # a permutation of columns picks them out in that order
+    perm = rng.permutation(512)[:128]
+    P = np.zeros((3, 128, 512)); P[:, np.arange(128), perm] = 1.0
+    assert np.array_equal(oracle_mod.up_v(lat, P), lat[:, :, perm])
+
+
+def test_absorb_q_identity_returns_q_exactly(oracle_mod):
+    """U^K_i = [I_128 | 0]: (U^K_i)^T q^C puts q^C in the first 128 columns
+    and zeros elsewhere."""
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal((4, 2, 128)); qr = rng.standard_normal((4, 2, 64))
+    U = np.zeros((2, 128, 512)); U[:, :, :128] = np.eye(128)
+    out = oracle_mod.absorb_q(q, qr, U)
+    assert np.array_equal(out[..., :128], q)
+    assert np.all(out[..., 128:512] == 0)
+
+
+@pytest.mark.parametrize("seed,s,lens,H", [(31, 1, (130, 1, 64, 0), 16), (32, 2, (70, 2, 129), 32),
+                                           (33, 1, (200,), 20)])
+def test_decode_latent_rows_is_bit_identical_to_decode_latent(oracle_mod, seed, s, lens, H):
+    """The batch form reorders only the loops: every output is the same bits
+    as the per-pair form, for head counts that do and do not fill whole groups
+    of 16, ragged and empty rows."""
+    cfg = W.MLAConfig("rows", B=len(lens), s=s, H=H, L=0, paged=True, seed=seed, d_model=64,
+                      seq_lens=lens)
+    d = W.make_decode_inputs(cfg)
+    q = oracle_mod.bf16_to_f64(W.make_q_abs(cfg))
+    a, la = oracle_mod.decode_latent(d["cache"], d["block_table"], d["seq_lens"], s, q)
+    b, lb = oracle_mod.decode_latent_rows(d["cache"], d["block_table"], d["seq_lens"], s, q)
+    assert np.array_equal(a.reshape(b.shape), b)
+    assert np.array_equal(la.reshape(lb.shape), lb)
+    rows = np.array([cfg.T - 1, 0], np.int32)
+    c, lc = oracle_mod.decode_latent_rows(d["cache"], d["block_table"], d["seq_lens"], s, q, rows=rows)
+    assert np.array_equal(c, b[rows]) and np.array_equal(lc, lb[rows])
+
+
+def test_decode_latent_rows_closed_forms(oracle_mod):
+    """One visible key returns its latent exactly; zero queries return the
+    plain mean of the visible latents (uniform weights)."""
+    cfg = W.MLAConfig("rows1", B=2, s=1, H=17, L=1, paged=True, seed=24, d_model=64)
+    d = W.make_decode_inputs(cfg)
+    q = oracle_mod.bf16_to_f64(W.make_q_abs(cfg))
+    lat, lse = oracle_mod.decode_latent_rows(d["cache"], d["block_table"], d["seq_lens"], 1, q)
+    c0 = oracle_mod.bf16_to_f64(d["c_kv"])
+    assert np.array_equal(lat, np.repeat(c0[:, None, :], cfg.H, axis=1))
+    cfg = W.MLAConfig("rows2", B=2, s=1, H=16, L=0, paged=True, seed=25, d_model=64, seq_lens=(90, 7))
+    d = W.make_decode_inputs(cfg)
+    lat, lse = oracle_mod.decode_latent_rows(d["cache"], d["block_table"], d["seq_lens"], 1,
+                                             np.zeros((cfg.T, cfg.H, 576)))
+    c = oracle_mod.bf16_to_f64(d["c_kv"])
+    starts = np.concatenate([[0], np.cumsum(d["seq_lens"])])
+    for b in range(2):
+        mean = c[starts[b]:starts[b + 1]].mean(axis=0)
+        np.testing.assert_allclose(lat[b], np.repeat(mean[None], cfg.H, axis=0), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[b], np.log(d["seq_lens"][b]), rtol=1e-14)
