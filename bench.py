@@ -363,9 +363,80 @@ def run_ours(args):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    if not args.no_per_config and world == 1:
+        line["per_config"] = per_config(M, [n for n in ("tiny", "v2lite", "v2", "longctx", "mtp")])
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------- every config's decode
+def per_config(M, names, iters=30):
+    """The decode call (plan + decode + combine) on each named workload: its
+    CUDA-event time on the launching stream (mean of `iters` back-to-back
+    calls after 3 warm-ups), latent-cache GB/s, TFLOP/s and roofline
+    fraction.  Inputs are generated on the device (seeded torch draws with
+    the workloads' distributions: cache and RoPE query N(0,1), absorbed
+    latent query N(0,1/4), a random block permutation, the workload's own
+    sequence lengths); timing does not depend on their values.  Workloads
+    whose cache fits in L2 are timed with a 256 MB L2 flush before each call
+    and also warm (no flush)."""
+    import torch
+    out = {}
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    E = torch.cuda.Event
+    for name in names:
+        cfg = W.CONFIGS[name]
+        sl = W.seq_lens_of(cfg)
+        table, nphys, _ = W.paging(cfg, sl)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(cfg.seed)
+        D = cfg.d_c + cfg.d_r
+        cache = torch.randn((nphys, cfg.block_size, D), generator=g, device="cuda").to(torch.bfloat16)
+        q = torch.randn((cfg.T, cfg.H, D), generator=g, device="cuda")
+        q[..., :cfg.d_c] *= 0.5
+        q = q.to(torch.bfloat16)
+        bt = torch.from_numpy(table).cuda()
+        slt = torch.from_numpy(sl).cuda()
+        dims = M.dims(cfg.H)
+        lat = torch.empty(cfg.T, cfg.H, cfg.d_c, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device="cuda")
+        ws = torch.empty(M.mla_decode_workspace_size(dims, cfg.B, cfg.s, table.shape[1] * 64),
+                         dtype=torch.uint8, device="cuda")
+        call = lambda: M.mla_decode(dims, q, cache, bt, slt, cfg.s, lat, lse, ws)
+        byts, flops, rows = algorithmic(cfg, sl, table.shape[1])
+        small = rows * 1152 < L2_BYTES
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+
+        def timed(do_flush):
+            ts = []
+            for _ in range(iters):
+                if do_flush:
+                    flush.fill_(1)
+                a, b = E(enable_timing=True), E(enable_timing=True)
+                a.record()
+                call()
+                b.record()
+                ts.append((a, b))
+            torch.cuda.synchronize()
+            return float(np.mean([x.elapsed_time(y) for x, y in ts])) / 1e3
+
+        t = timed(small)
+        hbm_t, tc_t = byts / (pk["hbm"] * 1e9), flops / (pk["tc"] * 1e12)
+        r = {"workload": cfg.describe, "us": t * 1e6, "cache_gbs": rows * 1152 / t / 1e9,
+             "gbs": byts / t / 1e9, "tflops": flops / t / 1e12,
+             "bound": "hbm" if hbm_t >= tc_t else "tensor", "roofline_us": max(hbm_t, tc_t) * 1e6,
+             "roofline_frac": max(hbm_t, tc_t) / t, "decode_ctas": M.mla_decode_ctas(dims, cfg.s),
+             "l2": "flushed before each call" if small else "cache larger than L2"}
+        if small:
+            r["warm_l2_us"] = timed(False) * 1e6
+        out[name] = r
+        del cache, q, lat, lse, ws, bt, slt
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------- CPU oracle (baseline)
@@ -463,6 +534,7 @@ def main():
     ap.add_argument("--simple", action="store_true", help="force the CUDA-core decode kernel")
     ap.add_argument("--batch", type=int, default=0, help="override the number of sequences (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip timing the decode of every workload")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps on the stream, not as a graph")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

@@ -1,0 +1,161 @@
+// absorb.cuh -- query absorption in one launch (sm_100a):
+//   q_abs[t][i][0:512]   = (U^K_i)^T q^C_{t,i}          (fp32 accumulation -> bf16)
+//   q_abs[t][i][512:576] = RoPE(q^R_{t,i}, q_pos[t])   (copied if q_pos is null)
+// (DeepSeek-V2 paper review, section 2: (q^C)^T U^K c = ((U^K)^T q^C)^T c;
+// section 3: a per-head RoPE query of 64 dims).
+//
+// CTA (i, m): head i, tokens [128m, 128m+128).  Per head the product is
+// [T x 128] . [128 x 512]: all of it fits one CTA, so U^K_i (128 KB) is read
+// once and every head runs in the first wave.  Warp 0 loads the token tile
+// of q^C (two 64-column chunks) and U^K_i (MN-major: for each of the two
+// 64-row K chunks, eight 64-column N chunks) with TMA in one go; warp 1
+// issues 16 tcgen05 MMAs (M=128, N=256, K=16) into two accumulators (TMEM
+// columns 0-255 and 256-511); warps 2-9 read them back, two warps per TMEM
+// lane quarter (thread = token row, half of the 512 columns each), and the
+// first of each pair also turns the row's RoPE query.  No TMA load uses
+// cluster multicast.
+#pragma once
+
+#include "dec_common.cuh"
+
+namespace mla {
+
+constexpr int kAbThreads = 320;
+constexpr int kAbA = 128 * 64 * 2;                // one q^C chunk: 128 tokens x 64 (16 KB)
+constexpr int kAbBChunk = 64 * 64 * 2;            // one U^K box: 64 K rows x 64 N (8 KB)
+constexpr int kAbB = 8 * kAbBChunk;               // one K chunk of U^K_i: 64 x 512 (64 KB)
+constexpr int kAbOffB = 2 * kAbA;                 // 32 KB
+constexpr int kAbOffBar = kAbOffB + 2 * kAbB;     // 163,840
+constexpr int kAbSmem = kAbOffBar + 512 + 1024;   // barriers, the RoPE table (256 B), alignment slack
+
+__global__ void __launch_bounds__(kAbThreads, 1)
+absorb_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_uk,
+              const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos, int T, int H,
+              bf16 *__restrict__ q_abs, double base, uint32_t *err, unsigned long long limit_ns)
+{
+    extern __shared__ uint8_t ab_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(ab_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kAbOffBar);
+    uint64_t *done = full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    double *theta = reinterpret_cast<double *>(smem + kAbOffBar + 64);   // [32] RoPE frequencies
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int head = blockIdx.x, m0 = blockIdx.y * 128;
+
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(full, 1);
+        sm100::mbar_init(done, 1);
+        *abort_flag = 0;
+        sm100::fence_mbar_init();
+        sm100::prefetch_tensormap(&map_q);
+        sm100::prefetch_tensormap(&map_uk);
+    }
+    if (warp == 9)  // theta_k = base^(-2k/64), k = 0..31 (the RoPE pairs)
+        theta[lane] = pow(base, -2.0 * (double)lane / (double)kDr);
+    if (warp == 1) {
+        sm100::tmem_alloc(tmem_slot, 512);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (sm100::elect_one()) {
+            sm100::mbar_arrive_expect_tx(full, 2 * kAbA + 2 * kAbB);
+            for (int kc = 0; kc < 2; ++kc) {
+                sm100::tma_load_3d(&map_q, full, smem + kc * kAbA, 64 * kc, m0, head);
+                for (int j = 0; j < 8; ++j)
+                    sm100::tma_load_3d(&map_uk, full, smem + kAbOffB + kc * kAbB + j * kAbBChunk, 64 * j, 64 * kc, head);
+            }
+        }
+    } else if (warp == 1) {
+        if (sm100::elect_one()) {
+            if (sm100::mbar_wait(full, 0, abort_flag, err, limit_ns)) {
+                sm100::tc_fence_after();
+                const uint32_t idesc = sm100::idesc_bf16(128, 256, 0, 1);
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc) {
+                    const uint64_t ad = sm100::desc_kmajor(sm100::smem_u32(smem + kc * kAbA), 128, sm100::kSw128);
+#pragma unroll
+                    for (int nh = 0; nh < 2; ++nh) {
+                        const uint64_t bd = sm100::desc_mnmajor_sw128(
+                            sm100::smem_u32(smem + kAbOffB + kc * kAbB + 4 * nh * kAbBChunk), kAbBChunk);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            sm100::umma_ss(tmem + 256 * nh, ad + (uint64_t)((kk * 32) >> 4),
+                                           bd + (uint64_t)((kk * 16 * 128) >> 4), idesc, (kc | kk) != 0);
+                    }
+                }
+            }
+            sm100::umma_commit(done);
+        }
+    } else {
+        // epilogue: warp w (2..9) reads TMEM lane quarter w % 4 (thread = token
+        // row), columns [256 h, 256 h + 256) with h = (w - 2) / 4
+        const int qd = warp & 3, h = (warp - 2) >> 2;
+        const int t = m0 + 32 * qd + lane;
+        const bool ok = sm100::warp_wait(done, 0, abort_flag, err, limit_ns);
+        sm100::tc_fence_after();
+        bf16 *row = q_abs + ((long long)t * H + head) * kRow;
+        if (ok) {
+#pragma unroll 1
+            for (int c = 0; c < 256; c += 32) {
+                uint32_t v[32];
+                sm100::tmem_ld16(sm100::tmem_addr(tmem + 256 * h, 32 * qd, c), v);
+                sm100::tmem_ld16(sm100::tmem_addr(tmem + 256 * h, 32 * qd, c + 16), v + 16);
+                sm100::tmem_wait_ld();
+                if (t < T) {
+                    uint4 *d = reinterpret_cast<uint4 *>(row + 256 * h + c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d[e] = make_uint4(pack_bf162(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                                          pack_bf162(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                                          pack_bf162(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                                          pack_bf162(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+                }
+            }
+        }
+        if (t < T) {
+            // RoPE pairs [16h, 16h+16) of the row's query: the angle p*theta_k
+            // is formed and reduced to [-pi, pi] in double precision (at
+            // positions up to 2^17 an fp32 product would be off by ~1e-2 rad),
+            // then its sine and cosine are taken in fp32
+            const __nv_bfloat162 *src = reinterpret_cast<const __nv_bfloat162 *>(q_rope + ((long long)t * H + head) * kDr);
+            const double p = q_pos ? (double)q_pos[t] : 0.0;
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int k = 16 * h + e;
+                const float2 x = __bfloat1622float2(src[k]);
+                if (q_pos) {
+                    const double ang = p * theta[k];
+                    const double red = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+                    float sn, cs;
+                    sincosf((float)red, &sn, &cs);
+                    o[e] = pack_bf162(x.x * cs - x.y * sn, x.x * sn + x.y * cs);
+                } else {
+                    o[e] = pack_bf162(x.x, x.y);
+                }
+            }
+            uint4 *d = reinterpret_cast<uint4 *>(row + kDc + 32 * h);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
+    }
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        if (*abort_flag) {
+            volatile int no_abort = 0;
+            sm100::mbar_wait(done, 0, &no_abort, err, limit_ns);
+        }
+        sm100::tc_fence_after();
+        sm100::tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace mla

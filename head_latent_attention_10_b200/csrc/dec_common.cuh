@@ -114,6 +114,7 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
                 int32_t *__restrict__ plan, uint32_t *err)
 {
     __shared__ int part[1024];
+    sm100::pdl_trigger();   // the decode kernel may set itself up meanwhile
     const int per = (B + 1023) / 1024;
     const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
     int sum = 0;
@@ -152,54 +153,84 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
 
 
 // ------------------------------------------------------------------ combine
-// grid (B, row blocks): sequences cut by range ends are merged by
-// log-sum-exp; sequences one range finished are already in place; queries
-// with no visible key get a zero latent and lse = -inf.
-__global__ void __launch_bounds__(128)
+// Sequences cut by range ends are merged by log-sum-exp; sequences one range
+// finished are already in place; queries with no visible key get a zero
+// latent and lse = -inf.  Work item = (sequence b, block of 16 of its s*H
+// rows); CTAs of 8 warps take items in turn, warp w rows 2w and 2w+1 of the
+// block, lane l latent columns [16l, 16l+16).  Every row index is checked
+// against s*H, every partial slot lies in [2 c0, 2 c1 + 1] with c1 < ranges.
+constexpr int kCombineRows = 16;
+constexpr int kCombineThreads = 256;
+
+__host__ __device__ inline int combine_items(int B, int s, int H)
+{
+    return B * ((s * H + kCombineRows - 1) / kCombineRows);
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
 dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
                    const float *__restrict__ part_lse2, const int32_t *__restrict__ seq_lens, int max_blocks,
-                   int s, int H, bf16 *__restrict__ out, float *__restrict__ out_lse)
+                   int B, int s, int H, bf16 *__restrict__ out, float *__restrict__ out_lse)
 {
-    const int b = blockIdx.x, tid = threadIdx.x;
+    sm100::pdl_wait();      // the decode kernel's partials and outputs are complete
     const int rows = s * H;
+    const int per_seq = (rows + kCombineRows - 1) / kCombineRows;
+    const int items = B * per_seq;
     const int q = plan[0];
-    const int a0 = plan[4 + b], a1 = plan[4 + b + 1];
-    int L = seq_lens[b];
-    L = L < 0 ? 0 : min(L, max_blocks * kBlock);
-    const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
-    const bool split = a1 > a0 && c0 != c1;
-    if (!split && L >= s) return;
-    for (int rr = blockIdx.y; rr < rows; rr += gridDim.y) {
-        const int t = rr / H;
-        const long long orow = (long long)b * rows + rr;
-        if (L - s + t + 1 <= 0) {
-            reinterpret_cast<uint2 *>(out + orow * kDc)[tid] = make_uint2(0, 0);
-            if (tid == 0 && out_lse) out_lse[orow] = -INFINITY;
-            continue;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int b = item / per_seq, rb = item % per_seq;
+        const int a0 = plan[4 + b], a1 = plan[4 + b + 1];
+        int L = seq_lens[b];
+        L = L < 0 ? 0 : min(L, max_blocks * kBlock);
+        const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
+        const bool split = a1 > a0 && c0 != c1;
+        if (!split && L >= s) continue;  // written by the decode kernel
+        for (int j = 0; j < kCombineRows / 8; ++j) {
+            const int rr = rb * kCombineRows + 2 * warp + j;
+            if (rr >= rows) break;
+            const int t = rr / H;
+            const long long orow = (long long)b * rows + rr;
+            uint4 *dst = reinterpret_cast<uint4 *>(out + orow * kDc + 16 * lane);
+            if (L - s + t + 1 <= 0) {
+                dst[0] = make_uint4(0, 0, 0, 0);
+                dst[1] = make_uint4(0, 0, 0, 0);
+                if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
+                continue;
+            }
+            if (!split) continue;
+            float M = -INFINITY;
+            for (int c = c0; c <= c1; ++c) {
+                const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
+                M = fmaxf(M, part_lse2[(long long)slot * rows + rr]);
+            }
+            float acc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+            float den = 0.f;
+            for (int c = c0; c <= c1; ++c) {
+                const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
+                const float l2 = part_lse2[(long long)slot * rows + rr];
+                const float w = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
+                den += w;
+                const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc + 16 * lane);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 v = src[e];
+                    acc[4 * e] = fmaf(w, v.x, acc[4 * e]);
+                    acc[4 * e + 1] = fmaf(w, v.y, acc[4 * e + 1]);
+                    acc[4 * e + 2] = fmaf(w, v.z, acc[4 * e + 2]);
+                    acc[4 * e + 3] = fmaf(w, v.w, acc[4 * e + 3]);
+                }
+            }
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = pack_bf162(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (lane == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
         }
-        if (!split) continue;
-        float M = -INFINITY;
-        for (int c = c0; c <= c1; ++c) {
-            const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
-            M = fmaxf(M, part_lse2[(long long)slot * rows + rr]);
-        }
-        float den = 0.f;
-        float4 acc = make_float4(0, 0, 0, 0);
-        for (int c = c0; c <= c1; ++c) {
-            const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
-            const float l2 = part_lse2[(long long)slot * rows + rr];
-            const float w = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
-            den += w;
-            const float4 v = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc)[tid];
-            acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-        }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        uint2 pk;
-        pk.x = pack_bf162(acc.x * inv, acc.y * inv);
-        pk.y = pack_bf162(acc.z * inv, acc.w * inv);
-        reinterpret_cast<uint2 *>(out + orow * kDc)[tid] = pk;
-        if (tid == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
     }
 }
 

@@ -1,5 +1,4 @@
-// k_simple.cuh -- CUDA-core kernels: the cache writers (from latents, and the
-// split-K finish of the append projection), the query RoPE, and a
+// k_simple.cuh -- CUDA-core kernels: the cache writer from latents and a
 // straightforward split-KV decode with its log-sum-exp combine
 // (MLA_FORCE_SIMPLE), a cross-check for the tensor-core decode.
 #pragma once
@@ -53,81 +52,6 @@ append_latent_kernel(const bf16 *__restrict__ c_kv, const bf16 *__restrict__ k_r
     float y0, y1;
     rope_pair(__low2float(kr), __high2float(kr), p, lane, kDr, base, &y0, &y1);
     reinterpret_cast<__nv_bfloat162 *>(dst + kDc)[lane] = __floats2bfloat162_rn(y0, y1);
-}
-
-// ------------------------------------------------- append, split-K finish
-// Sums the split-K partials of the append projection in slice order (so the
-// result does not depend on scheduling), turns the RoPE pairs (columns
-// 512..575) and writes the bf16 row to the token's cache slot.  One thread
-// per (token, 8 columns).
-__global__ void __launch_bounds__(256)
-append_finish_kernel(const float *__restrict__ scratch, int S, long long zs, int T,
-                     const int32_t *__restrict__ seq_idx, const int32_t *__restrict__ pos,
-                     const int32_t *__restrict__ block_table, int num_seqs, int max_blocks,
-                     bf16 *__restrict__ cache, int num_blocks, double base, uint32_t *err)
-{
-    constexpr int kChunks = kRow / 8;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= T * kChunks) return;
-    const int m = i / kChunks, c = (i % kChunks) * 8;
-    const int p = pos[m];
-    const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks, seq_idx[m], p,
-                                      c == 0 ? err : nullptr);
-    if (slot < 0) return;
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const float *src = scratch + (long long)m * kRow + c;
-    for (int z = 0; z < S; ++z) {
-        const float4 a = reinterpret_cast<const float4 *>(src + z * zs)[0];
-        const float4 b = reinterpret_cast<const float4 *>(src + z * zs)[1];
-        v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-        v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
-    }
-    if (c >= kDc) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float y0, y1;
-            rope_pair(v[2 * j], v[2 * j + 1], p, (c - kDc) / 2 + j, kDr, base, &y0, &y1);
-            v[2 * j] = y0;
-            v[2 * j + 1] = y1;
-        }
-    }
-    bf16x8 o;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o.v[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-    *reinterpret_cast<bf16x8 *>(cache + slot * kRow + c) = o;
-}
-
-// RoPE of the query's RoPE part into q_abs[t][h][512:576] (or a plain copy
-// when q_pos is null).  One warp per (token t, group of kRopeHeads heads):
-// lane k turns pair k, so the angle's sine and cosine are computed once per
-// (t, k) and applied to every head of the group.
-constexpr int kRopeHeads = 16;
-
-__global__ void __launch_bounds__(256)
-rope_q_kernel(const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos, int T, int H,
-              bf16 *__restrict__ q_abs, double base)
-{
-    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int groups = (H + kRopeHeads - 1) / kRopeHeads;
-    if (w >= T * groups) return;
-    const int t = w / groups, h0 = (w % groups) * kRopeHeads;
-    const int h1 = min(H, h0 + kRopeHeads);
-    double sn = 0.0, cs = 1.0;
-    if (q_pos) {
-        const double theta = pow(base, -2.0 * (double)lane / (double)kDr);
-        sincos((double)q_pos[t] * theta, &sn, &cs);
-    }
-    for (int h = h0; h < h1; ++h) {
-        const long long row = (long long)t * H + h;
-        const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(q_rope + row * kDr)[lane];
-        __nv_bfloat162 y = x;
-        if (q_pos) {
-            const double x0 = __low2float(x), x1 = __high2float(x);
-            y = __floats2bfloat162_rn((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
-        }
-        reinterpret_cast<__nv_bfloat162 *>(q_abs + row * kRow + kDc)[lane] = y;
-    }
 }
 
 // ------------------------------------------------------------- simple decode

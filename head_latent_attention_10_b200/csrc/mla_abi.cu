@@ -9,9 +9,12 @@
 #include <atomic>
 #include <mutex>
 
+#include "absorb.cuh"
+#include "append_proj.cuh"
 #include "common.cuh"
 #include "k_simple.cuh"
 #include "tc_decode64.cuh"
+#include "tc_decode_pair.cuh"
 #include "tc_gemm.cuh"
 #include "tmap.cuh"
 
@@ -112,12 +115,12 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
     return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
 }
 
-template <int BN, bool kBmn, class Epi, bool kSplitK = false>
+template <int BN, bool kBmn, class Epi>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
                            uint32_t *err, cudaStream_t st)
 {
     using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kSplitK>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
     if (e != cudaSuccess) return e;
@@ -125,6 +128,25 @@ cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, in
     kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, kWaitLimitNs);
     count_launch();
     return cudaGetLastError();
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream runs, and waits for it with pdl_wait().
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 // Workspace of the decode: [error word | pad] [partial latents] [partial lse2]
@@ -165,19 +187,58 @@ TcWs tc_ws(int H, int s, int B)
     return w;
 }
 
-// Ranges (persistent CTAs per row group) of the decode on the current device.
-int decode_ranges(int groups)
+int sm_count()
 {
     static std::atomic<int> sms_cache[kMaxDevices];
-    static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0) return 0;
-    if (ensure_smem_attr(tc_decode64_kernel, kD64Smem, attr_set) != cudaSuccess) return 0;
     int sms = sms_cache[dev].load(std::memory_order_acquire);
     if (sms <= 0) {
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 0;
         sms_cache[dev].store(sms, std::memory_order_release);
     }
+    return sms;
+}
+
+// The decode kernel a shape runs on: 128-row groups on CTA pairs when the
+// s*H rows of a sequence split into whole groups of 128, else 64-row groups.
+inline bool use_pair(int H, int s) { return (s * H) % 128 == 0; }
+
+// Ranges (persistent CTAs, or CTA pairs, per row group) of the decode on the
+// current device.
+int decode_ranges(int H, int s)
+{
+    static std::atomic<bool> attr64[kMaxDevices], attr_pair[kMaxDevices];
+    const int sms = sm_count();
+    if (sms <= 0) return 0;
+    if (use_pair(H, s)) {
+        if (ensure_smem_attr(tc_decode_pair_kernel, kPrSmem, attr_pair) != cudaSuccess) return 0;
+        // CTA pairs that can be resident at once (an odd SM left in a GPC
+        // takes no pair), so that every range starts in the first wave
+        static std::atomic<int> pairs_cache[kMaxDevices];
+        const int dev = current_device();
+        if (dev < 0) return 0;
+        int pairs = pairs_cache[dev].load(std::memory_order_acquire);
+        if (pairs <= 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(sms, 1, 1);
+            cfg.blockDim = dim3(kPrThreads, 1, 1);
+            cfg.dynamicSmemBytes = kPrSmem;
+            if (cudaOccupancyMaxActiveClusters(&pairs, tc_decode_pair_kernel, &cfg) != cudaSuccess || pairs <= 0) {
+                cudaGetLastError();
+                pairs = sms / 2;
+            }
+            if (pairs > sms / 2) pairs = sms / 2;
+            pairs_cache[dev].store(pairs, std::memory_order_release);
+        }
+        const int groups = s * H / 128;
+        int r = pairs / groups;
+        const int cap = (kMaxRanges / 2) / groups;
+        if (r > cap) r = cap;
+        return r > 0 ? r : 1;
+    }
+    if (ensure_smem_attr(tc_decode64_kernel, kD64Smem, attr64) != cudaSuccess) return 0;
+    const int groups = dec_groups(H, s);
     int r = sms / groups;
     const int cap = kMaxRanges / groups;
     if (r > cap) r = cap;
@@ -194,28 +255,6 @@ void *noalloc_scratch()
     return symbol_address(g_noalloc_scratch, addr);
 }
 
-// Split-K partial sums of the append projection: one array per device.
-constexpr size_t kAppendScratchFloats = 4u << 20;  // 16 MB
-__device__ __align__(256) float g_append_scratch[kAppendScratchFloats];
-
-float *append_scratch()
-{
-    static std::atomic<void *> addr[kMaxDevices];
-    return static_cast<float *>(symbol_address(g_append_scratch, addr));
-}
-
-// K slice of the split-K append projection: the narrowest 128 * 2^j that
-// divides d_model and whose partials fit the scratch; 0 when none does (or
-// when fewer than two slices would result).
-int append_kslice(int T, int d_model)
-{
-    for (int ks = 128; ks <= d_model / 2; ks *= 2) {
-        if (d_model % ks) continue;
-        if ((size_t)(d_model / ks) * (size_t)T * kRow <= kAppendScratchFloats) return ks;
-    }
-    return 0;
-}
-
 }  // namespace
 
 extern "C" {
@@ -223,8 +262,10 @@ extern "C" {
 int mla_decode_ctas(const mla_dims_t *dims, int s)
 {
     if (check_dims(dims) != MLA_OK || s <= 0) return 0;
-    const int g = dec_groups(dims->num_heads, s);
-    return decode_ranges(g) * g;
+    const int H = dims->num_heads;
+    if (use_pair(H, s)) return 2 * decode_ranges(H, s) * (s * H / 128);
+    const int g = dec_groups(H, s);
+    return decode_ranges(H, s) * g;
 }
 
 uint64_t mla_kernel_launches(void) { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
@@ -276,29 +317,27 @@ mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int 
     if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(cache))
         return MLA_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
+    if (d_model % (64 * kApSlices) == 0) {
+        // K split over a cluster of CTAs, partials reduced on chip, one launch
+        CUtensorMap mh, md, mr;
+        if (!tmap(&mh, h, d_model, T, 1, d_model, 0, 64, 128) ||
+            !tmap(&md, w_dkv, d_model, kDc, 1, d_model, 0, 64, 64) ||
+            !tmap(&mr, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
+            return MLA_ERR_CUDA;
+        static std::atomic<bool> attr_set[kMaxDevices];
+        if (ensure_smem_attr(append_proj_kernel, kApSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
+        AppendArgs aa{(bf16 *)cache, seq_idx, pos, block_table, T, d_model, num_seqs, max_blocks, num_blocks,
+                      rope_base(dims), err_word, kWaitLimitNs};
+        append_proj_kernel<<<dim3(9, (T + 127) / 128, kApSlices), kApThreads, kApSmem, s>>>(mh, md, mr, aa);
+        count_launch();
+        return cuda_status(cudaGetLastError());
+    }
+    // other widths: one pass over K per 128-token tile
     CUtensorMap ma, mb1, mb2;
     if (!tmap(&ma, h, d_model, T, 1, d_model, 0, 64, 128) ||
         !tmap(&mb1, w_dkv, d_model, kDc, 1, d_model, 0, 64, 256) ||
         !tmap(&mb2, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
         return MLA_ERR_CUDA;
-    const int ks = append_kslice(T, d_model);
-    if (ks > 0) {
-        // few tokens, long K: split K over CTAs, sum the slices in order
-        float *scr = append_scratch();
-        if (!scr) return MLA_ERR_CUDA;
-        const int S = d_model / ks;
-        const long long zs = (long long)T * kRow;
-        if (launch_tc_gemm<256, false, TcEpiPartial, true>(ma, mb1, T, kDc, ks, S, TcEpiPartial{scr, zs, kRow, 0},
-                                                          err_word, s) != cudaSuccess ||
-            launch_tc_gemm<64, false, TcEpiPartial, true>(ma, mb2, T, kDr, ks, S, TcEpiPartial{scr, zs, kRow, kDc},
-                                                         err_word, s) != cudaSuccess)
-            return MLA_ERR_CUDA;
-        append_finish_kernel<<<(T * (kRow / 8) + 255) / 256, 256, 0, s>>>(
-            scr, S, zs, T, seq_idx, pos, block_table, num_seqs, max_blocks, (bf16 *)cache, num_blocks,
-            rope_base(dims), err_word);
-        count_launch();
-        return cuda_status(cudaGetLastError());
-    }
     // c^KV = W^DKV h  (columns 0..511 of the row)
     TcEpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, 0,
                   rope_base(dims), err_word};
@@ -322,16 +361,17 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
         return MLA_ERR_INVALID_ARG;
     const int H = dims->num_heads;
     cudaStream_t s = as_stream(stream);
-    // per head i: q_abs[:, i, 0:512] = q_nope[:, i, :] (T x 128) . U^K_i (128 x 512)
+    // per head i: q_abs[:, i, 0:512] = q_nope[:, i, :] (T x 128) . U^K_i (128 x 512),
+    // and the RoPE part, in one launch
     CUtensorMap ma, mb;
     if (!tmap(&ma, q_nope, kDh, T, H, (uint64_t)H * kDh, kDh, 64, 128) ||
         !tmap(&mb, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64))
         return MLA_ERR_CUDA;
-    TcEpiStore e{(bf16 *)q_abs, kRow, (long long)H * kRow};
-    if (launch_tc_gemm<256, true>(ma, mb, T, kDc, kDh, H, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
-    const int warps = T * ((H + kRopeHeads - 1) / kRopeHeads);
-    rope_q_kernel<<<(warps + 7) / 8, 256, 0, s>>>((const bf16 *)q_rope, q_pos, T, H, (bf16 *)q_abs,
-                                                  rope_base(dims));
+    static std::atomic<bool> attr_set[kMaxDevices];
+    if (ensure_smem_attr(absorb_kernel, kAbSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
+    absorb_kernel<<<dim3(H, (T + 127) / 128), kAbThreads, kAbSmem, s>>>(ma, mb, (const bf16 *)q_rope, q_pos, T, H,
+                                                                         (bf16 *)q_abs, rope_base(dims), nullptr,
+                                                                         kWaitLimitNs);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
@@ -383,12 +423,23 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
     } else {
         const TcWs w = tc_ws(H, s, B);
         if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
-        const int groups = dec_groups(H, s);
-        const int ranges = decode_ranges(groups);
+        const bool pr = use_pair(H, s);
+        const int groups = pr ? s * H / 128 : dec_groups(H, s);
+        const int ranges = decode_ranges(H, s);
         if (ranges <= 0) return MLA_ERR_CUDA;
-        CUtensorMap mkv;
         const uint64_t rows = (uint64_t)num_blocks * kBlock;
-        if (!tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
+        PairMaps pm;
+        CUtensorMap mkv;
+        if (pr) {
+            const uint64_t qrows = (uint64_t)T * H;
+            if (!tmap(&pm.kv_lat, cache, kRow, rows, 1, kRow, 0, 64, kPrT) ||
+                !tmap(&pm.kv_rope, cache, kRow, rows, 1, kRow, 0, 32, kPrT) ||
+                !tmap(&pm.q_lat, q_abs, kRow, qrows, 1, kRow, 0, 64, 128) ||
+                !tmap(&pm.q_rope, q_abs, kRow, qrows, 1, kRow, 0, 32, 128))
+                return MLA_ERR_CUDA;
+        } else if (!tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kT64)) {
+            return MLA_ERR_CUDA;
+        }
         if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
         int32_t *plan = (int32_t *)(ws + w.off_plan);
         dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
@@ -413,14 +464,21 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.H = H;
         da.B = B;
         da.groups = groups;
-        tc_decode64_kernel<<<ranges * groups, kD64Threads, kD64Smem, strm>>>(mkv, da);
+        // the decode kernel sets itself up while the plan runs, and the
+        // combine launches while the decode's last CTAs finish
+        cudaError_t e = pr ? launch_pdl(tc_decode_pair_kernel, dim3(2 * ranges * groups), dim3(kPrThreads),
+                                        kPrSmem, strm, pm, da)
+                           : launch_pdl(tc_decode64_kernel, dim3(ranges * groups), dim3(kD64Threads), kD64Smem,
+                                        strm, mkv, da);
         count_launch();
-        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-        const int ry = s * H < 128 ? s * H : 128;
-        dec_combine_kernel<<<dim3(B, ry), 128, 0, strm>>>(plan, da.part_o, da.part_lse2, seq_lens, max_blocks, s, H,
-                                                          (bf16 *)out_latent, out_lse);
+        if (e != cudaSuccess) return MLA_ERR_CUDA;
+        const int items = combine_items(B, s, H);
+        const int cgrid = items < 4 * sm_count() ? items : 4 * sm_count();
+        e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
+                       (const float *)da.part_o, (const float *)da.part_lse2, seq_lens, max_blocks, B, s, H,
+                       (bf16 *)out_latent, out_lse);
         count_launch();
-        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+        if (e != cudaSuccess) return MLA_ERR_CUDA;
     }
     if (flags & MLA_SYNC_CHECK) {
         uint32_t host = 0;

@@ -94,6 +94,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = blockIdx.x % a.groups, rng = blockIdx.x / a.groups;
+    sm100::pdl_wait();  // the plan is complete
     const int32_t *seq_start = a.plan + 4;
     const int q_per = a.plan[0], total = a.plan[1];
     const int lo = rng * q_per, hi = min(lo + q_per, total);
@@ -457,6 +458,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     }
 
     // ------------------------------------------------------------ teardown
+    sm100::pdl_trigger();   // the combine may start launching
     sm100::tc_fence_before();
     __syncthreads();
     if (warp == 1 || warp == 2 || warp >= 4) {

@@ -12,9 +12,6 @@
 // A is K-major (rows of K contiguous).  B is either K-major (B^T stored
 // row-major, e.g. a weight [N][K]) or MN-major (B stored [K][N]).
 // Tensor maps are 3-D: A {K, M, Z}, B K-major {K, N, Z}, B MN-major {N, K, Z}.
-// Split-K mode (kSplitK): blockIdx.z picks a slice of K instead of a batch:
-// CTA z reduces K columns [z*K, (z+1)*K) of 2-D (Z = 1) operands, and the
-// epilogue receives z so that it can store a partial sum per slice.
 #pragma once
 
 #include "sm100.cuh"
@@ -34,7 +31,7 @@ struct GemmSmem {
     static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
 };
 
-template <int BN, bool kBmn, class Epi, bool kSplitK = false>
+template <int BN, bool kBmn, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, int M,
                int N, int K, Epi epi, uint32_t *err, unsigned long long limit_ns)
@@ -84,14 +81,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 uint8_t *a = smem + s * S::STAGE;
                 uint8_t *b = a + S::A;
                 sm100::mbar_arrive_expect_tx(&full[s], S::STAGE);
-                const int kx = (kSplitK ? z * nk + kb : kb) * 64, zz = kSplitK ? 0 : z;
-                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, zz);
+                const int kx = kb * 64;
+                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, z);
                 if (kBmn) {
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
-                        sm100::tma_load_3d(&mapB, &full[s], b + j * 8192, n0 + 64 * j, kx, zz);
+                        sm100::tma_load_3d(&mapB, &full[s], b + j * 8192, n0 + 64 * j, kx, z);
                 } else {
-                    sm100::tma_load_3d(&mapB, &full[s], b, kx, n0, zz);
+                    sm100::tma_load_3d(&mapB, &full[s], b, kx, n0, z);
                 }
             }
             if (*abort_flag) {
@@ -165,20 +162,6 @@ struct TcEpiStore {
         uint4 *p = reinterpret_cast<uint4 *>(base + z * bs + m * rs + n);
         p[0] = pk[0];
         p[1] = pk[1];
-    }
-};
-
-// Split-K partial sums: 16 fp32 outputs of slice z at
-// scratch[z*zs + m*ld + col0 + n] (16-byte aligned).
-struct TcEpiPartial {
-    float *scratch;
-    long long zs;
-    int ld, col0;
-    __device__ void operator()(int z, int m, int n, const float *v) const
-    {
-        float4 *p = reinterpret_cast<float4 *>(scratch + z * zs + (long long)m * ld + col0 + n);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
 };
 

@@ -23,12 +23,11 @@
  *   - Every pointer is caller-owned DEVICE memory unless stated otherwise.
  *     No call allocates device memory (no cudaMalloc, no allocating library
  *     routine).  mla_decode keeps its scratch in the caller's workspace;
- *     mla_absorb_q, mla_append_latent and mla_up_v need none.  Two calls use
- *     a fixed file-scope device array inside the library instead, one per
- *     device, held until the process exits: mla_append_cache (16 MB of
- *     split-K partial sums) and mla_decode_noalloc (MLA_NOALLOC_SCRATCH_BYTES).
- *     Calls of either kind that may overlap on one device race on that
- *     array (see their notes); calls ordered on one stream are safe.
+ *     mla_append_cache, mla_append_latent, mla_absorb_q and mla_up_v need
+ *     none.  One call, mla_decode_noalloc, uses a fixed file-scope device
+ *     array inside the library instead (MLA_NOALLOC_SCRATCH_BYTES, one per
+ *     device, held until the process exits); calls of it that may overlap on
+ *     one device race on that array (see its notes).
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream).  Inputs are never modified,
  *     except the cache by the append calls.
@@ -117,13 +116,10 @@ const char *mla_status_string(mla_status_t status);
  *   err_word     optional device uint32; bits MLA_DEVERR_* are OR-ed in for
  *                tokens whose slot is invalid (those tokens are not written)
  * d_model must be a positive multiple of 64.  T = 0 is a no-op.
- * For few tokens (T * d_model small enough) the projection splits K over
- * many CTAs and keeps the fp32 partial sums in a 16 MB array inside the
- * library (one per device); the slices are summed in a fixed order, so the
- * result is deterministic.  Calls on one stream are ordered; calls that may
- * overlap on one device (different streams, unordered host threads) race on
- * that array.  The first call on a device looks up its address and should
- * precede any stream capture.
+ * When d_model is a multiple of 512 the projection splits K over a cluster
+ * of 8 CTAs per 64-column tile and sums their fp32 partials on chip in a
+ * fixed order (deterministic, one launch, no scratch outside the kernel's
+ * shared memory); other widths take one pass over K per 128-token tile.
  */
 mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int d_model,
                               const void *w_dkv, const void *w_kr,

@@ -152,12 +152,13 @@ def test_append_cache_projection(lib, cfg):
     assert np.array_equal(got[mask], cache0[mask])
 
 
-@pytest.mark.parametrize("d_model", [576, 1024], ids=["one_pass", "split_k"])
+@pytest.mark.parametrize("d_model", [576, 1024], ids=["one_pass", "cluster_split_k"])
 def test_append_cache_identity_weights_are_bit_exact(lib, d_model):
     """W^DKV = [I 0], W^KR = [0 I 0] at position 0 copies the first 576
     columns of h bit for bit (projection by I is exact in fp32, also when
-    the K sum is split over CTAs; RoPE at 0 is the identity).  576 runs the
-    GEMM in one pass over K, 1024 the split-K path."""
+    the K sum is split over the CTAs of a cluster; RoPE at 0 is the
+    identity).  576 runs the GEMM in one pass over K, 1024 the cluster
+    split-K kernel."""
     import torch
     cfg = W.MLAConfig("ident", B=2, s=1, H=16, L=0, paged=True, seed=301, d_model=d_model,
                       seq_lens=(5, 70))
@@ -310,3 +311,49 @@ def test_empty_batch_is_a_no_op(lib):
     cache = torch.empty(1, 64, 576, dtype=torch.bfloat16, device="cuda")
     out = torch.empty(0, 128, 512, dtype=torch.bfloat16, device="cuda")
     lib.mla_decode(d, q, cache, z.view(0, 1), z, 1, out, None, ws)
+
+
+@pytest.mark.parametrize("d_model", [2048, 5120])
+def test_append_cache_many_tokens(lib, d_model):
+    """More than one 128-token tile of the cluster split-K projection (T = 300,
+    a ragged last tile) against the fp64 projection, with every token in a
+    slot of its own."""
+    o = _oracle()
+    cfg = W.MLAConfig("app_many", B=4, s=1, H=16, L=0, paged=True, seed=311, d_model=d_model,
+                      seq_lens=(400, 130, 64, 700))
+    g = GpuWorkload(cfg)
+    a = W.make_append_inputs(cfg, 300)
+    rng = np.random.default_rng(12)
+    slots = rng.choice(int(np.sum(g.d["seq_lens"])), size=300, replace=False)
+    seq = g.d["tok_seq"][slots].astype(np.int32)
+    pos = g.d["tok_pos"][slots].astype(np.int32)
+    cache0 = host_bits(g.cache)
+    lib.mla_append_cache(g.dims, torch_bits(a["h"]), torch_bits(a["w_dkv"]), torch_bits(a["w_kr"]),
+                         i32(seq), i32(pos), g.block_table, g.cache, err_word=g.err)
+    got = host_bits(g.cache)
+    c_ref, kr_ref = o.kv_project(a["h"], a["w_dkv"], a["w_kr"], pos)
+    bt = g.d["block_table"]
+    blk, slot = bt[seq, pos // 64], pos % 64
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, :512]), c_ref, what="c_kv")
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, 512:]), kr_ref, what="k_rope")
+    mask = np.ones(got.shape[:2], bool); mask[blk, slot] = False
+    assert np.array_equal(got[mask], cache0[mask])
+    assert int(g.err.item()) == 0
+
+
+def test_absorb_q_many_tokens_and_rotated_copy(lib):
+    """Several 128-token tiles per head (T = 300, ragged), and with no
+    positions the RoPE part is the input copied bit for bit."""
+    import torch
+    o = _oracle()
+    cfg = W.MLAConfig("abs_many", B=150, s=2, H=32, L=64, paged=True, seed=312, d_model=2048)
+    d = W.make_decode_inputs(cfg, with_cache_pages=False)
+    dims = lib.dims(cfg.H)
+    q_abs = torch.empty(cfg.T, cfg.H, 576, dtype=torch.bfloat16, device="cuda")
+    lib.mla_absorb_q(dims, torch_bits(d["q_nope"]), torch_bits(d["q_rope"]), i32(d["q_pos"]), torch_bits(d["w_uk"]),
+                     q_abs)
+    ref = o.absorb_q(o.bf16_to_f64(d["q_nope"]), o.bf16_to_f64(d["q_rope"]), o.bf16_to_f64(d["w_uk"]),
+                     q_pos=d["q_pos"])
+    assert_parity(W.bf16_bits_to_f32(host_bits(q_abs)), ref, what="absorb_q, 300 tokens")
+    lib.mla_absorb_q(dims, torch_bits(d["q_nope"]), torch_bits(d["q_rope"]), None, torch_bits(d["w_uk"]), q_abs)
+    assert np.array_equal(host_bits(q_abs)[..., 512:], d["q_rope"])
