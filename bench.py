@@ -61,9 +61,9 @@ def algorithmic(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
 
 # DRAM bytes (read + write) the current decode kernel moves per cache token,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
-# tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (166.5 MB for
+# tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (166.9 MB for
 # 131,072 tokens).  Set to None whenever the decode kernel changes.
-DECODE_DRAM_BYTES_PER_TOKEN = 166.5e6 / (32 * 4096)
+DECODE_DRAM_BYTES_PER_TOKEN = 166.9e6 / (32 * 4096)
 
 
 class ClockSampler:

@@ -87,6 +87,33 @@ struct TileIter {
     }
 };
 
+// Warp-uniform bounded wait until *cnt >= target (a count other warps of the
+// CTA raise with atomicAdd after their tcgen05 fences); lane 0 polls, and the
+// verdict is broadcast.  Same give-up rules as sm100::mbar_wait.
+__device__ __forceinline__ bool wait_count(volatile int *cnt, int target, volatile int *abort, uint32_t *err,
+                                           unsigned long long limit_ns)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0 && *cnt < target) {
+        const uint64_t t0 = sm100::globaltimer_ns();
+        for (uint32_t i = 1; *cnt < target; ++i) {
+            if ((i & 255u) == 0) {
+                if (*abort) { ok = 0; break; }
+                if (sm100::globaltimer_ns() - t0 > limit_ns) {
+                    set_error(err, MLA_DEVERR_TIMEOUT);
+                    *abort = 1;
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        __threadfence_block();
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -155,16 +182,24 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
 // ------------------------------------------------------------------ combine
 // Sequences cut by range ends are merged by log-sum-exp; sequences one range
 // finished are already in place; queries with no visible key get a zero
-// latent and lse = -inf.  Work item = (sequence b, block of 16 of its s*H
-// rows); CTAs of 8 warps take items in turn, warp w rows 2w and 2w+1 of the
-// block, lane l latent columns [16l, 16l+16).  Every row index is checked
-// against s*H, every partial slot lies in [2 c0, 2 c1 + 1] with c1 < ranges.
-constexpr int kCombineRows = 16;
-constexpr int kCombineThreads = 256;
+// latent and lse = -inf.  One warp per (sequence b, row rr < s*H), CTAs of 8
+// warps over consecutive rows; lane l owns latent columns [16l, 16l+16).  The
+// pieces of a cut sequence are the ranges c0..c1 it spans; lane i reads the
+// log2-sum-exp of piece i (and i + 32, ...), and the partial rows are read
+// four pieces at a time so that 16 loads per lane are in flight.  Every
+// partial slot lies in [2 c0, 2 c1 + 1] with c1 < ranges.
+constexpr int kCombineWarps = 8;
+constexpr int kCombineThreads = 32 * kCombineWarps;
 
-__host__ __device__ inline int combine_items(int B, int s, int H)
+__host__ __device__ inline int combine_ctas(int B, int s, int H)
 {
-    return B * ((s * H + kCombineRows - 1) / kCombineRows);
+    const long long rows = (long long)B * s * H;
+    return (int)((rows + kCombineWarps - 1) / kCombineWarps);
+}
+
+__device__ __forceinline__ int piece_slot(int c, int c0, int a0, int q)
+{
+    return 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
 }
 
 __global__ void __launch_bounds__(kCombineThreads)
@@ -174,63 +209,73 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
 {
     sm100::pdl_wait();      // the decode kernel's partials and outputs are complete
     const int rows = s * H;
-    const int per_seq = (rows + kCombineRows - 1) / kCombineRows;
-    const int items = B * per_seq;
+    const long long items = (long long)B * rows;
     const int q = plan[0];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int item = blockIdx.x; item < items; item += gridDim.x) {
-        const int b = item / per_seq, rb = item % per_seq;
+    const int lane = threadIdx.x & 31;
+    for (long long w = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5); w < items;
+         w += (long long)gridDim.x * kCombineWarps) {
+        const int b = (int)(w / rows), rr = (int)(w % rows);
         const int a0 = plan[4 + b], a1 = plan[4 + b + 1];
         int L = seq_lens[b];
         L = L < 0 ? 0 : min(L, max_blocks * kBlock);
         const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
         const bool split = a1 > a0 && c0 != c1;
         if (!split && L >= s) continue;  // written by the decode kernel
-        for (int j = 0; j < kCombineRows / 8; ++j) {
-            const int rr = rb * kCombineRows + 2 * warp + j;
-            if (rr >= rows) break;
-            const int t = rr / H;
-            const long long orow = (long long)b * rows + rr;
-            uint4 *dst = reinterpret_cast<uint4 *>(out + orow * kDc + 16 * lane);
-            if (L - s + t + 1 <= 0) {
-                dst[0] = make_uint4(0, 0, 0, 0);
-                dst[1] = make_uint4(0, 0, 0, 0);
-                if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
-                continue;
-            }
-            if (!split) continue;
-            float M = -INFINITY;
-            for (int c = c0; c <= c1; ++c) {
-                const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
-                M = fmaxf(M, part_lse2[(long long)slot * rows + rr]);
-            }
-            float acc[16];
+        const int t = rr / H;
+        const long long orow = (long long)b * rows + rr;
+        uint4 *dst = reinterpret_cast<uint4 *>(out + orow * kDc + 16 * lane);
+        if (L - s + t + 1 <= 0) {
+            dst[0] = make_uint4(0, 0, 0, 0);
+            dst[1] = make_uint4(0, 0, 0, 0);
+            if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
+            continue;
+        }
+        if (!split) continue;
+        const int n = c1 - c0 + 1;
+        float M = -INFINITY;
+        for (int i = lane; i < n; i += 32)
+            M = fmaxf(M, part_lse2[(long long)piece_slot(c0 + i, c0, a0, q) * rows + rr]);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-            float den = 0.f;
-            for (int c = c0; c <= c1; ++c) {
-                const int slot = 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
-                const float l2 = part_lse2[(long long)slot * rows + rr];
-                const float w = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
-                den += w;
-                const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc + 16 * lane);
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float acc[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 v = src[e];
-                    acc[4 * e] = fmaf(w, v.x, acc[4 * e]);
-                    acc[4 * e + 1] = fmaf(w, v.y, acc[4 * e + 1]);
-                    acc[4 * e + 2] = fmaf(w, v.z, acc[4 * e + 2]);
-                    acc[4 * e + 3] = fmaf(w, v.w, acc[4 * e + 3]);
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+        float den = 0.f;
+        for (int i0 = 0; i0 < n; i0 += 4) {
+            float4 v[4][4];
+            float wgt[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                wgt[u] = 0.f;
+                if (i0 + u < n) {
+                    const int slot = piece_slot(c0 + i0 + u, c0, a0, q);
+                    const float l2 = part_lse2[(long long)slot * rows + rr];
+                    wgt[u] = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
+                    const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc + 16 * lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v[u][e] = src[e];
                 }
             }
-            const float inv = den > 0.f ? 1.f / den : 0.f;
-            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) pk[e] = pack_bf162(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            if (lane == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+            for (int u = 0; u < 4; ++u) {
+                if (i0 + u >= n) break;
+                den += wgt[u];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[4 * e] = fmaf(wgt[u], v[u][e].x, acc[4 * e]);
+                    acc[4 * e + 1] = fmaf(wgt[u], v[u][e].y, acc[4 * e + 1]);
+                    acc[4 * e + 2] = fmaf(wgt[u], v[u][e].z, acc[4 * e + 2]);
+                    acc[4 * e + 3] = fmaf(wgt[u], v[u][e].w, acc[4 * e + 3]);
+                }
+            }
         }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[e] = pack_bf162(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        if (lane == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
     }
 }
 

@@ -14,7 +14,6 @@
 #include "common.cuh"
 #include "k_simple.cuh"
 #include "tc_decode64.cuh"
-#include "tc_decode_pair.cuh"
 #include "tc_gemm.cuh"
 #include "tmap.cuh"
 
@@ -200,43 +199,12 @@ int sm_count()
     return sms;
 }
 
-// The decode kernel a shape runs on: 128-row groups on CTA pairs when the
-// s*H rows of a sequence split into whole groups of 128, else 64-row groups.
-inline bool use_pair(int H, int s) { return (s * H) % 128 == 0; }
-
-// Ranges (persistent CTAs, or CTA pairs, per row group) of the decode on the
-// current device.
+// Ranges (persistent CTAs per row group) of the decode on the current device.
 int decode_ranges(int H, int s)
 {
-    static std::atomic<bool> attr64[kMaxDevices], attr_pair[kMaxDevices];
+    static std::atomic<bool> attr64[kMaxDevices];
     const int sms = sm_count();
     if (sms <= 0) return 0;
-    if (use_pair(H, s)) {
-        if (ensure_smem_attr(tc_decode_pair_kernel, kPrSmem, attr_pair) != cudaSuccess) return 0;
-        // CTA pairs that can be resident at once (an odd SM left in a GPC
-        // takes no pair), so that every range starts in the first wave
-        static std::atomic<int> pairs_cache[kMaxDevices];
-        const int dev = current_device();
-        if (dev < 0) return 0;
-        int pairs = pairs_cache[dev].load(std::memory_order_acquire);
-        if (pairs <= 0) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(sms, 1, 1);
-            cfg.blockDim = dim3(kPrThreads, 1, 1);
-            cfg.dynamicSmemBytes = kPrSmem;
-            if (cudaOccupancyMaxActiveClusters(&pairs, tc_decode_pair_kernel, &cfg) != cudaSuccess || pairs <= 0) {
-                cudaGetLastError();
-                pairs = sms / 2;
-            }
-            if (pairs > sms / 2) pairs = sms / 2;
-            pairs_cache[dev].store(pairs, std::memory_order_release);
-        }
-        const int groups = s * H / 128;
-        int r = pairs / groups;
-        const int cap = (kMaxRanges / 2) / groups;
-        if (r > cap) r = cap;
-        return r > 0 ? r : 1;
-    }
     if (ensure_smem_attr(tc_decode64_kernel, kD64Smem, attr64) != cudaSuccess) return 0;
     const int groups = dec_groups(H, s);
     int r = sms / groups;
@@ -263,9 +231,7 @@ int mla_decode_ctas(const mla_dims_t *dims, int s)
 {
     if (check_dims(dims) != MLA_OK || s <= 0) return 0;
     const int H = dims->num_heads;
-    if (use_pair(H, s)) return 2 * decode_ranges(H, s) * (s * H / 128);
-    const int g = dec_groups(H, s);
-    return decode_ranges(H, s) * g;
+    return decode_ranges(H, s) * dec_groups(H, s);
 }
 
 uint64_t mla_kernel_launches(void) { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
@@ -423,23 +389,11 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
     } else {
         const TcWs w = tc_ws(H, s, B);
         if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
-        const bool pr = use_pair(H, s);
-        const int groups = pr ? s * H / 128 : dec_groups(H, s);
+        const int groups = dec_groups(H, s);
         const int ranges = decode_ranges(H, s);
         if (ranges <= 0) return MLA_ERR_CUDA;
-        const uint64_t rows = (uint64_t)num_blocks * kBlock;
-        PairMaps pm;
         CUtensorMap mkv;
-        if (pr) {
-            const uint64_t qrows = (uint64_t)T * H;
-            if (!tmap(&pm.kv_lat, cache, kRow, rows, 1, kRow, 0, 64, kPrT) ||
-                !tmap(&pm.kv_rope, cache, kRow, rows, 1, kRow, 0, 32, kPrT) ||
-                !tmap(&pm.q_lat, q_abs, kRow, qrows, 1, kRow, 0, 64, 128) ||
-                !tmap(&pm.q_rope, q_abs, kRow, qrows, 1, kRow, 0, 32, 128))
-                return MLA_ERR_CUDA;
-        } else if (!tmap(&mkv, cache, kRow, rows, 1, kRow, 0, 64, kT64)) {
-            return MLA_ERR_CUDA;
-        }
+        if (!tmap(&mkv, cache, kRow, (uint64_t)num_blocks * kBlock, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
         if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
         int32_t *plan = (int32_t *)(ws + w.off_plan);
         dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
@@ -466,14 +420,12 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         da.groups = groups;
         // the decode kernel sets itself up while the plan runs, and the
         // combine launches while the decode's last CTAs finish
-        cudaError_t e = pr ? launch_pdl(tc_decode_pair_kernel, dim3(2 * ranges * groups), dim3(kPrThreads),
-                                        kPrSmem, strm, pm, da)
-                           : launch_pdl(tc_decode64_kernel, dim3(ranges * groups), dim3(kD64Threads), kD64Smem,
-                                        strm, mkv, da);
+        cudaError_t e = launch_pdl(tc_decode64_kernel, dim3(ranges * groups), dim3(kD64Threads), kD64Smem, strm,
+                                   mkv, da);
         count_launch();
         if (e != cudaSuccess) return MLA_ERR_CUDA;
-        const int items = combine_items(B, s, H);
-        const int cgrid = items < 4 * sm_count() ? items : 4 * sm_count();
+        const int ctas = combine_ctas(B, s, H);
+        const int cgrid = ctas < 8 * sm_count() ? ctas : 8 * sm_count();
         e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
                        (const float *)da.part_o, (const float *)da.part_lse2, seq_lens, max_blocks, B, s, H,
                        (bf16 *)out_latent, out_lse);

@@ -1,5 +1,5 @@
 // tc_decode64.cuh -- absorbed-MLA decode on tcgen05 tensor cores (sm_100a),
-// one 64-token cache page per tile, two logits-issuing warps.
+// one 64-token cache page per tile, three logits-issuing warps.
 //
 // What it computes (DeepSeek-V2 paper review, sections 2-3): for every query
 // row (query token t of sequence b, head i), softmax_j(scale * q_abs . row_j)
@@ -12,11 +12,11 @@
 // Why this shape on B200: a tcgen05.mma costs a fixed ~34 ns to issue from one
 // thread whatever its size up to M=128, N=128, and M=64 runs at half rate, so
 // the 36 K-steps of one tile's logits take ~1.2 us to issue from one thread.
-// Two warps issue the logits of alternate tiles, each into its own buffer;
-// the P.C MMAs of a tile are issued by the softmax warp that completes its P
-// (no hand-off to another warp):
+// Three warps issue the logits of every third tile, each into its own buffer,
+// so a tile's logits start as soon as its page lands; the P.C MMAs of a tile
+// are issued by the softmax warp that completes its P (no hand-off):
 //
-//   S(k)  = Q C_k^T            M=64, N=64, K=576 (36 steps)   (warp 1 + (k & 1))
+//   S(k)  = Q C_k^T            M=64, N=64, K=576 (36 steps)   (warp 1 + k % 3)
 //   O    += P(k) C_k[:, 0:512]  M=64, N=2 x 256, K=64          (last softmax warp)
 //
 // Each logits buffer has a single issuer and the P.C MMAs are issued in tile
@@ -26,7 +26,7 @@
 //
 // TMEM (512 columns): a 64-row operand occupies one half of each 32-lane
 // quarter (row m at lane 32*(m/16) + m%16, plus 16 for the upper half):
-//   lanes 0-15:  S(even k) (columns 0-63) | S(odd k) (64-127) | Q (128-415, bf16 pairs)
+//   lanes 0-15:  S(k % 3 = 0, 1) (columns 0-127) | Q (128-415, bf16 pairs) | S(k % 3 = 2) (416-479)
 //   lanes 16-31: O (columns 0-511)
 // Q is the A operand of the logits MMAs, read from TMEM; an A operand in TMEM
 // must sit in the same lanes as its accumulator, hence S and Q share a half.
@@ -43,9 +43,9 @@
 //
 // Softmax: warps 4-7, one per TMEM quarter.  Threads i and 16+i of a warp
 // share row 16q+i: each reads half of the row's 64 logits, frees the buffer
-// for S(k+2), and does half of the exp work and half of the row's epilogue.
+// for S(k+3), and does half of the exp work and half of the row's epilogue.
 // Warp q also zeroes its quarter of a ragged tile's latent rows past the
-// sequence end.  Warp 3 has no role.
+// sequence end.
 // Online softmax in the log2 domain with lazy rescaling (O and l are rescaled
 // only when the running max grows by more than 8, a factor 256).
 //
@@ -73,6 +73,7 @@ constexpr int kD64PChunk = 8 * kD64Chunk;         // P of a tile goes where its 
 constexpr int kD64Smem = kD64OffBar + 512 + 1024;                // + alignment slack
 constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-511
 constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
+constexpr uint32_t kD64TmS2 = 416;                // third logits buffer: lanes 0-15, columns 416-479
 constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
 
 __global__ void __launch_bounds__(kD64Threads, 1)
@@ -84,9 +85,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kD64OffBar);
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
     uint64_t *kv_empty = bars + 21;  // [3] P.C MMAs of the stage done -> TMA, softmax
-    uint64_t *q_full = bars + 4;     // softmax (Q of a new sequence in TMEM) -> S issuers
-    uint64_t *s_full = bars + 6;     // [2] S issuer -> softmax (logits buffer b)
-    uint64_t *s_free = bars + 8;     // [2] softmax (buffer b read) -> S issuer
+    // Q of segment n is in TMEM once q_cnt >= 4 (n + 1) (each softmax warp adds
+    // 1 per segment): a count rather than a barrier phase, so that an issuer
+    // with no tile in some segments can never be two phases behind
+    volatile int *q_cnt = reinterpret_cast<volatile int *>(bars + 4);
+    uint64_t *s_full = bars + 26;    // [3] S issuer -> softmax (logits buffer b)
+    uint64_t *s_free = bars + 29;    // [3] softmax (buffer b read) -> S issuer
     int *p_cnt = reinterpret_cast<int *>(bars + 24);  // [3] softmax warps done with P of the stage
     uint64_t *mma_done = bars + 14;  // every MMA-issuing thread at teardown
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
@@ -103,13 +107,13 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kD64Stages; ++i) { sm100::mbar_init(&kv_full[i], 1); sm100::mbar_init(&kv_empty[i], 1); }
-        sm100::mbar_init(q_full, 4);
-        for (int i = 0; i < 2; ++i) {
+        *q_cnt = 0;
+        for (int i = 0; i < 3; ++i) {
             sm100::mbar_init(&s_full[i], 1);
             sm100::mbar_init(&s_free[i], 4);
         }
         for (int i = 0; i < kD64Stages; ++i) p_cnt[i] = 0;
-        sm100::mbar_init(mma_done, 6);
+        sm100::mbar_init(mma_done, 7);
         *abort_flag = 0;
         sm100::fence_mbar_init();
         sm100::prefetch_tensormap(&map_kv);
@@ -179,11 +183,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                         sm100::mbar_wait(&kv_full[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
             }
         }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp >= 1 && warp <= 3) {
         // --------------------------------------------------- logits MMAs
-        // warp 1 takes the even tiles and warp 2 the odd ones, each into its
-        // own logits buffer (columns 64b, b = k & 1), all 36 K steps
+        // warp 1 + b takes the tiles k with k % 3 = b, each into its own
+        // logits buffer, all 36 K steps
         const int b = warp - 1;
+        const uint32_t scol = b < 2 ? 64u * b : kD64TmS2;
         const uint32_t idesc_s = sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
         is.init(seq_start, a.B, lo, hi);
@@ -191,26 +196,24 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         bool ok = true;
         while (ok && is.ok) {
             const int kk = is.k, st = kk % kD64Stages;
-            if ((kk & 1) != b) {
+            if (kk % 3 != b) {
                 is.advance();
                 continue;
             }
             // the Q rows of this tile's sequence are written into TMEM by the
-            // softmax warps; q_full completes once per segment, and its phases
-            // are taken in order, including segments whose tiles all went to
-            // the other warp (a parity wait must not skip a phase)
-            while (ok && q_seg < is.seg) {
-                ++q_seg;
-                ok = sm100::warp_wait(q_full, q_seg & 1, abort_flag, a.err, lim);
+            // softmax warps, which count the segments they have written
+            if (q_seg < is.seg) {
+                ok = wait_count(q_cnt, 4 * (is.seg + 1), abort_flag, a.err, lim);
+                q_seg = is.seg;
             }
             if (!ok) break;
             ok = sm100::warp_wait(&kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
-            if (ok && kk >= 2) ok = sm100::warp_wait(&s_free[b], ((kk >> 1) - 1) & 1, abort_flag, a.err, lim);
+            if (ok && kk >= 3) ok = sm100::warp_wait(&s_free[b], ((kk / 3) - 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
             if (lane == 0) {
                 const uint64_t kd = sm100::desc_kmajor(sm100::smem_u32(stages + st * kD64Stage), 128, sm100::kSw128);
-                const uint32_t d = tmem + b * 64;
+                const uint32_t d = tmem + scol;
 #pragma unroll
                 for (int step = 0; step < 36; ++step) {          // 16-column K steps
                     const uint32_t off = (step >> 2) * kD64Chunk + (step & 3) * 32;
@@ -221,8 +224,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             __syncwarp();
             is.advance();
         }
-    } else if (warp == 3) {
-        // idle: the P.C MMAs are issued by the softmax warp that finishes P last
     } else {
         // -------------------------------------------------------- softmax
         // warp q (0..3) owns group rows [16q, 16q+16): row 16q+i's logits and
@@ -267,7 +268,10 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
             __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(q_full);
+            if (lane == 0) {
+                __threadfence_block();
+                atomicAdd(const_cast<int *>(q_cnt), 1);
+            }
         };
         TileIter it;
         it.init(seq_start, a.B, lo, hi);
@@ -285,16 +289,16 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 nseq = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks);
                 nvis = nseq - a.s + tq + 1;
             }
-            const int sb = k & 1;
-            ok = sm100::warp_wait(&s_full[sb], (k >> 1) & 1, abort_flag, a.err, lim);
+            const int sb = k % 3;
+            ok = sm100::warp_wait(&s_full[sb], (k / 3) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
             // raw logits of row r, columns [32h, 32h+32) (h = 0 for threads 0-15);
-            // then the buffer is handed back for S(k+2)
+            // then the buffer is handed back for S(k+3)
             float x[32];
             {
                 uint32_t sv[32];
-                sm100::tmem_ld16x2_32(lane_base + 64 * sb, sv);
+                sm100::tmem_ld16x2_32(lane_base + (sb < 2 ? 64u * sb : kD64TmS2), sv);
                 sm100::tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(sv[c]);
@@ -461,7 +465,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     sm100::pdl_trigger();   // the combine may start launching
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp == 1 || warp == 2 || warp >= 4) {
+    if (warp >= 1) {
         // every MMA this CTA issued retires before its TMEM is released
         if (lane == 0) sm100::umma_commit(mma_done);
         __syncwarp();

@@ -32,7 +32,15 @@ tests/test_oracle_pins.py, none is "parity unpinned":
   * absorb_q: a NumPy matmul, U^K = [I | 0] returning q^C exactly;
   * up_v, out_proj: a NumPy matmul, U^V = [I | 0] returning the first 128
     latent columns exactly;
-  * the cache accounting figures the review prints (section 4).
+  * the cache accounting figures the review prints (section 4);
+  * e4m3_values, e4m3_encode: the values the OCP FP8 specification prints
+    (1, 448, 2^-6, 2^-9, NaN), torch's own float8_e4m3fn conversion on every
+    code and on in-range values, round-to-nearest-even ties;
+  * quantize_rows: scales equal amax / 448, every code within half a step of
+    x / scale, the largest element of each part maps to 448 exactly;
+  * decode_latent_fp8_rows: bit-identical to decode_latent_rows on a cache of
+    E4M3-representable values with unit scales, and a brute-force NumPy
+    softmax on tiny inputs.
 """
 from __future__ import annotations
 
@@ -72,6 +80,17 @@ def load(path: str):
         [ctypes.c_int] * 7 + [ctypes.c_double, _u16p, ctypes.c_int, _i32p, ctypes.c_int, _i32p,
                               _f64p, ctypes.c_int, _i32p, _f64p, _f64p])
     lib.mla_oracle_decode_latent_rows.restype = ctypes.c_int
+    _u8p = ctypes.POINTER(ctypes.c_uint8)
+    _f32p = ctypes.POINTER(ctypes.c_float)
+    lib.mla_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.mla_oracle_e4m3_value.restype = ctypes.c_double
+    lib.mla_oracle_e4m3_values.argtypes = [ctypes.c_int, _u8p, _f64p]
+    lib.mla_oracle_e4m3_encode_n.argtypes = [ctypes.c_int, _f32p, _u8p]
+    lib.mla_oracle_quantize_rows.argtypes = [ctypes.c_int] * 3 + [_f32p, _u8p, _f32p]
+    lib.mla_oracle_decode_latent_fp8_rows.argtypes = (
+        [ctypes.c_int] * 7 + [_u8p, _f32p, ctypes.c_int, _i32p, ctypes.c_int, _i32p, _f64p, ctypes.c_int,
+                              _i32p, _f64p, _f64p])
+    lib.mla_oracle_decode_latent_fp8_rows.restype = ctypes.c_int
     lib.mla_oracle_up_v.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     lib.mla_oracle_out_proj.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     return lib
@@ -241,6 +260,62 @@ def decode_latent_rows(cache, block_table, seq_lens, s, q_abs, rows=None, block_
     rc = _lib().mla_oracle_decode_latent_rows(
         B, s, H, d_c, d_r, d_h, block_size, float(base), _p(cache, _u16p), num_blocks, _p(bt, _i32p),
         max_blocks, _p(sl, _i32p), _p(q_abs, _f64p), rr.size, _p(rr, _i32p), _p(out, _f64p), _p(lse, _f64p))
+    if rc != 0:
+        raise ValueError("block table entry out of range")
+    return out, lse
+
+
+# ------------------------------------------------------------- FP8 cache
+def e4m3_values(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> their values (float64; NaN for the NaN codes)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _lib().mla_oracle_e4m3_values(c.size, c.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), _p(out, _f64p))
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """float32 values -> nearest E4M3 codes (ties to even, saturating at 448)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _lib().mla_oracle_e4m3_encode_n(x.size, x.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                    out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
+
+
+def quantize_rows(rows, d_c=512):
+    """Cache rows [N][d_c + d_r] (float32) -> (codes uint8 [N][D], scales float32
+    [N][2]): scale = amax / 448 per part (c^KV, k^R), code = E4M3(x / scale)."""
+    r = np.ascontiguousarray(rows, dtype=np.float32)
+    N, D = r.shape
+    codes = np.empty((N, D), np.uint8)
+    scales = np.empty((N, 2), np.float32)
+    _lib().mla_oracle_quantize_rows(N, d_c, D - d_c, r.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                    codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                    scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return codes, scales
+
+
+def decode_latent_fp8_rows(codes, scales, block_table, seq_lens, s, q_abs, rows=None, block_size=64, d_r=64,
+                           d_h=128):
+    """Absorbed decode over the FP8 cache (codes [num_blocks][64][576] uint8,
+    scales [num_blocks][64][2] float32, k^R already rotated): (latent
+    [n_rows][H][d_c], lse [n_rows][H])."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    q_abs = _f64(q_abs)
+    T, H, D = q_abs.shape
+    d_c = D - d_r
+    B = sl.shape[0]
+    num_blocks = codes.size // (block_size * D)
+    max_blocks = bt.shape[-1] if bt.ndim > 1 else bt.size // max(B, 1)
+    rr = _i32(np.arange(T) if rows is None else rows)
+    out = np.zeros((rr.size, H, d_c)); lse = np.zeros((rr.size, H))
+    rc = _lib().mla_oracle_decode_latent_fp8_rows(
+        B, s, H, d_c, d_r, d_h, block_size, codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+        scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), num_blocks, _p(bt, _i32p), max_blocks,
+        _p(sl, _i32p), _p(q_abs, _f64p), rr.size, _p(rr, _i32p), _p(out, _f64p), _p(lse, _f64p))
     if rc != 0:
         raise ValueError("block table entry out of range")
     return out, lse

@@ -412,6 +412,166 @@ int mla_oracle_decode_latent_rows(int B, int s, int H, int d_c, int d_r, int d_h
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------ FP8 cache
+ * Row f1: the latent cache stored in 8-bit floating point.  The pages say the
+ * deployed model keeps its KV cache at about 6 bits per element and its
+ * weights in FP8 (DeepSeek-V2 paper review, sections 4 and 9), and that FP8
+ * values are E4M3 with fine-grained scaling factors (DeepSeek-V3 report
+ * summary, the FP8 training framework).  Reading used here: each cached row
+ * [c^KV | k^R (rotated)] is stored as E4M3 codes with one fp32 scale for its
+ * c^KV part and one for its k^R part, scale = amax / 448 (448 is the largest
+ * finite E4M3 value), code = E4M3(x / scale) rounded to nearest-even and
+ * saturated.  The scale and the quotient are taken in fp32, the precision the
+ * GPU quantizer uses, so both sides make the same integer decision.
+ *
+ * E4M3 (OCP 8-bit floating point): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits.  Exponent 1..15: (-1)^s 2^(e-7) (1 + m/8), except e = 15,
+ * m = 7, which is NaN; exponent 0: (-1)^s 2^-6 (m/8).  No infinities. */
+double mla_oracle_e4m3_value(uint8_t code)
+{
+    const int sgn = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+void mla_oracle_e4m3_values(int n, const uint8_t *codes, double *out)
+{
+    for (int i = 0; i < n; ++i) out[i] = mla_oracle_e4m3_value(codes[i]);
+}
+
+/* Nearest E4M3 code to x, ties to the even code, magnitudes above 448
+ * saturated to 448; found by comparing x with every finite value. */
+uint8_t mla_oracle_e4m3_encode(float x)
+{
+    if (x != x) return 0x7F;
+    const double a = fabs((double)x);
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        const double err = fabs(mla_oracle_e4m3_value((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    if (a > 448.0) best = 0x7E;
+    return (uint8_t)((signbit(x) ? 0x80 : 0) | best);
+}
+
+void mla_oracle_e4m3_encode_n(int n, const float *x, uint8_t *codes)
+{
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < n; ++i) codes[i] = mla_oracle_e4m3_encode(x[i]);
+}
+
+/* Quantizer of the FP8 cache: rows [N][d_c + d_r] fp32 -> codes [N][d_c + d_r]
+ * and scales [N][2] (c^KV part, k^R part); an all-zero part gets scale 1. */
+void mla_oracle_quantize_rows(int N, int d_c, int d_r, const float *rows, uint8_t *codes, float *scales)
+{
+    const int D = d_c + d_r;
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = part ? d_c : 0, c1 = part ? D : d_c;
+            float amax = 0.0f;
+            for (int c = c0; c < c1; ++c) {
+                const float a = fabsf(rows[(size_t)n * D + c]);
+                if (a > amax) amax = a;
+            }
+            const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+            scales[2 * (size_t)n + part] = sc;
+            for (int c = c0; c < c1; ++c)
+                codes[(size_t)n * D + c] = mla_oracle_e4m3_encode(rows[(size_t)n * D + c] / sc);
+        }
+    }
+}
+
+/* Absorbed-form decode over the FP8 cache, every head of a list of rows (the
+ * arithmetic of mla_oracle_decode_latent_rows on dequantized rows):
+ *   c_j = E4M3(code) * scale_c,  k^R_j = E4M3(code) * scale_r (already rotated)
+ *   l_j = (q_abs[0:d_c] . c_j + q_abs[d_c:] . k^R_j) / sqrt(d_h + d_r)
+ *   out = sum_j softmax_j(l) c_j
+ * codes [num_blocks][block_size][d_c+d_r] uint8, scales [num_blocks][block_size][2]
+ * fp32; out [n_rows][H][d_c], lse [n_rows][H].  Returns 0, or -1 if a block
+ * table entry is out of range. */
+int mla_oracle_decode_latent_fp8_rows(int B, int s, int H, int d_c, int d_r, int d_h, int block_size,
+                                      const uint8_t *codes, const float *scales, int num_blocks,
+                                      const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                                      const double *q_abs, int n_rows, const int32_t *rows, double *out,
+                                      double *lse)
+{
+    const int D = d_c + d_r;
+    const double scale = 1.0 / sqrt((double)(d_h + d_r));
+    const int G = 16;
+    const int n_grp = (H + G - 1) / G;
+    int bad = 0;
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int task = 0; task < n_rows * n_grp; ++task) {
+        const int ri = task / n_grp, h0 = (task % n_grp) * G;
+        const int h1 = h0 + G < H ? h0 + G : H, nh = h1 - h0;
+        const int row = rows[ri];
+        const int b = row / s, t = row % s;
+        const int n_vis = seq_lens[b] - s + t + 1;
+        for (int h = h0; h < h1; ++h) {
+            double *o = out + ((size_t)ri * H + h) * d_c;
+            for (int m = 0; m < d_c; ++m) o[m] = 0.0;
+            lse[(size_t)ri * H + h] = -INFINITY;
+        }
+        if (n_vis <= 0) continue;
+        double *score = (double *)malloc(sizeof(double) * (size_t)nh * (size_t)n_vis);
+        double *den = (double *)malloc(sizeof(double) * (size_t)nh);
+        double *x = (double *)malloc(sizeof(double) * (size_t)D);
+        for (int j = 0; j < n_vis; ++j) {
+            const int blk = block_table[(size_t)b * max_blocks + j / block_size];
+            if (blk < 0 || blk >= num_blocks) {
+                bad = 1;
+                for (int h = 0; h < nh; ++h) score[(size_t)h * n_vis + j] = -INFINITY;
+                continue;
+            }
+            const size_t slot = (size_t)blk * block_size + (size_t)(j % block_size);
+            for (int m = 0; m < D; ++m)
+                x[m] = mla_oracle_e4m3_value(codes[slot * D + m]) * (double)scales[2 * slot + (m < d_c ? 0 : 1)];
+            for (int h = 0; h < nh; ++h) {
+                const double *q = q_abs + ((size_t)row * H + h0 + h) * D;
+                double dot = 0.0;
+                for (int m = 0; m < d_c; ++m) dot += q[m] * x[m];
+                for (int m = d_c; m < D; ++m) dot += q[m] * x[m];
+                score[(size_t)h * n_vis + j] = dot * scale;
+            }
+        }
+        for (int h = 0; h < nh; ++h) {
+            double *sc = score + (size_t)h * n_vis;
+            double mx = -INFINITY;
+            for (int j = 0; j < n_vis; ++j) if (sc[j] > mx) mx = sc[j];
+            double dn = 0.0;
+            for (int j = 0; j < n_vis; ++j) { sc[j] = exp(sc[j] - mx); dn += sc[j]; }
+            den[h] = dn;
+            lse[(size_t)ri * H + h0 + h] = mx + log(dn);
+        }
+        for (int j = 0; j < n_vis; ++j) {
+            const int blk = block_table[(size_t)b * max_blocks + j / block_size];
+            if (blk < 0 || blk >= num_blocks) continue;
+            const size_t slot = (size_t)blk * block_size + (size_t)(j % block_size);
+            for (int m = 0; m < d_c; ++m)
+                x[m] = mla_oracle_e4m3_value(codes[slot * D + m]) * (double)scales[2 * slot];
+            for (int h = 0; h < nh; ++h) {
+                const double a = score[(size_t)h * n_vis + j] / den[h];
+                double *o = out + ((size_t)ri * H + h0 + h) * d_c;
+                for (int m = 0; m < d_c; ++m) o[m] += a * x[m];
+            }
+        }
+        free(score); free(den); free(x);
+    }
+    return bad ? -1 : 0;
+}
+
 /* Up-projection (step a7): out_heads[t][i] = U^V_i latent[t][i]
  * latent [T][H][d_c], w_uv [H][d_h][d_c] -> out_heads [T][H][d_h]. */
 void mla_oracle_up_v(int T, int H, int d_h, int d_c, const double *latent,

@@ -1,8 +1,8 @@
 """Index arithmetic of the split-KV plan and the combine kernel, emulated on
 the CPU for every workload (s*H from 16 to 256) and several SM counts: every
 partial slot the combine reads lies inside the workspace's partial area,
-every row it forms is below s*H, and every output element it writes lies
-inside the output.  The emulation restates the loops of dec_plan_kernel and
+every row it forms is below s*H, every output element it writes lies inside
+the output, and every row of every cut sequence is written once.  The emulation restates the loops of dec_plan_kernel and
 dec_combine_kernel (csrc/dec_common.cuh) index for index; the GPU tests then
 check the values."""
 import numpy as np
@@ -10,7 +10,7 @@ import pytest
 
 import mla_workloads as W
 
-COMBINE_ROWS, COMBINE_WARPS, BLOCK = 16, 8, 64
+COMBINE_WARPS, BLOCK = 8, 64
 
 
 def plan(seq_lens, s, max_blocks, ranges, tile=64):
@@ -24,9 +24,6 @@ def plan(seq_lens, s, max_blocks, ranges, tile=64):
 
 def ranges_of(sms, s, H):
     """Ranges per row group, as decode_ranges picks them."""
-    if (s * H) % 128 == 0:
-        groups = s * H // 128
-        return max(1, min(sms // 2 // groups, 74 // groups)), groups
     groups = (s * H + 63) // 64
     return max(1, min(sms // groups, 148 // groups)), groups
 
@@ -38,34 +35,32 @@ def workspace_slots(s, H):
 
 
 def emulate_combine(B, s, H, seq_lens, max_blocks, q, start, grid):
+    """The combine's loops: warp w of CTA blk takes rows blk*8 + w, then
+    strides by grid*8 over the B*s*H (sequence, row) items."""
     rows = s * H
-    per_seq = (rows + COMBINE_ROWS - 1) // COMBINE_ROWS
-    items = B * per_seq
+    items = B * rows
     reads, writes, rows_seen = [], [], set()
     for blk in range(grid):
-        for item in range(blk, items, grid):
-            b, rb = divmod(item, per_seq)
-            a0, a1 = int(start[b]), int(start[b + 1])
-            L = min(max(int(seq_lens[b]), 0), max_blocks * BLOCK)
-            c0 = a0 // q if a1 > a0 else 0
-            c1 = (a1 - 1) // q if a1 > a0 else 0
-            split = a1 > a0 and c0 != c1
-            if not split and L >= s:
-                continue
-            for warp in range(COMBINE_WARPS):
-                for j in range(COMBINE_ROWS // 8):
-                    rr = rb * COMBINE_ROWS + 2 * warp + j
-                    if rr >= rows:
-                        break
-                    t = rr // H
-                    orow = b * rows + rr
-                    rows_seen.add((b, rr))
-                    writes.append((orow * 512, orow * 512 + 32 * 16))   # 32 lanes x 16 columns
-                    if L - s + t + 1 <= 0 or not split:
-                        continue
-                    for c in range(c0, c1 + 1):
-                        slot = 2 * c + (1 if (c == c0 and a0 != c * q) else 0)
-                        reads.append((slot, rr))
+        for warp in range(COMBINE_WARPS):
+            for w in range(blk * COMBINE_WARPS + warp, items, grid * COMBINE_WARPS):
+                b, rr = divmod(w, rows)
+                a0, a1 = int(start[b]), int(start[b + 1])
+                L = min(max(int(seq_lens[b]), 0), max_blocks * BLOCK)
+                c0 = a0 // q if a1 > a0 else 0
+                c1 = (a1 - 1) // q if a1 > a0 else 0
+                split = a1 > a0 and c0 != c1
+                if not split and L >= s:
+                    continue
+                assert rr < rows
+                t = rr // H
+                orow = b * rows + rr
+                rows_seen.add((b, rr))
+                writes.append((orow * 512, orow * 512 + 32 * 16))   # 32 lanes x 16 columns
+                if L - s + t + 1 <= 0 or not split:
+                    continue
+                for c in range(c0, c1 + 1):
+                    slot = 2 * c + (1 if (c == c0 and a0 != c * q) else 0)
+                    reads.append((slot, rr))
     return reads, writes, rows_seen
 
 
@@ -78,7 +73,7 @@ def test_combine_indices_stay_in_bounds(name, sms):
     ranges, groups = ranges_of(sms, cfg.s, cfg.H)
     q, total, start = plan(sl, cfg.s, max_blocks, ranges)
     assert q * ranges >= total                      # every tile lies in some range
-    grid = min(cfg.B * ((cfg.s * cfg.H + 15) // 16), 4 * sms)
+    grid = min((cfg.B * cfg.s * cfg.H + COMBINE_WARPS - 1) // COMBINE_WARPS, 8 * sms)
     reads, writes, rows_seen = emulate_combine(cfg.B, cfg.s, cfg.H, sl, max_blocks, q, start, grid)
     rows = cfg.s * cfg.H
     nslot = workspace_slots(cfg.s, cfg.H)
@@ -92,11 +87,11 @@ def test_combine_indices_stay_in_bounds(name, sms):
 
 
 def test_combine_rows_bound_at_sixteen_rows():
-    """s*H = 16 (the V2-Lite shape): one item per sequence, only warp 0..7's
-    rows 0..15 are formed and none reaches past row 15."""
+    """s*H = 16 (the V2-Lite shape): no row past 15 is formed, and the rows
+    of an empty sequence are still written (zeroed)."""
     sl = np.array([4096, 4096, 100, 0], np.int32)
     q, total, start = plan(sl, 1, 64, ranges=3)
-    reads, writes, rows_seen = emulate_combine(4, 1, 16, sl, 64, q, start, grid=4)
+    reads, writes, rows_seen = emulate_combine(4, 1, 16, sl, 64, q, start, grid=3)
     assert all(rr < 16 for _, rr in reads)
     assert max(r for _, r in rows_seen) == 15
     # the empty sequence's rows are zeroed (written) though it has no partial

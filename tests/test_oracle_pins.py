@@ -588,3 +588,159 @@ def test_decode_latent_rows_closed_forms(oracle_mod):
         mean = c[starts[b]:starts[b + 1]].mean(axis=0)
         np.testing.assert_allclose(lat[b], np.repeat(mean[None], cfg.H, axis=0), rtol=0, atol=1e-14)
         np.testing.assert_allclose(lse[b], np.log(d["seq_lens"][b]), rtol=1e-14)
+
+
+# ------------------------------------------------------------- FP8 cache pins
+def test_e4m3_values_the_specification_prints(oracle_mod):
+    """OCP 8-bit floating point, E4M3: 0x38 = 1, 0x7E = 448 (largest finite),
+    0x08 = 2^-6 (smallest normal), 0x07 = 7/8 * 2^-6 (largest subnormal), 0x01 =
+    2^-9 (smallest subnormal), 0xC0 = -2, 0x7F and 0xFF are NaN, 0x80 = -0."""
+    v = oracle_mod.e4m3_values(np.array([0x38, 0x7E, 0x08, 0x07, 0x01, 0xC0, 0x00, 0x80], np.uint8))
+    assert list(v) == [1.0, 448.0, 2.0 ** -6, 0.875 * 2.0 ** -6, 2.0 ** -9, -2.0, 0.0, -0.0]
+    assert np.isnan(oracle_mod.e4m3_values(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def test_e4m3_matches_torch_on_every_code_and_in_range_values(oracle_mod):
+    """torch's float8_e4m3fn is an independent implementation of the same
+    format: every code decodes to the same value, and in-range floats
+    (|x| <= 448, where torch does not saturate) encode to the same code."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = oracle_mod.e4m3_values(codes)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    rng = np.random.default_rng(40)
+    x = np.concatenate([rng.standard_normal(20000) * 50, rng.standard_normal(20000) * 1e-2,
+                        rng.uniform(-448, 448, 20000), oracle_mod.e4m3_values(codes[ok & (np.abs(ref) <= 448)]),
+                        # exact midpoints between neighbouring values: ties go to the even code
+                        (ref[1:0x7E] + ref[2:0x7F]) / 2]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle_mod.e4m3_encode(x), want)
+
+
+def test_e4m3_encode_saturates_and_rounds_ties_to_even(oracle_mod):
+    codes = oracle_mod.e4m3_encode(np.array([448.0, 449.0, 464.0, 1e6, -1e6, 2.0 ** -10, 1.5 * 2.0 ** -9,
+                                             1.0625, 1.1875], np.float32))
+    # 464 is midway between 448 and the next step (480, not finite): it stays
+    # at the even 448; 2^-10 is midway between 0 and 2^-9: 0 (even);
+    # 1.0625 is midway between 1 (0x38) and 1.125 (0x39): 0x38; 1.1875
+    # between 1.125 (0x39) and 1.25 (0x3A): 0x3A
+    assert list(codes) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x00, 0x02, 0x38, 0x3A]
+
+
+def test_quantize_rows_scales_and_codes(oracle_mod):
+    rng = np.random.default_rng(41)
+    rows = (rng.standard_normal((50, 576)) * rng.uniform(0.01, 30, (50, 1))).astype(np.float32)
+    rows[3, :512] = 0.0                                   # an all-zero part gets scale 1
+    codes, scales = oracle_mod.quantize_rows(rows)
+    amax_c = np.abs(rows[:, :512]).max(1)
+    amax_r = np.abs(rows[:, 512:]).max(1)
+    np.testing.assert_array_equal(scales[:, 0], np.where(amax_c > 0, amax_c / np.float32(448), 1).astype(np.float32))
+    np.testing.assert_array_equal(scales[:, 1], (amax_r / np.float32(448)).astype(np.float32))
+    assert np.all(codes[3, :512] == 0)
+    vals = oracle_mod.e4m3_values(codes)
+    q = rows / np.repeat(scales, [512, 64], axis=1)
+    # every code is the nearest value (within half a step of its neighbours)
+    err = np.abs(vals - q)
+    step = np.maximum(np.abs(vals) * 2.0 ** -3, 2.0 ** -9)
+    assert np.all(err <= step / 2 + 1e-6 * np.abs(q))
+    # the element of largest magnitude lands on +-448
+    i = np.argmax(np.abs(rows[0, :512]))
+    assert abs(vals[0, i]) == 448.0
+
+
+def _fp8_tiny_cache(oracle_mod, cfg, rng, unit_scales=False):
+    """An FP8 cache for a workload: random E4M3-representable latents and
+    rotated keys, pages and table from the workload's paging."""
+    sl = W.seq_lens_of(cfg)
+    table, nphys, _ = W.paging(cfg, sl)
+    tok_seq, tok_pos = W.token_index(sl)
+    codes_tok = rng.integers(0, 0x7F, size=(tok_seq.size, 576)).astype(np.uint8)   # finite, non-negative
+    codes_tok |= (rng.integers(0, 2, size=codes_tok.shape).astype(np.uint8) << 7)  # signs
+    codes_tok[:, :] = np.where((codes_tok & 0x7F) == 0x7F, 0x7E, codes_tok)
+    scales_tok = np.ones((tok_seq.size, 2), np.float32) if unit_scales else \
+        rng.uniform(1e-3, 1e-2, (tok_seq.size, 2)).astype(np.float32)
+    codes = np.zeros((nphys, 64, 576), np.uint8)
+    scales = np.zeros((nphys, 64, 2), np.float32)
+    blk = table[tok_seq, tok_pos // 64]
+    codes[blk, tok_pos % 64] = codes_tok
+    scales[blk, tok_pos % 64] = scales_tok
+    return sl, table, codes, scales, codes_tok, scales_tok, tok_seq
+
+
+def test_decode_fp8_equals_bf16_decode_on_representable_values(oracle_mod):
+    """With unit scales and no RoPE part (zero codes, which rotate to zero in
+    the bf16 path too), an FP8 cache of E4M3 values holds exactly the values
+    of a bf16 cache: the two decodes agree bit for bit."""
+    rng = np.random.default_rng(42)
+    cfg = W.MLAConfig("f8", B=3, s=2, H=20, L=0, paged=True, seed=43, d_model=64, seq_lens=(130, 2, 65))
+    sl, table, codes, scales, codes_tok, _, tok_seq = _fp8_tiny_cache(oracle_mod, cfg, rng, unit_scales=True)
+    codes[..., 512:] = 0
+    vals = oracle_mod.e4m3_values(codes).astype(np.float32)        # exact in bf16 (3-bit mantissa)
+    bf = W.f32_to_bf16_bits(vals)
+    assert np.array_equal(W.bf16_bits_to_f32(bf), vals)
+    q = oracle_mod.bf16_to_f64(W.make_q_abs(cfg))
+    a, la = oracle_mod.decode_latent_fp8_rows(codes, scales, table, sl, cfg.s, q)
+    b, lb = oracle_mod.decode_latent_rows(bf, table, sl, cfg.s, q)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_decode_fp8_brute_force_tiny(oracle_mod):
+    """A textbook NumPy softmax over the dequantized rows (codes times their
+    part's scale, the RoPE key taken as already rotated)."""
+    rng = np.random.default_rng(44)
+    cfg = W.MLAConfig("f8b", B=2, s=1, H=3, L=0, paged=True, seed=45, d_model=64, seq_lens=(70, 9))
+    sl, table, codes, scales, codes_tok, scales_tok, tok_seq = _fp8_tiny_cache(oracle_mod, cfg, rng)
+    q = rng.standard_normal((cfg.T, cfg.H, 576))
+    got, lse = oracle_mod.decode_latent_fp8_rows(codes, scales, table, sl, cfg.s, q)
+    x = oracle_mod.e4m3_values(codes_tok) * np.repeat(scales_tok.astype(np.float64), [512, 64], axis=1)
+    starts = np.concatenate([[0], np.cumsum(sl)])
+    for b in range(cfg.B):
+        X = x[starts[b]:starts[b + 1]]
+        for h in range(cfg.H):
+            l = X @ q[b, h] / math.sqrt(192.0)
+            p = np.exp(l - l.max())
+            np.testing.assert_allclose(got[b, h], (p / p.sum()) @ X[:, :512], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(lse[b, h], l.max() + math.log(p.sum()), rtol=1e-13)
+
+
+FP8_MUTATIONS = {
+    "exponent_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "subnormal_scale": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "ties_to_odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    "wrong_max": ("const float sc = amax > 0.0f ? amax / 448.0f : 1.0f;",
+                  "const float sc = amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "rope_part_with_latent_scale": ("* (double)scales[2 * slot + (m < d_c ? 0 : 1)];", "* (double)scales[2 * slot];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FP8_MUTATIONS))
+def test_planted_fp8_mistakes_are_caught(oracle_mod, tmp_path, name):
+    """One plausible mistake in the FP8 routines of a copy of the oracle must
+    make one of the FP8 pins fail."""
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle_mod.__file__), "mla_oracle.c")).read()
+    old, new = FP8_MUTATIONS[name]
+    assert src.count(old) == 1, name
+    mutant = tmp_path / "m.c"
+    mutant.write_text(src.replace(old, new, 1))
+    so = tmp_path / "m.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(mutant), "-lm"], check=True)
+    saved = oracle_mod._LIB
+    oracle_mod._LIB = oracle_mod.load(str(so))
+    pins = (test_e4m3_values_the_specification_prints, test_e4m3_matches_torch_on_every_code_and_in_range_values,
+            test_e4m3_encode_saturates_and_rounds_ties_to_even, test_quantize_rows_scales_and_codes,
+            test_decode_fp8_brute_force_tiny)
+    try:
+        caught = False
+        for pin in pins:
+            try:
+                pin(oracle_mod)
+            except AssertionError:
+                caught = True
+                break
+        assert caught, f"mutation {name} was not caught"
+    finally:
+        oracle_mod._LIB = saved
