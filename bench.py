@@ -180,20 +180,45 @@ class Step:
         self.ws = torch.empty(M.mla_decode_workspace_size(self.dims, cfg.B, cfg.s, self.max_blocks * 64),
                               dtype=torch.uint8, device="cuda")
         self.stream = torch.cuda.current_stream()
+        # the append and the absorption are independent: the absorption runs
+        # on a side stream, forked from and joined back into the main one
+        self.side = torch.cuda.Stream()
+        self.ev_fork, self.ev_join = torch.cuda.Event(), torch.cuda.Event()
         torch.cuda.synchronize()
 
-    def run(self, inp=None, dec_events=None, out=None):
+    def run(self, inp=None, dec_events=None, out=None, serial_events=None):
+        """One step.  With `serial_events` (five events) every call runs on the
+        main stream, one after the other, with an event between calls."""
         M, x = self.M, (inp if inp is not None else self.dev)
-        M.mla_append_cache(self.dims, x["h"], self.w_dkv, self.w_kr, x["app_seq"], x["app_pos"],
-                           self.block_table, self.cache)
-        M.mla_absorb_q(self.dims, x["q_nope"], x["q_rope"], x["q_pos"], self.w_uk, self.q_abs)
+        main = self.torch.cuda.current_stream()
+        ev = serial_events
+        if ev is not None:
+            ev[0].record(main)
+            M.mla_append_cache(self.dims, x["h"], self.w_dkv, self.w_kr, x["app_seq"], x["app_pos"],
+                               self.block_table, self.cache)
+            ev[1].record(main)
+            M.mla_absorb_q(self.dims, x["q_nope"], x["q_rope"], x["q_pos"], self.w_uk, self.q_abs)
+            ev[2].record(main)
+        else:
+            self.ev_fork.record(main)
+            self.side.wait_event(self.ev_fork)
+            with self.torch.cuda.stream(self.side):
+                M.mla_absorb_q(self.dims, x["q_nope"], x["q_rope"], x["q_pos"], self.w_uk, self.q_abs)
+                self.ev_join.record(self.side)
+            M.mla_append_cache(self.dims, x["h"], self.w_dkv, self.w_kr, x["app_seq"], x["app_pos"],
+                               self.block_table, self.cache)
+            main.wait_event(self.ev_join)
         if dec_events is not None:
-            dec_events[0].record(self.stream)
+            dec_events[0].record(main)
         M.mla_decode(self.dims, self.q_abs, self.cache, self.block_table, self.seq_lens, self.cfg.s,
                      self.lat, self.lse, self.ws, flags=self.flags)
         if dec_events is not None:
-            dec_events[1].record(self.stream)
+            dec_events[1].record(main)
+        if ev is not None:
+            ev[3].record(main)
         M.mla_up_v(self.dims, self.lat, self.w_uv, self.out if out is None else out)
+        if ev is not None:
+            ev[4].record(main)
 
 
 def run_ours(args):
@@ -264,7 +289,14 @@ def run_ours(args):
         st.run(dec_events=dec[k])
     barrier()
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in dec]))
+    # the same calls one after the other on one stream, timed call by call
+    ser = [[E(enable_timing=True) for _ in range(5)] for _ in range(n_dec)]
+    for k in range(n_dec):
+        st.run(serial_events=ser[k])
+    barrier()
+    parts = [float(np.mean([e[i].elapsed_time(e[i + 1]) for e in ser])) for i in range(4)]
     ms, dec_ms = max_over_ranks([ms, dec_ms], world, "cuda")
+    parts = max_over_ranks(parts, world, "cuda")
     if graph is not None:
         del graph
         barrier()
@@ -358,6 +390,10 @@ def run_ours(args):
                                  if (cfg.name == "v2" and not args.simple and DECODE_DRAM_BYTES_PER_TOKEN)
                                  else None),
                      "peak_source": pk["source"] + (" burst" if bound == "tensor" else "")},
+        "step_calls_us": {"note": "each call timed on its own (stream launches, one after the other); "
+                                  "the timed step overlaps the append with the absorption on a side stream",
+                          "append": parts[0] * 1e3, "absorb": parts[1] * 1e3, "decode": parts[2] * 1e3,
+                          "up_v": parts[3] * 1e3},
         "e2e": {"value": tok / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": int(launches),
@@ -365,6 +401,8 @@ def run_ours(args):
     }
     if not args.no_per_config and world == 1:
         line["per_config"] = per_config(M, [n for n in ("tiny", "v2lite", "v2", "longctx", "mtp")])
+    if not args.no_prefill and world == 1:
+        line["prefill"] = prefill_bench(M)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     print(json.dumps(line), flush=True)
@@ -435,6 +473,89 @@ def per_config(M, names, iters=30):
             r["warm_l2_us"] = timed(False) * 1e6
         out[name] = r
         del cache, q, lat, lse, ws, bt, slt
+        torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------ expanded-form prefill
+PREFILL_WORKLOADS = {
+    "prompt4k": dict(B=1, s=4096, L=4096, H=128, seed=2001,
+                     describe="DeepSeek-V2-shaped prompt prefill: B=1, s=L=4096, H=128"),
+    "chunk1k_ctx8k": dict(B=1, s=1024, L=8192, H=128, seed=2002,
+                          describe="chunked prefill: the last 1024 of 8192 tokens, H=128"),
+    "v2lite_prompt4k": dict(B=4, s=4096, L=4096, H=16, seed=2003,
+                            describe="DeepSeek-V2-Lite-shaped prompt prefill: B=4, s=L=4096, H=16"),
+}
+
+
+def prefill_flops(B, s, L, H, d_c=512, d_r=64, d_h=128):
+    """(attention, expansion) flops of one mla_prefill call: 2 (d_h + d_r)
+    for the logit and 2 d_h for the weighted sum per visible (query, key,
+    head); 2 d_h d_c per row and head for each of K^C and V^C over the
+    call's B * round_up(L, 128) expanded rows."""
+    vis = s * (L - s) + s * (s + 1) // 2
+    att = 2.0 * B * H * vis * ((d_h + d_r) + d_h)
+    lpad = (L + 127) // 128 * 128
+    exp_ = 2.0 * 2.0 * B * lpad * H * d_h * d_c
+    return att, exp_
+
+
+def prefill_bench(M, names=tuple(PREFILL_WORKLOADS), iters=10):
+    """mla_prefill on each workload: CUDA-event time of the whole call
+    (gather + two expansion GEMMs + attention; mean of `iters` calls after 3
+    warm-ups, each call preceded by a 256 MB L2 flush), its TFLOP/s and the
+    fraction of the measured dense bf16 peak (the call is tensor-bound).
+    Inputs are seeded torch draws on the device with the workloads'
+    distributions (cache, q^C, q^R N(0,1); U^K, U^V N(0,1/512)); the cache
+    is paged through a random block permutation."""
+    import torch
+    out = {}
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    E = torch.cuda.Event
+    for name in names:
+        w = PREFILL_WORKLOADS[name]
+        B, s, L, H = w["B"], w["s"], w["L"], w["H"]
+        g = torch.Generator(device="cuda")
+        g.manual_seed(w["seed"])
+        nblk = (L + 63) // 64
+        nphys = B * nblk
+        cache = torch.randn((nphys, 64, 576), generator=g, device="cuda").to(torch.bfloat16)
+        bt = torch.randperm(nphys, generator=g, device="cuda").to(torch.int32).view(B, nblk).contiguous()
+        sl = torch.full((B,), L, dtype=torch.int32, device="cuda")
+        q_nope = torch.randn((B * s, H, 128), generator=g, device="cuda").to(torch.bfloat16)
+        q_rope = torch.randn((B * s, H, 64), generator=g, device="cuda").to(torch.bfloat16)
+        q_pos = (torch.arange(s, dtype=torch.int32, device="cuda") + (L - s)).repeat(B).contiguous()
+        w_uk = (torch.randn((H, 128, 512), generator=g, device="cuda") * 512 ** -0.5).to(torch.bfloat16)
+        w_uv = (torch.randn((H, 128, 512), generator=g, device="cuda") * 512 ** -0.5).to(torch.bfloat16)
+        dims = M.dims(H)
+        o = torch.empty((B * s, H, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B * s, H), dtype=torch.float32, device="cuda")
+        ws = torch.empty(M.mla_prefill_workspace_size(dims, B, s, L), dtype=torch.uint8, device="cuda")
+        call = lambda: M.mla_prefill(dims, q_nope, q_rope, q_pos, w_uk, w_uv, cache, bt, sl, s, L, o, lse, ws)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        n0 = M.mla_kernel_launches()
+        ts = []
+        for _ in range(iters):
+            flush.fill_(1)
+            a, b = E(enable_timing=True), E(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        launches = (M.mla_kernel_launches() - n0) // iters
+        t = float(np.mean([x.elapsed_time(y) for x, y in ts])) / 1e3
+        att, exp_ = prefill_flops(B, s, L, H)
+        achieved = (att + exp_) / t / 1e12
+        out[name] = {"workload": w["describe"], "us": t * 1e6, "tokens_per_s": B * s / t,
+                     "attention_gflop": att / 1e9, "expansion_gflop": exp_ / 1e9, "tflops": achieved,
+                     "bound": "tensor", "peak_tflops": pk["tc"], "roofline_frac": achieved / pk["tc"],
+                     "launches_per_call": int(launches), "l2": "flushed before each call",
+                     "error_word": M.mla_decode_error(ws)}
+        del cache, bt, sl, q_nope, q_rope, q_pos, w_uk, w_uv, o, lse, ws
         torch.cuda.empty_cache()
     return out
 
@@ -535,6 +656,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the number of sequences (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip timing the decode of every workload")
+    ap.add_argument("--no-prefill", action="store_true", help="skip timing the expanded-form prefill")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the prefill workloads")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps on the stream, not as a graph")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -542,6 +665,12 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.prefill_only:
+        import torch
+        import head_latent_attention_10_b200 as M
+        M.load_library()
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps({"prefill": prefill_bench(M)}), flush=True)
     else:
         run_ours(args)
 

@@ -22,7 +22,8 @@ MLA_SYNC_CHECK, MLA_FORCE_SIMPLE, MLA_DEBUG_STALL = 0x1, 0x2, 0x100
 
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",
-            "mla_kernel_launches", "mla_decode_ctas", "mla_decode_noalloc")
+            "mla_kernel_launches", "mla_decode_ctas", "mla_decode_noalloc",
+            "mla_prefill_workspace_size", "mla_prefill")
 
 
 class MLAError(RuntimeError):
@@ -34,13 +35,18 @@ class MLAError(RuntimeError):
 class mla_dims_t(ctypes.Structure):
     _fields_ = [("num_heads", ctypes.c_int32), ("d_c", ctypes.c_int32), ("d_rope", ctypes.c_int32),
                 ("d_head", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("rope_base", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("rope_base", ctypes.c_float),
+                ("rope_scaling", ctypes.c_float), ("rope_original_ctx", ctypes.c_int32),
+                ("rope_yarn_alpha", ctypes.c_float), ("rope_yarn_beta", ctypes.c_float)]
 
 
 def dims(num_heads: int, softmax_scale: float = 0.0, rope_base: float = 10000.0, d_c: int = 512,
-         d_rope: int = 64, d_head: int = 128, block_size: int = 64) -> mla_dims_t:
-    """Shape descriptor; softmax_scale <= 0 selects 1/sqrt(d_head + d_rope)."""
-    return mla_dims_t(num_heads, d_c, d_rope, d_head, block_size, softmax_scale, rope_base)
+         d_rope: int = 64, d_head: int = 128, block_size: int = 64, rope_scaling: float = 0.0,
+         rope_original_ctx: int = 0, rope_yarn_alpha: float = 0.0, rope_yarn_beta: float = 0.0) -> mla_dims_t:
+    """Shape descriptor; softmax_scale <= 0 selects 1/sqrt(d_head + d_rope);
+    rope_scaling > 1 selects YaRN-scaled RoPE frequencies."""
+    return mla_dims_t(num_heads, d_c, d_rope, d_head, block_size, softmax_scale, rope_base, rope_scaling,
+                      rope_original_ctx, rope_yarn_alpha, rope_yarn_beta)
 
 
 _LIB = None
@@ -58,8 +64,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     D = ctypes.POINTER(mla_dims_t)
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_status_string.argtypes = [_i]
-    lib.mla_append_cache.argtypes = [D, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp]
-    lib.mla_append_latent.argtypes = [D, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _vp]
+    _f = ctypes.c_float
+    lib.mla_append_cache.argtypes = [D, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _f, _vp, _vp]
+    lib.mla_append_latent.argtypes = [D, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _vp, _i, _vp, _f, _vp, _vp]
     lib.mla_absorb_q.argtypes = [D, _vp, _vp, _vp, _vp, _i, _vp, _vp]
     lib.mla_decode_workspace_size.argtypes = [D, _i, _i, _i]
     lib.mla_decode_workspace_size.restype = ctypes.c_size_t
@@ -70,11 +77,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_up_v.argtypes = [D, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]
     lib.mla_decode_ctas.argtypes = [D, _i]
     lib.mla_decode_ctas.restype = _i
+    lib.mla_prefill_workspace_size.argtypes = [D, _i, _i, _i]
+    lib.mla_prefill_workspace_size.restype = ctypes.c_size_t
+    lib.mla_prefill.argtypes = [D, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp,
+                                _vp, ctypes.c_size_t, ctypes.c_uint32, _vp]
     lib.mla_kernel_launches.argtypes = []
     lib.mla_kernel_launches.restype = ctypes.c_uint64
     for name in EXPORTED:
         if name not in ("mla_status_string", "mla_decode_workspace_size", "mla_kernel_launches",
-                        "mla_decode_ctas"):
+                        "mla_decode_ctas", "mla_prefill_workspace_size"):
             getattr(lib, name).restype = _i
     _LIB = lib
     return lib
@@ -105,21 +116,25 @@ def mla_status_string(status: int) -> str:
     return load_library().mla_status_string(status).decode()
 
 
-def mla_append_cache(d, h, w_dkv, w_kr, seq_idx, pos, block_table, cache, err_word=None, stream=None):
-    """c^KV = W^DKV h and k^R = RoPE(W^KR h, pos) written to the paged cache."""
+def mla_append_cache(d, h, w_dkv, w_kr, seq_idx, pos, block_table, cache, err_word=None, stream=None,
+                     kv_norm_weight=None, kv_norm_eps=1e-6):
+    """c^KV = W^DKV h (RMS-normalised with kv_norm_weight if given) and
+    k^R = RoPE(W^KR h, pos) written to the paged cache."""
     T, d_model = h.shape
     _check(load_library().mla_append_cache(
         ctypes.byref(d), _ptr(h), T, d_model, _ptr(w_dkv), _ptr(w_kr), _ptr(seq_idx), _ptr(pos),
         _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(cache), cache.shape[0],
-        _ptr(err_word), _stream(stream)), "mla_append_cache")
+        _ptr(kv_norm_weight), kv_norm_eps, _ptr(err_word), _stream(stream)), "mla_append_cache")
 
 
-def mla_append_latent(d, c_kv, k_rope, seq_idx, pos, block_table, cache, err_word=None, stream=None):
-    """[c_kv | RoPE(k_rope, pos)] written to the paged cache."""
+def mla_append_latent(d, c_kv, k_rope, seq_idx, pos, block_table, cache, err_word=None, stream=None,
+                      kv_norm_weight=None, kv_norm_eps=1e-6):
+    """[c_kv (RMS-normalised with kv_norm_weight if given) | RoPE(k_rope, pos)]
+    written to the paged cache."""
     _check(load_library().mla_append_latent(
         ctypes.byref(d), _ptr(c_kv), _ptr(k_rope), c_kv.shape[0], _ptr(seq_idx), _ptr(pos),
         _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(cache), cache.shape[0],
-        _ptr(err_word), _stream(stream)), "mla_append_latent")
+        _ptr(kv_norm_weight), kv_norm_eps, _ptr(err_word), _stream(stream)), "mla_append_latent")
 
 
 def mla_absorb_q(d, q_nope, q_rope, q_pos, w_uk, q_abs, stream=None):
@@ -172,6 +187,22 @@ def mla_decode_error(workspace, clear: bool = False, stream=None) -> int:
     _check(load_library().mla_decode_error(_ptr(workspace), ctypes.byref(v), int(clear),
                                            _stream(stream)), "mla_decode_error")
     return int(v.value)
+
+
+def mla_prefill_workspace_size(d, B: int, s: int, max_seq_len: int) -> int:
+    return int(load_library().mla_prefill_workspace_size(ctypes.byref(d), B, s, max_seq_len))
+
+
+def mla_prefill(d, q_nope, q_rope, q_pos, w_uk, w_uv, cache, block_table, seq_lens, s, max_seq_len,
+                out, out_lse, workspace, flags: int = 0, stream=None):
+    """Expanded-form attention of the last s tokens of each sequence over its
+    cached latents; writes the per-head outputs out [B*s][H][d_head]."""
+    B = seq_lens.shape[0]
+    _check(load_library().mla_prefill(
+        ctypes.byref(d), _ptr(q_nope), _ptr(q_rope), _ptr(q_pos), _ptr(w_uk), _ptr(w_uv), _ptr(cache),
+        cache.shape[0], _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, s, max_seq_len,
+        _ptr(out), _ptr(out_lse), _ptr(workspace), workspace.numel() * workspace.element_size(), flags,
+        _stream(stream)), "mla_prefill")
 
 
 def mla_up_v(d, latent, w_uv, out_heads, w_o=None, out_model=None, stream=None):

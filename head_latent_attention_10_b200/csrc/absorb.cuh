@@ -11,9 +11,9 @@
 // 64-row K chunks, eight 64-column N chunks) with TMA in one go; warp 1
 // issues 16 tcgen05 MMAs (M=128, N=256, K=16) into two accumulators (TMEM
 // columns 0-255 and 256-511); warps 2-9 read them back, two warps per TMEM
-// lane quarter (thread = token row, half of the 512 columns each), and the
-// first of each pair also turns the row's RoPE query.  No TMA load uses
-// cluster multicast.
+// lane quarter (thread = token row, half of the 512 columns each, and half of
+// the row's RoPE pairs) into a swizzled staging tile, which one thread stores
+// with TMA.  No TMA load uses cluster multicast.
 #pragma once
 
 #include "dec_common.cuh"
@@ -26,12 +26,14 @@ constexpr int kAbBChunk = 64 * 64 * 2;            // one U^K box: 64 K rows x 64
 constexpr int kAbB = 8 * kAbBChunk;               // one K chunk of U^K_i: 64 x 512 (64 KB)
 constexpr int kAbOffB = 2 * kAbA;                 // 32 KB
 constexpr int kAbOffBar = kAbOffB + 2 * kAbB;     // 163,840
+constexpr int kAbStageChunk = 128 * 128;          // one 64-column chunk of the output tile (16 KB)
 constexpr int kAbSmem = kAbOffBar + 512 + 1024;   // barriers, the RoPE table (256 B), alignment slack
 
 __global__ void __launch_bounds__(kAbThreads, 1)
 absorb_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_uk,
+              const __grid_constant__ CUtensorMap map_out,
               const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos, int T, int H,
-              bf16 *__restrict__ q_abs, double base, uint32_t *err, unsigned long long limit_ns)
+              bf16 *__restrict__ q_abs, const RopeTable rope, uint32_t *err, unsigned long long limit_ns)
 {
     extern __shared__ uint8_t ab_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(ab_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -52,8 +54,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         sm100::prefetch_tensormap(&map_q);
         sm100::prefetch_tensormap(&map_uk);
     }
-    if (warp == 9)  // theta_k = base^(-2k/64), k = 0..31 (the RoPE pairs)
-        theta[lane] = pow(base, -2.0 * (double)lane / (double)kDr);
+    if (warp == 9)  // the frequency of RoPE pair k = lane
+        theta[lane] = rope.theta[lane];
     if (warp == 1) {
         sm100::tmem_alloc(tmem_slot, 512);
         sm100::tmem_relinquish();
@@ -95,38 +97,51 @@ absorb_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         }
     } else {
         // epilogue: warp w (2..9) reads TMEM lane quarter w % 4 (thread = token
-        // row), columns [256 h, 256 h + 256) with h = (w - 2) / 4
+        // row r), columns [256 h, 256 h + 256) with h = (w - 2) / 4, and writes
+        // its bf16 values into a staging copy of the output tile in the (now
+        // free) input buffers: nine 64-column chunks of [128 rows][128 B]
+        // with 128-byte swizzle (16-byte unit u of row r at u ^ (r & 7)),
+        // chunk 8 being the RoPE part.  One thread then stores the chunks with
+        // TMA (rows past T are not written), so the global writes are whole
+        // lines instead of one 16-byte piece of 32 different rows per warp
+        // instruction.
         const int qd = warp & 3, h = (warp - 2) >> 2;
-        const int t = m0 + 32 * qd + lane;
+        const int r = 32 * qd + lane, t = m0 + r;
         const bool ok = sm100::warp_wait(done, 0, abort_flag, err, limit_ns);
         sm100::tc_fence_after();
-        bf16 *row = q_abs + ((long long)t * H + head) * kRow;
-        if (ok) {
+        auto stage_unit = [&](int chunk, int u, uint4 v) {
+            *reinterpret_cast<uint4 *>(smem + chunk * kAbStageChunk + r * 128 + ((u ^ (r & 7)) << 4)) = v;
+        };
 #pragma unroll 1
-            for (int c = 0; c < 256; c += 32) {
-                uint32_t v[32];
-                sm100::tmem_ld16(sm100::tmem_addr(tmem + 256 * h, 32 * qd, c), v);
-                sm100::tmem_ld16(sm100::tmem_addr(tmem + 256 * h, 32 * qd, c + 16), v + 16);
-                sm100::tmem_wait_ld();
-                if (t < T) {
-                    uint4 *d = reinterpret_cast<uint4 *>(row + 256 * h + c);
+        for (int c = 0; c < 4; ++c) {
+            uint32_t v[64];
+            if (ok) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        d[e] = make_uint4(pack_bf162(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                                          pack_bf162(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                                          pack_bf162(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                                          pack_bf162(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
-                }
+                for (int q = 0; q < 4; ++q)
+                    sm100::tmem_ld16(sm100::tmem_addr(tmem + 256 * h, 32 * qd, 64 * c + 16 * q), v + 16 * q);
+                sm100::tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = 0u;
             }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                stage_unit(4 * h + c, u,
+                           make_uint4(pack_bf162(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
+                                      pack_bf162(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                                      pack_bf162(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                                      pack_bf162(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7]))));
         }
+        // RoPE pairs [16h, 16h+16) of the row's query: the angle p*theta_k is
+        // formed and reduced to [-pi, pi] in double precision (at positions up
+        // to 2^17 an fp32 product would be off by ~1e-2 rad), then its sine
+        // and cosine are taken in fp32
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = 0u;
         if (t < T) {
-            // RoPE pairs [16h, 16h+16) of the row's query: the angle p*theta_k
-            // is formed and reduced to [-pi, pi] in double precision (at
-            // positions up to 2^17 an fp32 product would be off by ~1e-2 rad),
-            // then its sine and cosine are taken in fp32
             const __nv_bfloat162 *src = reinterpret_cast<const __nv_bfloat162 *>(q_rope + ((long long)t * H + head) * kDr);
             const double p = q_pos ? (double)q_pos[t] : 0.0;
-            uint32_t o[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const int k = 16 * h + e;
@@ -141,9 +156,15 @@ absorb_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
                     o[e] = pack_bf162(x.x, x.y);
                 }
             }
-            uint4 *d = reinterpret_cast<uint4 *>(row + kDc + 32 * h);
+        }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) d[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        for (int u = 0; u < 4; ++u) stage_unit(8, 4 * h + u, make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]));
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 epilogue warps
+        if (warp == 2 && lane == 0) {
+            for (int j = 0; j < 9; ++j) sm100::tma_store_3d(&map_out, smem + j * kAbStageChunk, 64 * j, head, m0);
+            sm100::tma_store_commit();
+            sm100::tma_store_wait_read();
         }
     }
     sm100::tc_fence_before();

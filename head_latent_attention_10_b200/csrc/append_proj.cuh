@@ -10,7 +10,7 @@
 // columns [64n, 64n+64) (n = 8: the 64 RoPE columns, from W^KR) of tokens
 // [128m, 128m+128) over the K slice [z Ks, (z+1) Ks), Ks = d_model / 8.  The
 // 8 K slices of a tile form a cluster.  Each CTA streams its slice of h and W
-// through a 4-stage TMA ring into an M=128, N=64 tcgen05 accumulator, then
+// through a 6-stage TMA ring into an M=128, N=64 tcgen05 accumulator, then
 // sends row r of its fp32 partial to CTA r / 16 of the cluster (distributed
 // shared memory), which sums the 8 partials of its 16 rows in slice order
 // (the result does not depend on timing), turns the RoPE pairs and writes
@@ -24,12 +24,12 @@
 namespace mla {
 
 constexpr int kApSlices = 8;                      // K slices = cluster size
-constexpr int kApStages = 4;
+constexpr int kApStages = 6;
 constexpr int kApThreads = 192;
 constexpr int kApA = 128 * 64 * 2;                // h chunk: 128 tokens x 64 (16 KB)
 constexpr int kApB = 64 * 64 * 2;                 // W chunk: 64 outputs x 64 (8 KB)
 constexpr int kApStage = kApA + kApB;
-constexpr int kApOffRed = kApStages * kApStage;                  // 98,304
+constexpr int kApOffRed = kApStages * kApStage;                  // 147,456
 constexpr int kApRed = kApSlices * 16 * 64 * 4;                  // 32 KB: [slice][16 rows][64] fp32
 constexpr int kApOffBar = kApOffRed + kApRed;
 constexpr int kApSmem = kApOffBar + 256 + 1024;
@@ -38,7 +38,7 @@ struct AppendArgs {
     bf16 *cache;
     const int32_t *seq_idx, *pos, *block_table;
     int T, K, num_seqs, max_blocks, num_blocks;
-    double base;
+    RopeTable rope;
     uint32_t *err;
     unsigned long long limit_ns;
 };
@@ -199,7 +199,7 @@ append_proj_kernel(const __grid_constant__ CUtensorMap map_h, const __grid_const
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float y0, y1;
-                        rope_pair(o[2 * e], o[2 * e + 1], p, c8 / 2 + e, kDr, a.base, &y0, &y1);
+                        rope_turn(o[2 * e], o[2 * e + 1], p, a.rope.theta[c8 / 2 + e], &y0, &y1);
                         o[2 * e] = y0;
                         o[2 * e + 1] = y1;
                     }

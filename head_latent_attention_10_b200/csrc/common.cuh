@@ -31,18 +31,35 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits)
 
 __device__ __forceinline__ float bf2f(bf16 v) { return __bfloat162float(v); }
 
-// RoPE of one pair (x0, x1) = (x[2k], x[2k+1]) at position pos: turn by
-// pos * base^(-2k/d_r).  The angle is formed in double precision: at
-// positions up to 2^17 an fp32 angle would be off by ~1e-2 rad.
-__device__ __forceinline__ void rope_pair(float x0, float x1, int pos, int k, int d_r,
-                                          double base, float *y0, float *y1)
+// The frequency of each RoPE pair k = (x[2k], x[2k+1]), k < d_r / 2: base^(-2k/d_r)
+// for plain RoPE, or its YaRN interpolation (computed on the host per call).
+struct RopeTable {
+    double theta[kDr / 2];
+};
+
+// RoPE of one pair (x0, x1) at position pos: turn by pos * theta.  The angle is
+// formed in double precision: at positions up to 2^17 an fp32 angle would be
+// off by ~1e-2 rad.
+__device__ __forceinline__ void rope_turn(float x0, float x1, int pos, double theta, float *y0, float *y1)
 {
-    const double theta = pow(base, -2.0 * (double)k / (double)d_r);
     const double ang = (double)pos * theta;
     double sn, cs;
     sincos(ang, &sn, &cs);
     *y0 = (float)((double)x0 * cs - (double)x1 * sn);
     *y1 = (float)((double)x0 * sn + (double)x1 * cs);
+}
+
+// Root mean square normalisation factor of a latent row, from the sum of its
+// squares: 1 / sqrt(ss / d_c + eps).
+__device__ __forceinline__ float rms_inv(float ss, float eps)
+{
+    return 1.0f / sqrtf(ss / (float)kDc + eps);
+}
+
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
 }
 
 // 16-byte vector of 8 bf16

@@ -114,11 +114,6 @@ __device__ __forceinline__ bool wait_count(volatile int *cnt, int target, volati
     return ok != 0;
 }
 
-__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
-{
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
 
 __device__ __forceinline__ void fence_proxy_async_smem()
 {

@@ -15,6 +15,7 @@
 #include "k_simple.cuh"
 #include "tc_decode64.cuh"
 #include "tc_gemm.cuh"
+#include "tc_prefill.cuh"
 #include "tmap.cuh"
 
 using namespace mla;
@@ -37,6 +38,9 @@ mla_status_t check_dims(const mla_dims_t *d)
     if (d->d_c != kDc || d->d_rope != kDr || d->d_head != kDh || d->block_size != kBlock)
         return MLA_ERR_UNSUPPORTED;
     if (d->num_heads < 16 || d->num_heads > 128 || d->num_heads % 16 != 0) return MLA_ERR_UNSUPPORTED;
+    if (d->rope_scaling > 1.f && d->rope_yarn_beta > 0.f &&
+        d->rope_yarn_beta <= (d->rope_yarn_alpha > 0.f ? d->rope_yarn_alpha : 1.f))
+        return MLA_ERR_INVALID_ARG;
     return MLA_OK;
 }
 
@@ -48,6 +52,33 @@ inline float softmax_scale(const mla_dims_t *d)
 inline double rope_base(const mla_dims_t *d)
 {
     return d->rope_base > 0.f ? (double)d->rope_base : 10000.0;
+}
+
+// The frequency of each RoPE pair k: theta_k = base^(-2k/d_r), or with YaRN
+// scaling s > 1 (DeepSeek-V2 paper review, long-context passage: scale 40
+// over the 4K pre-training context) the NTK-by-parts interpolation: pair k
+// makes r_k = L0 theta_k / (2 pi) turns over the original context L0; with
+// the ramp g = clamp((r_k - alpha) / (beta - alpha), 0, 1) its frequency is
+// (1 - g) theta_k / s + g theta_k.
+RopeTable rope_table(const mla_dims_t *d)
+{
+    RopeTable t;
+    const double base = rope_base(d), s = (double)d->rope_scaling;
+    const double L0 = d->rope_original_ctx > 0 ? (double)d->rope_original_ctx : 4096.0;
+    const double alpha = d->rope_yarn_alpha > 0.f ? (double)d->rope_yarn_alpha : 1.0;
+    const double beta = d->rope_yarn_beta > 0.f ? (double)d->rope_yarn_beta : 32.0;
+    const double pi = 3.14159265358979323846;
+    for (int k = 0; k < kDr / 2; ++k) {
+        const double th = pow(base, -2.0 * (double)k / (double)kDr);
+        if (s <= 1.0) {
+            t.theta[k] = th;
+            continue;
+        }
+        double g = (L0 * th / (2.0 * pi) - alpha) / (beta - alpha);
+        g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+        t.theta[k] = (1.0 - g) * th / s + g * th;
+    }
+    return t;
 }
 
 inline mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
@@ -114,17 +145,19 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
     return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
 }
 
-template <int BN, bool kBmn, class Epi>
+// C = A B on tcgen05; `c` is the output tensor map of the staged (TMA store)
+// epilogue, unused by the others.
+template <int BN, bool kBmn, class Epi, bool kAshared = false>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
-                           uint32_t *err, cudaStream_t st)
+                           uint32_t *err, cudaStream_t st, const CUtensorMap *c = nullptr)
 {
     using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kAshared>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
     if (e != cudaSuccess) return e;
     dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
-    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, M, N, K, epi, err, kWaitLimitNs);
+    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, c ? *c : a, M, N, K, epi, err, kWaitLimitNs);
     count_launch();
     return cudaGetLastError();
 }
@@ -186,6 +219,26 @@ TcWs tc_ws(int H, int s, int B)
     return w;
 }
 
+// Prefill workspace: [error word][gathered rows [B Lpad][576]][rotated q^R
+// [B s][H][64]][K^C [B Lpad][H][128]][V^C [B Lpad][H][128]]
+struct PfWs {
+    size_t off_rows, off_qr, off_kc, off_vc, total;
+    int lpad;
+};
+
+PfWs pf_ws(int H, int B, int s, int max_seq_len)
+{
+    PfWs w;
+    w.lpad = (max_seq_len + 127) / 128 * 128;
+    const size_t rows = (size_t)B * w.lpad;
+    w.off_rows = kWsAlign;
+    w.off_qr = align_up(w.off_rows + rows * kRow * 2, kWsAlign);
+    w.off_kc = align_up(w.off_qr + (size_t)B * s * H * kDr * 2, kWsAlign);
+    w.off_vc = align_up(w.off_kc + rows * H * kDh * 2, kWsAlign);
+    w.total = align_up(w.off_vc + rows * H * kDh * 2, kWsAlign);
+    return w;
+}
+
 int sm_count()
 {
     static std::atomic<int> sms_cache[kMaxDevices];
@@ -223,6 +276,45 @@ void *noalloc_scratch()
     return symbol_address(g_noalloc_scratch, addr);
 }
 
+// The projection half of mla_append_cache: c^KV = W^DKV h and k^R =
+// RoPE(W^KR h) written as bf16 rows to the tokens' page slots.
+mla_status_t append_project(const mla_dims_t *dims, const void *h, int T, int d_model, const void *w_dkv,
+                            const void *w_kr, const int32_t *seq_idx, const int32_t *pos,
+                            const int32_t *block_table, int num_seqs, int max_blocks, void *cache,
+                            int num_blocks, uint32_t *err_word, cudaStream_t s)
+{
+    if (d_model % (64 * kApSlices) == 0) {
+        // K split over a cluster of CTAs, partials reduced on chip, one launch
+        CUtensorMap mh, md, mr;
+        if (!tmap(&mh, h, d_model, T, 1, d_model, 0, 64, 128) ||
+            !tmap(&md, w_dkv, d_model, kDc, 1, d_model, 0, 64, 64) ||
+            !tmap(&mr, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
+            return MLA_ERR_CUDA;
+        static std::atomic<bool> attr_set[kMaxDevices];
+        if (ensure_smem_attr(append_proj_kernel, kApSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
+        AppendArgs aa{(bf16 *)cache, seq_idx, pos, block_table, T, d_model, num_seqs, max_blocks, num_blocks,
+                      rope_table(dims), err_word, kWaitLimitNs};
+        append_proj_kernel<<<dim3(9, (T + 127) / 128, kApSlices), kApThreads, kApSmem, s>>>(mh, md, mr, aa);
+        count_launch();
+        return cuda_status(cudaGetLastError());
+    }
+    // other widths: one pass over K per 128-token tile
+    CUtensorMap ma, mb1, mb2;
+    if (!tmap(&ma, h, d_model, T, 1, d_model, 0, 64, 128) ||
+        !tmap(&mb1, w_dkv, d_model, kDc, 1, d_model, 0, 64, 256) ||
+        !tmap(&mb2, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
+        return MLA_ERR_CUDA;
+    // c^KV = W^DKV h  (columns 0..511 of the row)
+    TcEpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, 0,
+                  rope_table(dims), err_word};
+    if (launch_tc_gemm<256, false>(ma, mb1, T, kDc, d_model, 1, e, err_word, s) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    // k^R = RoPE(W^KR h)  (columns 512..575)
+    TcEpiAppend e2{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, kDc, 1,
+                   rope_table(dims), nullptr};
+    return cuda_status(launch_tc_gemm<64, false>(ma, mb2, T, kDr, d_model, 1, e2, err_word, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -252,7 +344,8 @@ const char *mla_status_string(mla_status_t s)
 mla_status_t mla_append_latent(const mla_dims_t *dims, const void *c_kv, const void *k_rope, int T,
                                const int32_t *seq_idx, const int32_t *pos,
                                const int32_t *block_table, int num_seqs, int max_blocks, void *cache,
-                               int num_blocks, uint32_t *err_word, void *stream)
+                               int num_blocks, const void *kv_norm_weight, float kv_norm_eps,
+                               uint32_t *err_word, void *stream)
 {
     mla_status_t st = check_dims(dims);
     if (st != MLA_OK) return st;
@@ -260,10 +353,11 @@ mla_status_t mla_append_latent(const mla_dims_t *dims, const void *c_kv, const v
     if (T == 0) return MLA_OK;
     if (!c_kv || !k_rope || !seq_idx || !pos || !block_table || !cache) return MLA_ERR_INVALID_ARG;
     if (!aligned16(c_kv) || !aligned16(cache) || ((uintptr_t)k_rope & 3u)) return MLA_ERR_INVALID_ARG;
+    if (kv_norm_weight && (!aligned16(kv_norm_weight) || !(kv_norm_eps >= 0.f))) return MLA_ERR_INVALID_ARG;
     const int threads = 256, per = threads / 32;
     append_latent_kernel<<<(T + per - 1) / per, threads, 0, as_stream(stream)>>>(
         (const bf16 *)c_kv, (const bf16 *)k_rope, T, seq_idx, pos, block_table, num_seqs, max_blocks,
-        (bf16 *)cache, num_blocks, rope_base(dims), err_word);
+        (bf16 *)cache, num_blocks, rope_table(dims), (const bf16 *)kv_norm_weight, kv_norm_eps, err_word);
     count_launch();
     return cuda_status(cudaGetLastError());
 }
@@ -271,8 +365,8 @@ mla_status_t mla_append_latent(const mla_dims_t *dims, const void *c_kv, const v
 mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int d_model,
                               const void *w_dkv, const void *w_kr, const int32_t *seq_idx,
                               const int32_t *pos, const int32_t *block_table, int num_seqs,
-                              int max_blocks, void *cache, int num_blocks, uint32_t *err_word,
-                              void *stream)
+                              int max_blocks, void *cache, int num_blocks, const void *kv_norm_weight,
+                              float kv_norm_eps, uint32_t *err_word, void *stream)
 {
     mla_status_t st = check_dims(dims);
     if (st != MLA_OK) return st;
@@ -282,37 +376,18 @@ mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int 
     if (!h || !w_dkv || !w_kr || !seq_idx || !pos || !block_table || !cache) return MLA_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr) || !aligned16(cache))
         return MLA_ERR_INVALID_ARG;
+    if (kv_norm_weight && (!aligned16(kv_norm_weight) || !(kv_norm_eps >= 0.f))) return MLA_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
-    if (d_model % (64 * kApSlices) == 0) {
-        // K split over a cluster of CTAs, partials reduced on chip, one launch
-        CUtensorMap mh, md, mr;
-        if (!tmap(&mh, h, d_model, T, 1, d_model, 0, 64, 128) ||
-            !tmap(&md, w_dkv, d_model, kDc, 1, d_model, 0, 64, 64) ||
-            !tmap(&mr, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
-            return MLA_ERR_CUDA;
-        static std::atomic<bool> attr_set[kMaxDevices];
-        if (ensure_smem_attr(append_proj_kernel, kApSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
-        AppendArgs aa{(bf16 *)cache, seq_idx, pos, block_table, T, d_model, num_seqs, max_blocks, num_blocks,
-                      rope_base(dims), err_word, kWaitLimitNs};
-        append_proj_kernel<<<dim3(9, (T + 127) / 128, kApSlices), kApThreads, kApSmem, s>>>(mh, md, mr, aa);
-        count_launch();
-        return cuda_status(cudaGetLastError());
-    }
-    // other widths: one pass over K per 128-token tile
-    CUtensorMap ma, mb1, mb2;
-    if (!tmap(&ma, h, d_model, T, 1, d_model, 0, 64, 128) ||
-        !tmap(&mb1, w_dkv, d_model, kDc, 1, d_model, 0, 64, 256) ||
-        !tmap(&mb2, w_kr, d_model, kDr, 1, d_model, 0, 64, 64))
-        return MLA_ERR_CUDA;
-    // c^KV = W^DKV h  (columns 0..511 of the row)
-    TcEpiAppend e{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, 0, 0,
-                  rope_base(dims), err_word};
-    if (launch_tc_gemm<256, false>(ma, mb1, T, kDc, d_model, 1, e, err_word, s) != cudaSuccess)
-        return MLA_ERR_CUDA;
-    // k^R = RoPE(W^KR h)  (columns 512..575)
-    TcEpiAppend e2{(bf16 *)cache, seq_idx, pos, block_table, num_seqs, max_blocks, num_blocks, kDc, 1,
-                   rope_base(dims), nullptr};
-    return cuda_status(launch_tc_gemm<64, false>(ma, mb2, T, kDr, d_model, 1, e2, err_word, s));
+    const mla_status_t pst = append_project(dims, h, T, d_model, w_dkv, w_kr, seq_idx, pos, block_table, num_seqs,
+                                            max_blocks, cache, num_blocks, err_word, s);
+    if (pst != MLA_OK || !kv_norm_weight) return pst;
+    // RMSNorm of the latent rows just written (their columns come from
+    // different CTAs of the projection, so the row's norm is taken after it)
+    latent_rmsnorm_kernel<<<(T + 7) / 8, 256, 0, s>>>(T, seq_idx, pos, block_table, num_seqs, max_blocks,
+                                                      (bf16 *)cache, num_blocks, (const bf16 *)kv_norm_weight,
+                                                      kv_norm_eps);
+    count_launch();
+    return cuda_status(cudaGetLastError());
 }
 
 mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void *q_rope,
@@ -329,14 +404,16 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
     cudaStream_t s = as_stream(stream);
     // per head i: q_abs[:, i, 0:512] = q_nope[:, i, :] (T x 128) . U^K_i (128 x 512),
     // and the RoPE part, in one launch
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo;
     if (!tmap(&ma, q_nope, kDh, T, H, (uint64_t)H * kDh, kDh, 64, 128) ||
-        !tmap(&mb, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64))
+        !tmap(&mb, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64) ||
+        !make_tmap_3d(&mo, q_abs, kRow, H, T, (uint64_t)kRow * 2, (uint64_t)H * kRow * 2, 64, 1, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))   // q_abs as {576, H, T}: box 64 columns x 1 head x 128 tokens
         return MLA_ERR_CUDA;
     static std::atomic<bool> attr_set[kMaxDevices];
     if (ensure_smem_attr(absorb_kernel, kAbSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
-    absorb_kernel<<<dim3(H, (T + 127) / 128), kAbThreads, kAbSmem, s>>>(ma, mb, (const bf16 *)q_rope, q_pos, T, H,
-                                                                         (bf16 *)q_abs, rope_base(dims), nullptr,
+    absorb_kernel<<<dim3(H, (T + 127) / 128), kAbThreads, kAbSmem, s>>>(ma, mb, mo, (const bf16 *)q_rope, q_pos, T, H,
+                                                                         (bf16 *)q_abs, rope_table(dims), nullptr,
                                                                          kWaitLimitNs);
     count_launch();
     return cuda_status(cudaGetLastError());
@@ -487,12 +564,14 @@ mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const v
     const int H = dims->num_heads;
     cudaStream_t s = as_stream(stream);
     // per head i: out[:, i, :] = latent[:, i, :] (T x 512) . (U^V_i)^T (512 x 128)
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo;
     if (!tmap(&ma, latent, kDc, T, H, (uint64_t)H * kDc, kDc, 64, 128) ||
-        !tmap(&mb, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128))
+        !tmap(&mb, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128) ||
+        !make_tmap_3d(&mo, out_heads, kDh, H, T, (uint64_t)kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))   // out_heads as {128, H, T}
         return MLA_ERR_CUDA;
-    TcEpiStore e{(bf16 *)out_heads, kDh, (long long)H * kDh};
-    if (launch_tc_gemm<128, false>(ma, mb, T, kDh, kDc, H, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_tc_gemm<128, false>(ma, mb, T, kDh, kDc, H, TcEpiTmaStore{}, nullptr, s, &mo) != cudaSuccess)
+        return MLA_ERR_CUDA;
     if (w_o) {
         // out_model = out_heads (T x H*128) . W^O^T
         const int K = H * kDh;
@@ -502,6 +581,110 @@ mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const v
         TcEpiStore e2{(bf16 *)out_model, 0, d_model};
         if (launch_tc_gemm<256, false>(ma2, mb2, T, d_model, K, 1, e2, nullptr, s) != cudaSuccess)
             return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+size_t mla_prefill_workspace_size(const mla_dims_t *dims, int B, int s, int max_seq_len)
+{
+    if (check_dims(dims) != MLA_OK || B < 0 || s <= 0 || max_seq_len < s) return 0;
+    return pf_ws(dims->num_heads, B, s, max_seq_len).total;
+}
+
+mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void *q_rope, const int32_t *q_pos,
+                         const void *w_uk, const void *w_uv, const void *cache, int num_blocks,
+                         const int32_t *block_table, int max_blocks, const int32_t *seq_lens, int B, int s,
+                         int max_seq_len, void *out, float *out_lse, void *workspace, size_t ws_bytes,
+                         uint32_t flags, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (B < 0 || s <= 0 || num_blocks < 0 || max_blocks < 0 || max_seq_len < s) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    if (num_blocks == 0 || max_blocks == 0) return MLA_ERR_INVALID_ARG;
+    if (!q_nope || !q_rope || !w_uk || !w_uv || !cache || !block_table || !seq_lens || !out)
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(cache) ||
+        !aligned16(out))
+        return MLA_ERR_INVALID_ARG;
+    if (!workspace) return MLA_ERR_WORKSPACE;
+    const int H = dims->num_heads;
+    const PfWs w = pf_ws(H, B, s, max_seq_len);
+    if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+    const long long rows_total = (long long)B * w.lpad;
+    if (rows_total > (1ll << 31) - 1 || (long long)B * s * H > (1ll << 31) - 1) return MLA_ERR_UNSUPPORTED;
+    const int M = (int)rows_total;
+    cudaStream_t strm = as_stream(stream);
+    char *ws = (char *)workspace;
+    uint32_t *err = (uint32_t *)ws;
+    bf16 *rows = (bf16 *)(ws + w.off_rows), *q_rot = (bf16 *)(ws + w.off_qr);
+    bf16 *kc = (bf16 *)(ws + w.off_kc), *vc = (bf16 *)(ws + w.off_vc);
+    const long long cap_blocks = (long long)max_blocks * kBlock;
+    const int l_cap = cap_blocks < max_seq_len ? (int)cap_blocks : max_seq_len;
+
+    // tensor maps: the expansion GEMMs (rows x U^K_i^T, rows x U^V_i^T, one
+    // activation matrix against per-head weights) and the attention
+    CUtensorMap ma, muk, muv, mkc, mvc;
+    if (!tmap(&ma, rows, kDc, M, 1, kRow, 0, 64, 128) ||
+        !tmap(&muk, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128) ||
+        !tmap(&muv, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128) ||
+        !make_tmap_3d(&mkc, kc, kDh, H, M, kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_3d(&mvc, vc, kDh, H, M, kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return MLA_ERR_CUDA;
+    PrefillMaps pm;
+    {
+        const uint64_t qdims[4] = {(uint64_t)kDh, (uint64_t)H, (uint64_t)s, (uint64_t)B};
+        const uint64_t qstr[3] = {(uint64_t)kDh * 2, (uint64_t)H * kDh * 2, (uint64_t)s * H * kDh * 2};
+        const uint64_t rdims[4] = {(uint64_t)kDr, (uint64_t)H, (uint64_t)s, (uint64_t)B};
+        const uint64_t rstr[3] = {(uint64_t)kDr * 2, (uint64_t)H * kDr * 2, (uint64_t)s * H * kDr * 2};
+        const uint32_t box[4] = {64, 1, 128, 1};
+        if (!make_tmap_4d(&pm.qc, q_nope, qdims, qstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_4d(&pm.qr, q_rot, rdims, rstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_4d(&pm.out, out, qdims, qstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_3d(&pm.kr, rows, kRow, M, 1, kRow * 2, (uint64_t)M * kRow * 2, 64, 128, 1,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+            return MLA_ERR_CUDA;
+        pm.kc = mkc;
+        pm.vc = mvc;
+    }
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
+    {
+        const long long work = rows_total * (kRow / 8) + (long long)B * s * H * (kDr / 2);
+        long long blocks = (work + 255) / 256;
+        if (blocks > 8ll * sm_count()) blocks = 8ll * sm_count();
+        prefill_prepare_kernel<<<(int)blocks, 256, 0, strm>>>((const bf16 *)cache, num_blocks, block_table,
+                                                              max_blocks, seq_lens, B, s, H, w.lpad, l_cap, rows,
+                                                              (const bf16 *)q_rope, q_pos, q_rot, rope_table(dims),
+                                                              err);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+    if (launch_tc_gemm<128, false, TcEpiTmaStore, true>(ma, muk, M, kDh, kDc, H, TcEpiTmaStore{}, err, strm,
+                                                         &mkc) != cudaSuccess ||
+        launch_tc_gemm<128, false, TcEpiTmaStore, true>(ma, muv, M, kDh, kDc, H, TcEpiTmaStore{}, err, strm,
+                                                         &mvc) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    PrefillArgs pa;
+    pa.seq_lens = seq_lens;
+    pa.s = s;
+    pa.H = H;
+    pa.lpad = w.lpad;
+    pa.l_cap = l_cap;
+    pa.scale_log2 = softmax_scale(dims) * kLog2e;
+    pa.out_lse = out_lse;
+    pa.err = err;
+    pa.limit_ns = kWaitLimitNs;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    if (ensure_smem_attr(tc_prefill_kernel, kPfSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
+    tc_prefill_kernel<<<dim3((s + 255) / 256, H, B), kPfThreads, kPfSmem, strm>>>(pm, pa);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (flags & MLA_SYNC_CHECK) {
+        uint32_t h = 0;
+        if (cudaMemcpyAsync(&h, err, sizeof h, cudaMemcpyDeviceToHost, strm) != cudaSuccess ||
+            cudaStreamSynchronize(strm) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (h) return MLA_ERR_DEVICE;
     }
     return MLA_OK;
 }

@@ -9,8 +9,10 @@
 // with tcgen05.ld (one TMEM lane = one output row per thread) and hand 16
 // columns at a time to the epilogue functor.
 //
-// A is K-major (rows of K contiguous).  B is either K-major (B^T stored
-// row-major, e.g. a weight [N][K]) or MN-major (B stored [K][N]).
+// A is K-major (rows of K contiguous); with kAshared every batch entry z uses
+// batch entry 0 of A (one activation matrix against per-head weights).  B is
+// either K-major (B^T stored row-major, e.g. a weight [N][K]) or MN-major (B
+// stored [K][N]).
 // Tensor maps are 3-D: A {K, M, Z}, B K-major {K, N, Z}, B MN-major {N, K, Z}.
 #pragma once
 
@@ -31,10 +33,11 @@ struct GemmSmem {
     static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
 };
 
-template <int BN, bool kBmn, class Epi>
+template <int BN, bool kBmn, class Epi, bool kAshared = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, int M,
-               int N, int K, Epi epi, uint32_t *err, unsigned long long limit_ns)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+               const __grid_constant__ CUtensorMap mapC, int M, int N, int K, Epi epi, uint32_t *err,
+               unsigned long long limit_ns)
 {
     using S = GemmSmem<BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -82,7 +85,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 uint8_t *b = a + S::A;
                 sm100::mbar_arrive_expect_tx(&full[s], S::STAGE);
                 const int kx = kb * 64;
-                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, z);
+                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, kAshared ? 0 : z);
                 if (kBmn) {
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
@@ -126,7 +129,41 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         const bool ok = sm100::warp_wait(done, 0, abort_flag, err, limit_ns);
         sm100::tc_fence_after();
         const int m = m0 + q * 32 + lane;
-        if (ok) {
+        if constexpr (Epi::kStaged) {
+            // bf16 tile staged in the drained ring as 64-column chunks of
+            // [128 rows][128 B] (128-byte swizzle), stored with TMA by one
+            // thread: whole lines rather than 32 rows' pieces per instruction
+            const int r = q * 32 + lane;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t v[32];
+                if (ok) {
+                    sm100::tmem_ld16(sm100::tmem_addr(tmem, q * 32, c), v);
+                    sm100::tmem_ld16(sm100::tmem_addr(tmem, q * 32, c + 16), v + 16);
+                    sm100::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                uint8_t *chunk = smem + (c / 64) * 16384;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int uu = ((c % 64) / 8) + u;
+                    *reinterpret_cast<uint4 *>(chunk + r * 128 + ((uu ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf162(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
+                                   pack_bf162(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                                   pack_bf162(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                                   pack_bf162(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
+            if (warp == 2 && lane == 0) {
+                for (int c = 0; c < BN; c += 64) sm100::tma_store_3d(&mapC, smem + (c / 64) * 16384, n0 + c, z, m0);
+                sm100::tma_store_commit();
+                sm100::tma_store_wait_read();
+            }
+        } else if (ok) {
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 uint32_t r[16];
@@ -149,8 +186,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 }
 
 // ------------------------------------------------------------- epilogues
+// bf16 output stored with TMA from a staged tile through the kernel's output
+// tensor map, which covers the output as {N, Z, M} (columns, batch entry,
+// rows) with box {64, 1, 128}.
+struct TcEpiTmaStore {
+    static constexpr bool kStaged = true;
+    __device__ void operator()(int, int, int, const float *) const {}
+};
+
 // 16 consecutive outputs -> bf16 at base + z*bs + m*rs + n (32-byte aligned).
 struct TcEpiStore {
+    static constexpr bool kStaged = false;
     bf16 *base;
     long long bs, rs;
     __device__ void operator()(int z, int m, int n, const float *v) const
@@ -168,11 +214,12 @@ struct TcEpiStore {
 // Append: token m's projected columns go to its cache slot; with `rope` the
 // 16 columns are RoPE dims n..n+15 (8 pairs) and are turned first.
 struct TcEpiAppend {
+    static constexpr bool kStaged = false;
     bf16 *cache;
     const int32_t *seq_idx, *pos, *block_table;
     int num_seqs, max_blocks, num_blocks, col0;
     int rope;
-    double base;
+    RopeTable tab;
     uint32_t *err;
     __device__ void operator()(int, int m, int n, const float *v) const
     {
@@ -185,7 +232,7 @@ struct TcEpiAppend {
         for (int i = 0; i < 16; ++i) o[i] = v[i];
         if (rope) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) rope_pair(v[2 * i], v[2 * i + 1], p, n / 2 + i, kDr, base, &o[2 * i], &o[2 * i + 1]);
+            for (int i = 0; i < 8; ++i) rope_turn(v[2 * i], v[2 * i + 1], p, tab.theta[n / 2 + i], &o[2 * i], &o[2 * i + 1]);
         }
         uint4 pk[2];
         __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(pk);

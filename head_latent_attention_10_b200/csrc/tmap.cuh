@@ -33,8 +33,9 @@ inline EncodeTiledFn encode_fn()
 
 struct TmapKey {
     const void *ptr;
-    uint64_t dims[3], strides[2];
-    uint32_t box[3];
+    uint32_t rank;
+    uint64_t dims[4], strides[3];
+    uint32_t box[4];
     int swizzle;
     bool operator==(const TmapKey &o) const { return memcmp(this, &o, sizeof *this) == 0; }
 };
@@ -45,21 +46,26 @@ inline CUtensorMapSwizzle swizzle_for(uint32_t inner_bytes)
                               : (inner_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// bf16 tensor of rank 3: dims innermost first (elements), strides of dims 1
-// and 2 in bytes, box in elements.  Out-of-range elements read as zero.
-inline bool make_tmap_3d(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw)
+// bf16 tensor of rank 3 or 4: dims innermost first (elements), strides of
+// dims 1.. in bytes, box in elements.  Out-of-range elements read as zero and
+// are not written by stores.
+inline bool make_tmap_nd(CUtensorMap *out, const void *ptr, uint32_t rank, const uint64_t *dims,
+                         const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw)
 {
     static std::mutex mu;
     static TmapKey keys[64];
     static CUtensorMap maps[64];
     static int used = 0, next = 0;
+    if (rank < 1 || rank > 4) return false;
     TmapKey k;
     memset(&k, 0, sizeof k);
     k.ptr = ptr;
-    k.dims[0] = d0; k.dims[1] = d1; k.dims[2] = d2;
-    k.strides[0] = s1; k.strides[1] = s2;
-    k.box[0] = b0; k.box[1] = b1; k.box[2] = b2;
+    k.rank = rank;
+    for (uint32_t i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+        if (i + 1 < rank) k.strides[i] = strides[i];
+    }
     k.swizzle = (int)sw;
     {
         std::lock_guard<std::mutex> g(mu);
@@ -71,12 +77,15 @@ inline bool make_tmap_3d(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_
     }
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t gdim[3] = {d0, d1, d2};
-    cuuint64_t gstr[2] = {s1, s2};
-    cuuint32_t box[3] = {b0, b1, b2};
-    cuuint32_t estr[3] = {1, 1, 1};
+    cuuint64_t gdim[4], gstr[3];
+    cuuint32_t cbox[4], estr[4] = {1, 1, 1, 1};
+    for (uint32_t i = 0; i < rank; ++i) {
+        gdim[i] = k.dims[i];
+        cbox[i] = k.box[i];
+        if (i + 1 < rank) gstr[i] = k.strides[i];
+    }
     CUtensorMap m;
-    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), gdim, gstr, box, estr,
+    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), gdim, gstr, cbox, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
@@ -87,6 +96,20 @@ inline bool make_tmap_3d(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_
     if (used < 64) ++used;
     *out = m;
     return true;
+}
+
+inline bool make_tmap_3d(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw)
+{
+    const uint64_t dims[3] = {d0, d1, d2}, strides[2] = {s1, s2};
+    const uint32_t box[3] = {b0, b1, b2};
+    return make_tmap_nd(out, ptr, 3, dims, strides, box, sw);
+}
+
+inline bool make_tmap_4d(CUtensorMap *out, const void *ptr, const uint64_t (&dims)[4], const uint64_t (&strides)[3],
+                         const uint32_t (&box)[4], CUtensorMapSwizzle sw)
+{
+    return make_tmap_nd(out, ptr, 4, dims, strides, box, sw);
 }
 
 }  // namespace mla

@@ -22,9 +22,9 @@
  *     bit patterns), row-major, contiguous, 16-byte aligned.
  *   - Every pointer is caller-owned DEVICE memory unless stated otherwise.
  *     No call allocates device memory (no cudaMalloc, no allocating library
- *     routine).  mla_decode keeps its scratch in the caller's workspace;
- *     mla_append_cache, mla_append_latent, mla_absorb_q and mla_up_v need
- *     none.  One call, mla_decode_noalloc, uses a fixed file-scope device
+ *     routine).  mla_decode and mla_prefill keep their scratch in the
+ *     caller's workspace; mla_append_cache, mla_append_latent, mla_absorb_q
+ *     and mla_up_v need none.  One call, mla_decode_noalloc, uses a fixed file-scope device
  *     array inside the library instead (MLA_NOALLOC_SCRATCH_BYTES, one per
  *     device, held until the process exits); calls of it that may overlap on
  *     one device race on that array (see its notes).
@@ -92,8 +92,21 @@ typedef struct {
     int32_t d_rope;      /* RoPE key / query width, 64 */
     int32_t d_head;      /* per-head content width, 128 */
     int32_t block_size;  /* tokens per cache block, 64 */
-    float softmax_scale; /* <= 0 selects 1/sqrt(d_head + d_rope) */
+    float softmax_scale; /* <= 0 selects 1/sqrt(d_head + d_rope); a caller
+                            using YaRN passes its attention temperature here */
     float rope_base;     /* RoPE base; <= 0 selects 10000 */
+    /* YaRN frequency scaling of RoPE [DeepSeek-V2 paper review, long-context
+     * passage: the 4K pre-training context extended with YaRN, scale 40].
+     * With rope_scaling = s > 1, pair k (base frequency theta_k = base^(-2k/d_rope))
+     * makes r_k = L0 theta_k / (2 pi) turns over the original context L0; with
+     * the ramp g = clamp((r_k - alpha) / (beta - alpha), 0, 1) it turns at
+     * (1 - g) theta_k / s + g theta_k.  Used by every call that rotates (the
+     * appends for k^R, mla_absorb_q for q^R).  rope_scaling <= 1: plain RoPE.
+     * beta must exceed alpha (MLA_ERR_INVALID_ARG otherwise). */
+    float rope_scaling;        /* s; <= 1 selects plain RoPE */
+    int32_t rope_original_ctx; /* L0; <= 0 selects 4096 */
+    float rope_yarn_alpha;     /* alpha; <= 0 selects 1 */
+    float rope_yarn_beta;      /* beta; <= 0 selects 32 */
 } mla_dims_t;
 
 /* Human-readable name of a status code (static storage). */
@@ -113,6 +126,11 @@ const char *mla_status_string(mla_status_t status);
  *   seq_idx, pos [T] int32                (device)
  *   block_table  [num_seqs][max_blocks] int32 (device)
  *   cache        [num_blocks][block_size][d_c+d_rope] bf16, written in place
+ *   kv_norm_weight  optional [d_c] bf16 RMSNorm weight w; when given, the
+ *                latent row is stored as c / sqrt(mean(c^2) + kv_norm_eps) * w
+ *                (the RMSNorm after the compressed latent, DeepSeek-V2 paper
+ *                review, section 2), taken on the bf16 projection output.
+ *                NULL: no normalisation.  kv_norm_eps must be >= 0.
  *   err_word     optional device uint32; bits MLA_DEVERR_* are OR-ed in for
  *                tokens whose slot is invalid (those tokens are not written)
  * d_model must be a positive multiple of 64.  T = 0 is a no-op.
@@ -125,20 +143,23 @@ mla_status_t mla_append_cache(const mla_dims_t *dims, const void *h, int T, int 
                               const void *w_dkv, const void *w_kr,
                               const int32_t *seq_idx, const int32_t *pos,
                               const int32_t *block_table, int num_seqs, int max_blocks,
-                              void *cache, int num_blocks, uint32_t *err_word, void *stream);
+                              void *cache, int num_blocks, const void *kv_norm_weight,
+                              float kv_norm_eps, uint32_t *err_word, void *stream);
 
 /*
  * mla_append_latent -- the RoPE-and-scatter half of step a1, for callers that
  * already hold the latent: writes [c_kv[t] | RoPE(k_rope[t], pos[t])] to the
  * slot of (seq_idx[t], pos[t]).  Same sources as mla_append_cache.
- *   c_kv   [T][d_c] bf16, copied bit for bit
+ *   c_kv   [T][d_c] bf16, copied bit for bit (or RMS-normalised when
+ *          kv_norm_weight is given)
  *   k_rope [T][d_rope] bf16, the raw (unrotated) RoPE key W^KR h
  * Other arguments as for mla_append_cache.
  */
 mla_status_t mla_append_latent(const mla_dims_t *dims, const void *c_kv, const void *k_rope,
                                int T, const int32_t *seq_idx, const int32_t *pos,
                                const int32_t *block_table, int num_seqs, int max_blocks,
-                               void *cache, int num_blocks, uint32_t *err_word, void *stream);
+                               void *cache, int num_blocks, const void *kv_norm_weight,
+                               float kv_norm_eps, uint32_t *err_word, void *stream);
 
 /*
  * mla_absorb_q -- step a2: absorb U^K into the query.
@@ -242,6 +263,54 @@ mla_status_t mla_decode_noalloc(const mla_dims_t *dims, const void *q_abs, const
 mla_status_t mla_up_v(const mla_dims_t *dims, const void *latent, int T, const void *w_uv,
                       const void *w_o, int d_model, void *out_heads, void *out_model,
                       void *stream);
+
+/*
+ * mla_prefill_workspace_size -- bytes of device workspace mla_prefill needs
+ * for B sequences of s new query tokens whose lengths are at most
+ * max_seq_len (0 for invalid dims or sizes).
+ */
+size_t mla_prefill_workspace_size(const mla_dims_t *dims, int B, int s, int max_seq_len);
+
+/*
+ * mla_prefill -- prefill of a chunk of s query tokens per sequence in the
+ * expanded form: each head's keys and values are materialised from the cached
+ * latents and attended to directly,
+ *   k_{j,i} = [U^K_i c^KV_j ; k^R_j],   v_{j,i} = U^V_i c^KV_j,
+ *   out[t][i] = sum_j softmax_j(softmax_scale * [q^C_{t,i} ; q^R_{t,i}] . k_{j,i}) v_{j,i}
+ *   [DeepSeek-V2 paper review, section 2 (k^C = W^UK c^KV, v^C = W^UV c^KV)
+ *    and section 3 (per-head query [q^C; q^R], the shared RoPE key, the
+ *    1/sqrt(d_head + d_rope) scale); DeepSeek-V3 report summary, Method 1]
+ * It gives what mla_absorb_q + mla_decode + mla_up_v give for the same
+ * queries (the two forms are equal up to rounding) at fewer flops when s is
+ * large.  The s tokens are the last s of each sequence: query t of sequence
+ * b sits at position seq_lens[b] - s + t and sees the positions up to it.
+ *   q_nope      [B*s][H][d_head] bf16 (row = b*s + t), q^C
+ *   q_rope      [B*s][H][d_rope] bf16, q^R, rotated here to q_pos[b*s + t]
+ *               (q_pos [B*s] int32), or taken as already rotated if q_pos
+ *               is NULL
+ *   w_uk, w_uv  [H][d_head][d_c] bf16 (U^K_i, U^V_i)
+ *   cache, num_blocks, block_table [B][max_blocks], seq_lens [B]: as for
+ *               mla_decode; the cache rows must hold the chunk's own tokens
+ *   max_seq_len an upper bound of seq_lens (>= s); the call expands
+ *               B * round_up(max_seq_len, 128) latent rows per head
+ *   out         [B*s][H][d_head] bf16 (per-head outputs, O not applied)
+ *   out_lse     [B*s][H] fp32 natural-log softmax denominator, or NULL
+ *   workspace   ws_bytes >= mla_prefill_workspace_size(); its first 4 bytes
+ *               are the device error word (cleared by the call, read with
+ *               mla_decode_error); the rest holds the gathered latents, the
+ *               rotated q^R and the expanded K^C and V^C.
+ *   flags       MLA_SYNC_CHECK
+ * A sequence with seq_lens[b] < s, > max_seq_len or > max_blocks * 64 gets
+ * zero outputs, lse = -inf and MLA_DEVERR_SEQ_LEN.  B = 0 is a no-op; with
+ * B > 0, num_blocks and max_blocks must be at least 1.  Calls that share a
+ * workspace must not overlap on the GPU.
+ */
+mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void *q_rope,
+                         const int32_t *q_pos, const void *w_uk, const void *w_uv, const void *cache,
+                         int num_blocks, const int32_t *block_table, int max_blocks,
+                         const int32_t *seq_lens, int B, int s, int max_seq_len, void *out,
+                         float *out_lse, void *workspace, size_t ws_bytes, uint32_t flags,
+                         void *stream);
 
 /*
  * mla_decode_ctas -- number of CTAs (the persistent grid) the tensor-core

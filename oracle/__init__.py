@@ -40,7 +40,12 @@ tests/test_oracle_pins.py, none is "parity unpinned":
     x / scale, the largest element of each part maps to 448 exactly;
   * decode_latent_fp8_rows: bit-identical to decode_latent_rows on a cache of
     E4M3-representable values with unit scales, and a brute-force NumPy
-    softmax on tiny inputs.
+    softmax on tiny inputs;
+  * rmsnorm_rows: unit root-mean-square output with unit weights, scale
+    invariance, the constant-row closed form;
+  * yarn_theta, rope_rows_theta: scale 1 gives the plain RoPE frequencies and
+    rotations, pairs far below the ramp are divided by s and pairs far above
+    it are unchanged, the ramp is continuous, the rotation preserves norms.
 """
 from __future__ import annotations
 
@@ -91,6 +96,9 @@ def load(path: str):
         [ctypes.c_int] * 7 + [_u8p, _f32p, ctypes.c_int, _i32p, ctypes.c_int, _i32p, _f64p, ctypes.c_int,
                               _i32p, _f64p, _f64p])
     lib.mla_oracle_decode_latent_fp8_rows.restype = ctypes.c_int
+    lib.mla_oracle_rmsnorm_rows.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _f64p, ctypes.c_double, _f64p]
+    lib.mla_oracle_yarn_theta.argtypes = [ctypes.c_int] + [ctypes.c_double] * 5 + [_f64p]
+    lib.mla_oracle_rope_rows_theta.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _i32p, _f64p, _f64p]
     lib.mla_oracle_up_v.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     lib.mla_oracle_out_proj.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     return lib
@@ -319,6 +327,31 @@ def decode_latent_fp8_rows(codes, scales, block_table, seq_lens, s, q_abs, rows=
     if rc != 0:
         raise ValueError("block table entry out of range")
     return out, lse
+
+
+# ------------------------------------------------------------ append extras
+def rmsnorm_rows(x, w, eps=1e-6) -> np.ndarray:
+    """x [N][d] -> x / sqrt(mean(x^2) + eps) * w, row by row."""
+    x, w = _f64(x), _f64(w)
+    y = np.empty_like(x)
+    _lib().mla_oracle_rmsnorm_rows(x.shape[0], x.shape[1], _p(x, _f64p), _p(w, _f64p), float(eps), _p(y, _f64p))
+    return y
+
+
+def yarn_theta(d_r=64, base=10000.0, s=40.0, L0=4096.0, alpha=1.0, beta=32.0) -> np.ndarray:
+    """The RoPE frequency of each of the d_r / 2 pairs under YaRN scaling s."""
+    th = np.empty(d_r // 2)
+    _lib().mla_oracle_yarn_theta(d_r, float(base), float(s), float(L0), float(alpha), float(beta), _p(th, _f64p))
+    return th
+
+
+def rope_rows_theta(x, pos, theta) -> np.ndarray:
+    """RoPE of each row x[n] at position pos[n] with the frequencies theta."""
+    x, pos, theta = _f64(x), _i32(pos), _f64(theta)
+    y = np.empty_like(x)
+    _lib().mla_oracle_rope_rows_theta(x.shape[0], x.shape[1], _p(x, _f64p), _p(pos, _i32p), _p(theta, _f64p),
+                                      _p(y, _f64p))
+    return y
 
 
 def up_v(latent, w_uv) -> np.ndarray:

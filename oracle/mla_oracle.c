@@ -572,6 +572,62 @@ int mla_oracle_decode_latent_fp8_rows(int B, int s, int H, int d_c, int d_r, int
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------- append extras (f4)
+ * DeepSeek-V2 paper review, section 2: the deployed model also puts an
+ * RMSNorm after the compressed latent; the long-context passage: the 4K
+ * pre-training context is extended with YaRN, scale 40.  The pages give no
+ * further constants; the readings used here (listed in the design notes):
+ *   - RMSNorm of the latent row: c_m <- c_m / sqrt(mean(c^2) + eps) * w_m.
+ *   - YaRN frequencies (the NTK-by-parts interpolation of the YaRN method):
+ *     pair k has theta_k = base^(-2k/d_r) and wavelength lambda_k =
+ *     2 pi / theta_k; r_k = L0 / lambda_k rotations over the original
+ *     context L0; ramp g = clamp((r_k - alpha) / (beta - alpha), 0, 1);
+ *     theta'_k = (1 - g) theta_k / s + g theta_k.  With s <= 1 the plain
+ *     RoPE frequencies are used. */
+void mla_oracle_rmsnorm_rows(int N, int d, const double *x, const double *w, double eps, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        double ss = 0.0;
+        for (int m = 0; m < d; ++m) ss += x[(size_t)n * d + m] * x[(size_t)n * d + m];
+        const double inv = 1.0 / sqrt(ss / (double)d + eps);
+        for (int m = 0; m < d; ++m) y[(size_t)n * d + m] = x[(size_t)n * d + m] * inv * w[m];
+    }
+}
+
+void mla_oracle_yarn_theta(int d_r, double base, double s, double L0, double alpha, double beta, double *theta)
+{
+    const double pi = 3.14159265358979323846;
+    for (int k = 0; k < d_r / 2; ++k) {
+        const double th = pow(base, -2.0 * (double)k / (double)d_r);
+        if (s <= 1.0) {
+            theta[k] = th;
+            continue;
+        }
+        const double r = L0 / (2.0 * pi / th);
+        double g = (r - alpha) / (beta - alpha);
+        if (g < 0.0) g = 0.0;
+        if (g > 1.0) g = 1.0;
+        theta[k] = (1.0 - g) * th / s + g * th;
+    }
+}
+
+/* RoPE of rows [N][d_r] at positions pos[N] with given frequencies theta[d_r/2]:
+ * pair k = (x[2k], x[2k+1]) turned by pos * theta[k]. */
+void mla_oracle_rope_rows_theta(int N, int d_r, const double *x, const int32_t *pos, const double *theta,
+                                double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < d_r / 2; ++k) {
+            const double ang = (double)pos[n] * theta[k];
+            const double c = cos(ang), sn = sin(ang);
+            const double x0 = x[(size_t)n * d_r + 2 * k], x1 = x[(size_t)n * d_r + 2 * k + 1];
+            y[(size_t)n * d_r + 2 * k] = x0 * c - x1 * sn;
+            y[(size_t)n * d_r + 2 * k + 1] = x0 * sn + x1 * c;
+        }
+}
+
 /* Up-projection (step a7): out_heads[t][i] = U^V_i latent[t][i]
  * latent [T][H][d_c], w_uv [H][d_h][d_c] -> out_heads [T][H][d_h]. */
 void mla_oracle_up_v(int T, int H, int d_h, int d_c, const double *latent,

@@ -79,8 +79,14 @@ def test_argument_errors(M):
     assert lib.mla_absorb_q(ctypes.byref(d), None, p, None, p, 4, p, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_up_v(ctypes.byref(d), p, 4, p, p, 100, p, p, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_up_v(ctypes.byref(d), p, 4, None, None, 0, p, None, None) == M.MLA_ERR_INVALID_ARG
-    assert lib.mla_append_cache(ctypes.byref(d), p, 4, 100, p, p, p, p, p, 1, 1, p, 1, None, None) == M.MLA_ERR_UNSUPPORTED
-    assert lib.mla_append_latent(ctypes.byref(d), p, p, -1, p, p, p, 1, 1, p, 1, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_cache(ctypes.byref(d), p, 4, 100, p, p, p, p, p, 1, 1, p, 1, None, 0.0, None, None) == M.MLA_ERR_UNSUPPORTED
+    assert lib.mla_append_latent(ctypes.byref(d), p, p, -1, p, p, p, 1, 1, p, 1, None, 0.0, None, None) == M.MLA_ERR_INVALID_ARG
+    # a misaligned norm weight, a negative eps, a YaRN ramp with beta <= alpha
+    q = ctypes.c_void_p(258)
+    assert lib.mla_append_latent(ctypes.byref(d), p, p, 1, p, p, p, 1, 1, p, 1, q, 1e-6, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_latent(ctypes.byref(d), p, p, 1, p, p, p, 1, 1, p, 1, p, -1.0, None, None) == M.MLA_ERR_INVALID_ARG
+    bad = M.dims(128, rope_scaling=40.0, rope_yarn_alpha=32.0, rope_yarn_beta=1.0)
+    assert lib.mla_append_latent(ctypes.byref(bad), p, p, 1, p, p, p, 1, 1, p, 1, None, 0.0, None, None) == M.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_error(None, None, 0, None) == M.MLA_ERR_INVALID_ARG
 
 
@@ -201,3 +207,35 @@ def test_noalloc_rejects_tensor_core_shapes_beyond_its_scratch(M, H, s):
     assert lib.mla_kernel_launches() == n0
     # the size the call refused is indeed beyond the scratch
     assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, s, 64) > M.MLA_NOALLOC_SCRATCH_BYTES
+
+
+def test_prefill_argument_errors_and_workspace(M):
+    """mla_prefill rejects bad arguments before any device work, and its
+    workspace grows with the sequences it expands."""
+    lib = _raw(M)
+    d = M.dims(128)
+    p = ctypes.c_void_p(256)
+    big = 1 << 40
+    n0 = lib.mla_kernel_launches()
+    call = lambda dd, qn=p, B=1, s=4, msl=64, ws=p, wsb=big, nb=1, mb=1: lib.mla_prefill(
+        dd, qn, p, None, p, p, p, nb, p, mb, p, B, s, msl, p, None, ws, wsb, 0, None)
+    assert call(None) == M.MLA_ERR_INVALID_ARG
+    assert call(ctypes.byref(d), qn=None) == M.MLA_ERR_INVALID_ARG
+    assert call(ctypes.byref(d), qn=ctypes.c_void_p(258)) == M.MLA_ERR_INVALID_ARG   # misaligned
+    assert call(ctypes.byref(d), s=0) == M.MLA_ERR_INVALID_ARG
+    assert call(ctypes.byref(d), s=65, msl=64) == M.MLA_ERR_INVALID_ARG             # max_seq_len < s
+    assert call(ctypes.byref(d), nb=0) == M.MLA_ERR_INVALID_ARG
+    assert call(ctypes.byref(d), mb=0) == M.MLA_ERR_INVALID_ARG
+    assert call(ctypes.byref(d), ws=None) == M.MLA_ERR_WORKSPACE
+    assert call(ctypes.byref(d), wsb=4096) == M.MLA_ERR_WORKSPACE
+    assert call(ctypes.byref(M.dims(24))) == M.MLA_ERR_UNSUPPORTED
+    assert lib.mla_prefill(ctypes.byref(d), None, None, None, None, None, None, 0, None, 0, None, 0, 1, 1,
+                           None, None, None, 0, 0, None) == M.MLA_OK               # B = 0
+    assert lib.mla_kernel_launches() == n0
+    a = lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 128, 1000)
+    b = lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 128, 1024)   # same 128-row padding
+    c = lib.mla_prefill_workspace_size(ctypes.byref(d), 2, 128, 1000)
+    assert 0 < a == b < c and a % 256 == 0
+    # K^C and V^C dominate: 2 x rows x H x 128 bf16
+    assert a >= 2 * 1024 * 128 * 128 * 2
+    assert lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 129, 128) == 0

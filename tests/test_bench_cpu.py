@@ -59,3 +59,15 @@ def test_single_rank_is_the_plain_workload():
     cfg = W.CONFIGS["v2"]
     assert bench.replica_config(cfg, 0) is cfg
     assert bench.max_over_ranks([1.5, 2.5], 1, "cpu") == [1.5, 2.5]
+
+
+def test_prefill_flop_count_matches_brute_force():
+    """The prefill's algorithmic flops: visible (query, key) pairs counted one
+    by one on small shapes, and the expansion over the padded rows."""
+    import bench
+    for B, s, L, H in [(1, 1, 1, 16), (2, 5, 9, 16), (1, 200, 520, 32), (3, 130, 130, 16)]:
+        vis = sum(L - s + t + 1 for t in range(s))
+        att, exp_ = bench.prefill_flops(B, s, L, H)
+        assert att == 2.0 * B * H * vis * (192 + 128)
+        lpad = -(-L // 128) * 128
+        assert exp_ == 2.0 * 2 * B * lpad * H * 128 * 512

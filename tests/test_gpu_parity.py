@@ -357,3 +357,96 @@ def test_absorb_q_many_tokens_and_rotated_copy(lib):
     assert_parity(W.bf16_bits_to_f32(host_bits(q_abs)), ref, what="absorb_q, 300 tokens")
     lib.mla_absorb_q(dims, torch_bits(d["q_nope"]), torch_bits(d["q_rope"]), None, torch_bits(d["w_uk"]), q_abs)
     assert np.array_equal(host_bits(q_abs)[..., 512:], d["q_rope"])
+
+
+# ------------------------------------------------- append extras (row f4)
+YARN = dict(rope_scaling=40.0, rope_original_ctx=4096, rope_yarn_alpha=1.0, rope_yarn_beta=32.0)
+
+
+def _norm_weight(seed):
+    rng = np.random.default_rng(seed)
+    return W.f32_to_bf16_bits((1.0 + 0.1 * rng.standard_normal(512)).astype(np.float32))
+
+
+def test_append_latent_rmsnorm_and_yarn(lib):
+    """mla_append_latent with an RMSNorm weight and YaRN-scaled RoPE (scale 40
+    over a 4096-token original context) against the fp64 RMSNorm of the bf16
+    latent and the fp64 rotation at the YaRN frequencies."""
+    o = _oracle()
+    cfg = W.MLAConfig("f4_lat", B=3, s=1, H=16, L=0, paged=True, seed=501, d_model=2048,
+                      seq_lens=(5000, 70, 131))
+    d = W.make_decode_inputs(cfg, with_cache_pages=False)
+    dims = lib.dims(cfg.H, **YARN)
+    import torch
+    cache = torch.full((d["num_blocks"], 64, 576), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bt = i32(d["block_table"])
+    w = _norm_weight(502)
+    lib.mla_append_latent(dims, torch_bits(d["c_kv"]), torch_bits(d["k_rope"]), i32(d["tok_seq"]), i32(d["tok_pos"]),
+                          bt, cache, kv_norm_weight=torch_bits(w), kv_norm_eps=1e-6)
+    got = host_bits(cache)
+    blk = d["block_table"][d["tok_seq"], d["tok_pos"] // 64]
+    slot = d["tok_pos"] % 64
+    c_ref = o.rmsnorm_rows(o.bf16_to_f64(d["c_kv"]), o.bf16_to_f64(w), 1e-6)
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, :512]), c_ref, what="RMS-normalised latent")
+    th = o.yarn_theta(s=40.0, L0=4096.0, alpha=1.0, beta=32.0)
+    kr_ref = o.rope_rows_theta(o.bf16_to_f64(d["k_rope"]), d["tok_pos"], th)
+    assert_parity(W.bf16_bits_to_f32(got[blk, slot, 512:]), kr_ref, what="YaRN-rotated k^R")
+    # YaRN moved the slow pairs: far positions differ from plain RoPE
+    plain = o.rope_rows(o.bf16_to_f64(d["k_rope"]), d["tok_pos"])
+    far = d["tok_pos"] > 2000
+    assert np.max(np.abs(kr_ref[far] - plain[far])) > 0.1
+
+
+@pytest.mark.parametrize("d_model", [5120, 576], ids=["cluster_split_k", "one_pass"])
+def test_append_cache_rmsnorm_and_yarn(lib, d_model):
+    """The projection path with RMSNorm and YaRN: the oracle projects in fp64,
+    rounds the latent to bf16 (the projection's output precision), normalises
+    it in fp64 and rotates the raw k^R at the YaRN frequencies."""
+    import torch
+    o = _oracle()
+    cfg = W.MLAConfig("f4_app", B=3, s=1, H=16, L=0, paged=True, seed=503, d_model=d_model,
+                      seq_lens=(3000, 64, 700))
+    g = GpuWorkload(cfg)
+    a = W.make_append_inputs(cfg, 150)
+    rng = np.random.default_rng(504)
+    slots = rng.choice(int(np.sum(g.d["seq_lens"])), size=150, replace=False)
+    seq = g.d["tok_seq"][slots].astype(np.int32)
+    pos = g.d["tok_pos"][slots].astype(np.int32)
+    dims = lib.dims(cfg.H, **YARN)
+    w = _norm_weight(505)
+    lib.mla_append_cache(dims, torch_bits(a["h"]), torch_bits(a["w_dkv"]), torch_bits(a["w_kr"]), i32(seq), i32(pos),
+                         g.block_table, g.cache, err_word=g.err, kv_norm_weight=torch_bits(w), kv_norm_eps=1e-6)
+    got = host_bits(g.cache)
+    c, kr_raw = o.kv_project(a["h"], a["w_dkv"], a["w_kr"], np.zeros_like(pos))   # RoPE at 0: the raw key
+    c_bf16 = W.bf16_bits_to_f32(W.f32_to_bf16_bits(c.astype(np.float32))).astype(np.float64)
+    c_ref = o.rmsnorm_rows(c_bf16, o.bf16_to_f64(w), 1e-6)
+    kr_ref = o.rope_rows_theta(kr_raw, pos, o.yarn_theta(s=40.0, L0=4096.0, alpha=1.0, beta=32.0))
+    bt = g.d["block_table"]
+    blk, sl = bt[seq, pos // 64], pos % 64
+    assert_parity(W.bf16_bits_to_f32(got[blk, sl, :512]), c_ref, what="RMS-normalised projected latent")
+    assert_parity(W.bf16_bits_to_f32(got[blk, sl, 512:]), kr_ref, what="YaRN-rotated projected k^R")
+    assert int(g.err.item()) == 0
+
+
+def test_absorb_q_yarn(lib):
+    """mla_absorb_q with YaRN-scaled RoPE at query positions up to 131071
+    against the fp64 rotation at the YaRN frequencies; the latent part is the
+    plain absorption."""
+    import torch
+    o = _oracle()
+    rng = np.random.default_rng(506)
+    T, H = 40, 64
+    q_nope = W.f32_to_bf16_bits(rng.standard_normal((T, H, 128)).astype(np.float32))
+    q_rope = W.f32_to_bf16_bits(rng.standard_normal((T, H, 64)).astype(np.float32))
+    w_uk = W.f32_to_bf16_bits((rng.standard_normal((H, 128, 512)) / np.sqrt(512)).astype(np.float32))
+    q_pos = rng.integers(0, 131072, T).astype(np.int32)
+    dims = lib.dims(H, **YARN)
+    q_abs = torch.empty(T, H, 576, dtype=torch.bfloat16, device="cuda")
+    lib.mla_absorb_q(dims, torch_bits(q_nope), torch_bits(q_rope), i32(q_pos), torch_bits(w_uk), q_abs)
+    got = W.bf16_bits_to_f32(host_bits(q_abs))
+    th = o.yarn_theta(s=40.0, L0=4096.0, alpha=1.0, beta=32.0)
+    qr = o.bf16_to_f64(q_rope)
+    ref_r = o.rope_rows_theta(qr.reshape(-1, 64), np.repeat(q_pos, H), th).reshape(qr.shape)
+    assert_parity(got[..., 512:], ref_r, what="YaRN-rotated q^R")
+    ref = o.absorb_q(o.bf16_to_f64(q_nope), qr, o.bf16_to_f64(w_uk))
+    assert_parity(got[..., :512], ref[..., :512], what="absorbed latent query")

@@ -744,3 +744,54 @@ def test_planted_fp8_mistakes_are_caught(oracle_mod, tmp_path, name):
         assert caught, f"mutation {name} was not caught"
     finally:
         oracle_mod._LIB = saved
+
+
+# ------------------------------------------------------- append extras pins
+def test_rmsnorm_rows_closed_forms(oracle_mod):
+    rng = np.random.default_rng(50)
+    x = rng.standard_normal((20, 512)) * rng.uniform(0.1, 30, (20, 1))
+    ones = np.ones(512)
+    y = oracle_mod.rmsnorm_rows(x, ones, eps=0.0)
+    np.testing.assert_allclose(np.sqrt((y ** 2).mean(1)), 1.0, rtol=1e-14)       # unit RMS
+    np.testing.assert_allclose(oracle_mod.rmsnorm_rows(7.5 * x, ones, eps=0.0), y, rtol=1e-13)  # scale invariant
+    c = np.full((1, 512), -3.0)                                                  # constant row: sign * w
+    w = rng.standard_normal(512)
+    np.testing.assert_allclose(oracle_mod.rmsnorm_rows(c, w, eps=0.0)[0], -w, rtol=1e-15)
+    # eps enters under the root: a zero row stays zero, a tiny row is damped
+    assert np.all(oracle_mod.rmsnorm_rows(np.zeros((1, 512)), w, eps=1e-6) == 0)
+    t = np.full((1, 512), 1e-3)
+    np.testing.assert_allclose(oracle_mod.rmsnorm_rows(t, ones, eps=1e-6)[0], 1e-3 / math.sqrt(1e-6 + 1e-6),
+                               rtol=1e-14)
+
+
+def test_yarn_theta_reduces_to_rope_and_interpolates(oracle_mod):
+    base = 10000.0
+    plain = base ** (-2.0 * np.arange(32) / 64)
+    np.testing.assert_allclose(oracle_mod.yarn_theta(s=1.0), plain, rtol=5e-16)  # numpy and libm pow: an ulp apart at most
+    th = oracle_mod.yarn_theta(s=40.0, L0=4096.0, alpha=1.0, beta=32.0)
+    rot = 4096.0 * plain / (2 * math.pi)                 # rotations over the original context
+    hi, lo = rot > 32.0, rot < 1.0
+    assert hi.any() and lo.any()
+    np.testing.assert_allclose(th[hi], plain[hi], rtol=1e-15)        # fast pairs unchanged
+    np.testing.assert_allclose(th[lo], plain[lo] / 40.0, rtol=1e-15)  # slow pairs interpolated by s
+    mid = ~(hi | lo)
+    g = (rot[mid] - 1.0) / 31.0
+    np.testing.assert_allclose(th[mid], (1 - g) * plain[mid] / 40.0 + g * plain[mid], rtol=1e-14)
+    assert np.all(np.diff(th) < 0)                       # still strictly decreasing with k
+
+
+def test_rope_rows_theta_matches_plain_rope_and_preserves_norms(oracle_mod):
+    rng = np.random.default_rng(51)
+    pos = np.array([0, 1, 4095, 65536, 131071], np.int32)
+    x = rng.standard_normal((pos.size, 64))
+    plain = oracle_mod.rope_rows_theta(x, pos, oracle_mod.yarn_theta(s=1.0))
+    np.testing.assert_allclose(plain, oracle_mod.rope_rows(x, pos), rtol=0, atol=1e-12)
+    y = oracle_mod.rope_rows_theta(x, pos, oracle_mod.yarn_theta(s=40.0))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    assert np.array_equal(y[0], x[0])
+    # relative positions: <R_m q, R_n k> depends on n - m only, also with YaRN
+    th = oracle_mod.yarn_theta(s=40.0)
+    q, k = rng.standard_normal((1, 64)), rng.standard_normal((1, 64))
+    a = oracle_mod.rope_rows_theta(q, np.array([7], np.int32), th) @ oracle_mod.rope_rows_theta(k, np.array([900], np.int32), th).T
+    b = oracle_mod.rope_rows_theta(q, np.array([7007], np.int32), th) @ oracle_mod.rope_rows_theta(k, np.array([7900], np.int32), th).T
+    assert abs(a - b) < 1e-10
