@@ -59,6 +59,14 @@ def algorithmic(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
     return byts, flops, rows_read
 
 
+def algorithmic_fp8(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
+    """As `algorithmic`, for the FP8 cache: a cache row is 576 one-byte codes
+    plus two fp32 scales (584 B/token)."""
+    byts, flops, rows_read = algorithmic(cfg, seq_lens, max_blocks)
+    D = cfg.d_c + cfg.d_r
+    return byts - rows_read * D * 2 + rows_read * (D + 8), flops, rows_read
+
+
 # DRAM bytes (read + write) the current decode kernel moves per cache token,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
 # tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (166.9 MB for
@@ -401,6 +409,7 @@ def run_ours(args):
     }
     if not args.no_per_config and world == 1:
         line["per_config"] = per_config(M, [n for n in ("tiny", "v2lite", "v2", "longctx", "mtp")])
+        line["per_config_fp8"] = per_config(M, [n for n in ("v2lite", "v2", "longctx", "mtp")], fp8=True)
     if not args.no_prefill and world == 1:
         line["prefill"] = prefill_bench(M)
     if not args.no_cpu_baseline:
@@ -409,7 +418,7 @@ def run_ours(args):
 
 
 # ---------------------------------------------------- every config's decode
-def per_config(M, names, iters=30):
+def per_config(M, names, iters=30, fp8=False):
     """The decode call (plan + decode + combine) on each named workload: its
     CUDA-event time on the launching stream (mean of `iters` back-to-back
     calls after 3 warm-ups), latent-cache GB/s, TFLOP/s and roofline
@@ -431,7 +440,15 @@ def per_config(M, names, iters=30):
         g = torch.Generator(device="cuda")
         g.manual_seed(cfg.seed)
         D = cfg.d_c + cfg.d_r
-        cache = torch.randn((nphys, cfg.block_size, D), generator=g, device="cuda").to(torch.bfloat16)
+        if fp8:
+            # E4M3 bit patterns with a random sign, exponent field 5..9 and
+            # mantissa (no NaN code), scales uniform in [0.1, 0.3]
+            bits = torch.randint(0, 1 << 30, (nphys, cfg.block_size, D), generator=g, device="cuda")
+            codes = ((bits & 0x80) | (((bits >> 8) % 5 + 5) << 3) | ((bits >> 16) & 7)).to(torch.uint8)
+            scales = torch.rand((nphys, cfg.block_size, 2), generator=g, device="cuda") * 0.2 + 0.1
+            cache = None
+        else:
+            cache = torch.randn((nphys, cfg.block_size, D), generator=g, device="cuda").to(torch.bfloat16)
         q = torch.randn((cfg.T, cfg.H, D), generator=g, device="cuda")
         q[..., :cfg.d_c] *= 0.5
         q = q.to(torch.bfloat16)
@@ -442,9 +459,15 @@ def per_config(M, names, iters=30):
         lse = torch.empty(cfg.T, cfg.H, dtype=torch.float32, device="cuda")
         ws = torch.empty(M.mla_decode_workspace_size(dims, cfg.B, cfg.s, table.shape[1] * 64),
                          dtype=torch.uint8, device="cuda")
-        call = lambda: M.mla_decode(dims, q, cache, bt, slt, cfg.s, lat, lse, ws)
-        byts, flops, rows = algorithmic(cfg, sl, table.shape[1])
-        small = rows * 1152 < L2_BYTES
+        if fp8:
+            call = lambda: M.mla_decode_fp8(dims, q, codes, scales, bt, slt, cfg.s, lat, lse, ws)
+            byts, flops, rows = algorithmic_fp8(cfg, sl, table.shape[1])
+            row_bytes = 584
+        else:
+            call = lambda: M.mla_decode(dims, q, cache, bt, slt, cfg.s, lat, lse, ws)
+            byts, flops, rows = algorithmic(cfg, sl, table.shape[1])
+            row_bytes = 1152
+        small = rows * row_bytes < L2_BYTES
         for _ in range(3):
             call()
         torch.cuda.synchronize()
@@ -464,7 +487,8 @@ def per_config(M, names, iters=30):
 
         t = timed(small)
         hbm_t, tc_t = byts / (pk["hbm"] * 1e9), flops / (pk["tc"] * 1e12)
-        r = {"workload": cfg.describe, "us": t * 1e6, "cache_gbs": rows * 1152 / t / 1e9,
+        r = {"workload": cfg.describe + (" (FP8 E4M3 cache)" if fp8 else ""), "us": t * 1e6,
+             "cache_gbs": rows * row_bytes / t / 1e9,
              "gbs": byts / t / 1e9, "tflops": flops / t / 1e12,
              "bound": "hbm" if hbm_t >= tc_t else "tensor", "roofline_us": max(hbm_t, tc_t) * 1e6,
              "roofline_frac": max(hbm_t, tc_t) / t, "decode_ctas": M.mla_decode_ctas(dims, cfg.s),
@@ -473,6 +497,8 @@ def per_config(M, names, iters=30):
             r["warm_l2_us"] = timed(False) * 1e6
         out[name] = r
         del cache, q, lat, lse, ws, bt, slt
+        if fp8:
+            del codes, scales
         torch.cuda.empty_cache()
     return out
 
@@ -658,6 +684,8 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="skip timing the decode of every workload")
     ap.add_argument("--no-prefill", action="store_true", help="skip timing the expanded-form prefill")
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill workloads")
+    ap.add_argument("--decode-only", default="", help="comma-separated workloads: time only their decode calls")
+    ap.add_argument("--fp8", action="store_true", help="with --decode-only: the FP8-cache decode")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps on the stream, not as a graph")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -665,6 +693,13 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        import torch
+        import head_latent_attention_10_b200 as M
+        M.load_library()
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        key = "per_config_fp8" if args.fp8 else "per_config"
+        print(json.dumps({key: per_config(M, args.decode_only.split(","), fp8=args.fp8)}), flush=True)
     elif args.prefill_only:
         import torch
         import head_latent_attention_10_b200 as M

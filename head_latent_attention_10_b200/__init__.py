@@ -23,7 +23,7 @@ MLA_SYNC_CHECK, MLA_FORCE_SIMPLE, MLA_DEBUG_STALL = 0x1, 0x2, 0x100
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",
             "mla_kernel_launches", "mla_decode_ctas", "mla_decode_noalloc",
-            "mla_prefill_workspace_size", "mla_prefill")
+            "mla_prefill_workspace_size", "mla_prefill", "mla_append_latent_fp8", "mla_decode_fp8")
 
 
 class MLAError(RuntimeError):
@@ -81,6 +81,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_prefill_workspace_size.restype = ctypes.c_size_t
     lib.mla_prefill.argtypes = [D, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp, _vp,
                                 _vp, ctypes.c_size_t, ctypes.c_uint32, _vp]
+    lib.mla_append_latent_fp8.argtypes = [D, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _vp, _vp, _i, _vp, _f, _vp, _vp]
+    lib.mla_decode_fp8.argtypes = [D, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _vp, _vp, _vp, ctypes.c_size_t,
+                                   ctypes.c_uint32, _vp]
     lib.mla_kernel_launches.argtypes = []
     lib.mla_kernel_launches.restype = ctypes.c_uint64
     for name in EXPORTED:
@@ -203,6 +206,28 @@ def mla_prefill(d, q_nope, q_rope, q_pos, w_uk, w_uv, cache, block_table, seq_le
         cache.shape[0], _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, s, max_seq_len,
         _ptr(out), _ptr(out_lse), _ptr(workspace), workspace.numel() * workspace.element_size(), flags,
         _stream(stream)), "mla_prefill")
+
+
+def mla_append_latent_fp8(d, c_kv, k_rope, seq_idx, pos, block_table, codes, scales, err_word=None,
+                          stream=None, kv_norm_weight=None, kv_norm_eps=1e-6):
+    """The row [c_kv | RoPE(k_rope, pos)] (RMS-normalised latent if
+    kv_norm_weight is given) quantized to E4M3 codes [num_blocks][64][576]
+    uint8 with per-part fp32 scales [num_blocks][64][2]."""
+    _check(load_library().mla_append_latent_fp8(
+        ctypes.byref(d), _ptr(c_kv), _ptr(k_rope), c_kv.shape[0], _ptr(seq_idx), _ptr(pos),
+        _ptr(block_table), block_table.shape[0], block_table.shape[1], _ptr(codes), _ptr(scales),
+        codes.shape[0], _ptr(kv_norm_weight), kv_norm_eps, _ptr(err_word), _stream(stream)),
+        "mla_append_latent_fp8")
+
+
+def mla_decode_fp8(d, q_abs, codes, scales, block_table, seq_lens, s, out_latent, out_lse, workspace,
+                   flags: int = 0, stream=None):
+    """Absorbed attention over the FP8 latent cache; writes out_latent and out_lse."""
+    B = seq_lens.shape[0]
+    _check(load_library().mla_decode_fp8(
+        ctypes.byref(d), _ptr(q_abs), _ptr(codes), _ptr(scales), codes.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), B, s, _ptr(out_latent), _ptr(out_lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), flags, _stream(stream)), "mla_decode_fp8")
 
 
 def mla_up_v(d, latent, w_uv, out_heads, w_o=None, out_model=None, stream=None):

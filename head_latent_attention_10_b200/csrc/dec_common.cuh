@@ -23,6 +23,7 @@ struct DecArgs {
     uint32_t *err;
     unsigned long long limit_ns;
     int stall_tile;       // test hook: the page load of this tile of every range is never issued (-1: none)
+    const float *scales;  // FP8 cache only: [num_blocks][64][2] fp32 per-part scales
     float scale_log2;
     int max_blocks, num_blocks, s, H, B, groups;
 };

@@ -26,80 +26,12 @@ __device__ __forceinline__ long long cache_slot(const int32_t *block_table, int 
     return (long long)blk * kBlock + (pos % kBlock);
 }
 
-// ------------------------------------------------------- append from latents
-// One warp per token: lanes copy the 1 KB latent (2 x 16 B each), optionally
-// RMS-normalised with weight norm_w, and turn RoPE pair `lane` of the key.
-__global__ void __launch_bounds__(256)
-append_latent_kernel(const bf16 *__restrict__ c_kv, const bf16 *__restrict__ k_rope, int T,
-                     const int32_t *__restrict__ seq_idx, const int32_t *__restrict__ pos,
-                     const int32_t *__restrict__ block_table, int num_seqs, int max_blocks,
-                     bf16 *__restrict__ cache, int num_blocks, const RopeTable rope,
-                     const bf16 *__restrict__ norm_w, float eps, uint32_t *err)
+// RMSNorm of a latent row held by the 32 lanes of a warp (lane l: values
+// [8l, 8l+8) in v0 and [256+8l, 256+8l+8) in v1), in place: sum of squares in
+// fp32, x * inv * w rounded to bf16.
+__device__ __forceinline__ void rmsnorm_lanes(uint4 &v0, uint4 &v1, const bf16 *__restrict__ norm_w, float eps,
+                                              int lane)
 {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= T) return;
-    const int p = pos[warp];
-    const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks,
-                                      seq_idx[warp], p, lane == 0 ? err : nullptr);
-    if (slot < 0) return;
-    bf16 *dst = cache + slot * kRow;
-    const uint4 *src = reinterpret_cast<const uint4 *>(c_kv + (long long)warp * kDc);
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-    uint4 v0 = src[lane], v1 = src[lane + 32];
-    if (norm_w) {
-        // the latent row's 512 values: lane l holds [8l, 8l+8) and [256+8l, 256+8l+8)
-        float x[16];
-        const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
-        const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
-        float ss = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 a = __bfloat1622float2(h0[i]), b = __bfloat1622float2(h1[i]);
-            x[2 * i] = a.x; x[2 * i + 1] = a.y; x[8 + 2 * i] = b.x; x[8 + 2 * i + 1] = b.y;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) ss += x[i] * x[i];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = rms_inv(ss, eps);
-        const uint4 w0 = reinterpret_cast<const uint4 *>(norm_w)[lane];
-        const uint4 w1 = reinterpret_cast<const uint4 *>(norm_w)[lane + 32];
-        const __nv_bfloat162 *g0 = reinterpret_cast<const __nv_bfloat162 *>(&w0);
-        const __nv_bfloat162 *g1 = reinterpret_cast<const __nv_bfloat162 *>(&w1);
-        __nv_bfloat162 *o0 = reinterpret_cast<__nv_bfloat162 *>(&v0);
-        __nv_bfloat162 *o1 = reinterpret_cast<__nv_bfloat162 *>(&v1);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 a = __bfloat1622float2(g0[i]), b = __bfloat1622float2(g1[i]);
-            o0[i] = __floats2bfloat162_rn(x[2 * i] * inv * a.x, x[2 * i + 1] * inv * a.y);
-            o1[i] = __floats2bfloat162_rn(x[8 + 2 * i] * inv * b.x, x[8 + 2 * i + 1] * inv * b.y);
-        }
-    }
-    d4[lane] = v0;
-    d4[lane + 32] = v1;
-    const __nv_bfloat162 kr =
-        reinterpret_cast<const __nv_bfloat162 *>(k_rope + (long long)warp * kDr)[lane];
-    float y0, y1;
-    rope_turn(__low2float(kr), __high2float(kr), p, rope.theta[lane], &y0, &y1);
-    reinterpret_cast<__nv_bfloat162 *>(dst + kDc)[lane] = __floats2bfloat162_rn(y0, y1);
-}
-
-// RMS normalisation, in place, of the latent part of the cache rows of T
-// tokens (the projection path writes the rows first): one warp per token.
-__global__ void __launch_bounds__(256)
-latent_rmsnorm_kernel(int T, const int32_t *__restrict__ seq_idx, const int32_t *__restrict__ pos,
-                      const int32_t *__restrict__ block_table, int num_seqs, int max_blocks,
-                      bf16 *__restrict__ cache, int num_blocks, const bf16 *__restrict__ norm_w, float eps)
-{
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= T) return;
-    const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks, seq_idx[warp], pos[warp],
-                                      nullptr);
-    if (slot < 0) return;
-    uint4 *row = reinterpret_cast<uint4 *>(cache + slot * kRow);
-    uint4 v0 = row[lane], v1 = row[lane + 32];
     float x[16];
     const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
     const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
@@ -126,6 +58,68 @@ latent_rmsnorm_kernel(int T, const int32_t *__restrict__ seq_idx, const int32_t 
         o0[i] = __floats2bfloat162_rn(x[2 * i] * inv * a.x, x[2 * i + 1] * inv * a.y);
         o1[i] = __floats2bfloat162_rn(x[8 + 2 * i] * inv * b.x, x[8 + 2 * i + 1] * inv * b.y);
     }
+}
+
+// The cache row of token t as the lanes of a warp hold it: lane l has latent
+// values [8l, 8l+8) (v0) and [256+8l, 256+8l+8) (v1), RMS-normalised if
+// norm_w is given, and RoPE pair l of the key turned to position p (kr).
+__device__ __forceinline__ void latent_row_lanes(const bf16 *__restrict__ c_kv, const bf16 *__restrict__ k_rope,
+                                                 int t, int p, int lane, const RopeTable &rope,
+                                                 const bf16 *__restrict__ norm_w, float eps, uint4 &v0, uint4 &v1,
+                                                 __nv_bfloat162 &kr)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(c_kv + (long long)t * kDc);
+    v0 = src[lane];
+    v1 = src[lane + 32];
+    if (norm_w) rmsnorm_lanes(v0, v1, norm_w, eps, lane);
+    const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(k_rope + (long long)t * kDr)[lane];
+    float y0, y1;
+    rope_turn(__low2float(x), __high2float(x), p, rope.theta[lane], &y0, &y1);
+    kr = __floats2bfloat162_rn(y0, y1);
+}
+
+// ------------------------------------------------------- append from latents
+// One warp per token: lanes copy the 1 KB latent (2 x 16 B each), optionally
+// RMS-normalised with weight norm_w, and turn RoPE pair `lane` of the key.
+__global__ void __launch_bounds__(256)
+append_latent_kernel(const bf16 *__restrict__ c_kv, const bf16 *__restrict__ k_rope, int T,
+                     const int32_t *__restrict__ seq_idx, const int32_t *__restrict__ pos,
+                     const int32_t *__restrict__ block_table, int num_seqs, int max_blocks,
+                     bf16 *__restrict__ cache, int num_blocks, const RopeTable rope,
+                     const bf16 *__restrict__ norm_w, float eps, uint32_t *err)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= T) return;
+    const int p = pos[warp];
+    const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks,
+                                      seq_idx[warp], p, lane == 0 ? err : nullptr);
+    if (slot < 0) return;
+    uint4 v0, v1;
+    __nv_bfloat162 kr;
+    latent_row_lanes(c_kv, k_rope, warp, p, lane, rope, norm_w, eps, v0, v1, kr);
+    bf16 *dst = cache + slot * kRow;
+    reinterpret_cast<uint4 *>(dst)[lane] = v0;
+    reinterpret_cast<uint4 *>(dst)[lane + 32] = v1;
+    reinterpret_cast<__nv_bfloat162 *>(dst + kDc)[lane] = kr;
+}
+
+// RMS normalisation, in place, of the latent part of the cache rows of T
+// tokens (the projection path writes the rows first): one warp per token.
+__global__ void __launch_bounds__(256)
+latent_rmsnorm_kernel(int T, const int32_t *__restrict__ seq_idx, const int32_t *__restrict__ pos,
+                      const int32_t *__restrict__ block_table, int num_seqs, int max_blocks,
+                      bf16 *__restrict__ cache, int num_blocks, const bf16 *__restrict__ norm_w, float eps)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= T) return;
+    const long long slot = cache_slot(block_table, num_seqs, max_blocks, num_blocks, seq_idx[warp], pos[warp],
+                                      nullptr);
+    if (slot < 0) return;
+    uint4 *row = reinterpret_cast<uint4 *>(cache + slot * kRow);
+    uint4 v0 = row[lane], v1 = row[lane + 32];
+    rmsnorm_lanes(v0, v1, norm_w, eps, lane);
     row[lane] = v0;
     row[lane + 32] = v1;
 }

@@ -147,12 +147,12 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
 
 // C = A B on tcgen05; `c` is the output tensor map of the staged (TMA store)
 // epilogue, unused by the others.
-template <int BN, bool kBmn, class Epi, bool kAshared = false>
+template <int BN, bool kBmn, class Epi>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
                            uint32_t *err, cudaStream_t st, const CUtensorMap *c = nullptr)
 {
     using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kAshared>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
     if (e != cudaSuccess) return e;
@@ -258,12 +258,78 @@ int decode_ranges(int H, int s)
     static std::atomic<bool> attr64[kMaxDevices];
     const int sms = sm_count();
     if (sms <= 0) return 0;
-    if (ensure_smem_attr(tc_decode64_kernel, kD64Smem, attr64) != cudaSuccess) return 0;
+    if (ensure_smem_attr(tc_decode64_kernel<false>, kD64Smem, attr64) != cudaSuccess) return 0;
     const int groups = dec_groups(H, s);
     int r = sms / groups;
     const int cap = kMaxRanges / groups;
     if (r > cap) r = cap;
     return r > 0 ? r : 1;
+}
+
+// The tensor-core decode (plan, decode kernel, combine) on a bf16 cache, or
+// on an FP8 cache (codes + per-part scales) with kFp8.
+template <bool kFp8>
+mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void *cache, const float *scales,
+                           int num_blocks, const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                           int B, int s, void *out_latent, float *out_lse, char *ws, size_t ws_bytes,
+                           uint32_t flags, cudaStream_t strm)
+{
+    const int H = dims->num_heads;
+    uint32_t *err = (uint32_t *)ws;
+    const TcWs w = tc_ws(H, s, B);
+    if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
+    const int groups = dec_groups(H, s);
+    const int ranges = decode_ranges(H, s);
+    if (ranges <= 0) return MLA_ERR_CUDA;
+    CUtensorMap mkv;
+    if (kFp8) {
+        if (!make_tmap_3d_u8(&mkv, cache, kRow, (uint64_t)num_blocks * kBlock, 1, kRow, (uint64_t)num_blocks * kBlock * kRow,
+                             64, kT64, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return MLA_ERR_CUDA;
+        static std::atomic<bool> attr8[kMaxDevices];
+        if (ensure_smem_attr(tc_decode64_kernel<true>, kD64SmemFp8, attr8) != cudaSuccess) return MLA_ERR_CUDA;
+    } else {
+        if (!tmap(&mkv, cache, kRow, (uint64_t)num_blocks * kBlock, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
+    }
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
+    int32_t *plan = (int32_t *)(ws + w.off_plan);
+    dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    DecArgs da;
+    da.q_abs = (const bf16 *)q_abs;
+    da.block_table = block_table;
+    da.seq_lens = seq_lens;
+    da.plan = plan;
+    da.out = (bf16 *)out_latent;
+    da.out_lse = out_lse;
+    da.part_o = (float *)(ws + w.off_o);
+    da.part_lse2 = (float *)(ws + w.off_lse);
+    da.err = err;
+    da.limit_ns = (flags & MLA_DEBUG_STALL) ? kStallWaitLimitNs : kWaitLimitNs;
+    da.stall_tile = (flags & MLA_DEBUG_STALL) ? 0 : -1;
+    da.scales = scales;
+    da.scale_log2 = softmax_scale(dims) * kLog2e;
+    da.max_blocks = max_blocks;
+    da.num_blocks = num_blocks;
+    da.s = s;
+    da.H = H;
+    da.B = B;
+    da.groups = groups;
+    // the decode kernel sets itself up while the plan runs, and the
+    // combine launches while the decode's last CTAs finish
+    cudaError_t e = launch_pdl(tc_decode64_kernel<kFp8>, dim3(ranges * groups),
+                               dim3(kFp8 ? kD64ThreadsFp8 : kD64Threads), kFp8 ? kD64SmemFp8 : kD64Smem, strm, mkv,
+                               da);
+    count_launch();
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    const int ctas = combine_ctas(B, s, H);
+    const int cgrid = ctas < 8 * sm_count() ? ctas : 8 * sm_count();
+    e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
+                   (const float *)da.part_o, (const float *)da.part_lse2, seq_lens, max_blocks, B, s, H,
+                   (bf16 *)out_latent, out_lse);
+    count_launch();
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 // Decode scratch for callers that pass no workspace: one array per device,
@@ -464,50 +530,9 @@ mla_status_t mla_decode(const mla_dims_t *dims, const void *q_abs, const void *c
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     } else {
-        const TcWs w = tc_ws(H, s, B);
-        if (ws_bytes < w.total) return MLA_ERR_WORKSPACE;
-        const int groups = dec_groups(H, s);
-        const int ranges = decode_ranges(H, s);
-        if (ranges <= 0) return MLA_ERR_CUDA;
-        CUtensorMap mkv;
-        if (!tmap(&mkv, cache, kRow, (uint64_t)num_blocks * kBlock, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
-        if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
-        int32_t *plan = (int32_t *)(ws + w.off_plan);
-        dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
-        count_launch();
-        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-        DecArgs da;
-        da.q_abs = (const bf16 *)q_abs;
-        da.block_table = block_table;
-        da.seq_lens = seq_lens;
-        da.plan = plan;
-        da.out = (bf16 *)out_latent;
-        da.out_lse = out_lse;
-        da.part_o = (float *)(ws + w.off_o);
-        da.part_lse2 = (float *)(ws + w.off_lse);
-        da.err = err;
-        da.limit_ns = (flags & MLA_DEBUG_STALL) ? kStallWaitLimitNs : kWaitLimitNs;
-        da.stall_tile = (flags & MLA_DEBUG_STALL) ? 0 : -1;
-        da.scale_log2 = scale_log2;
-        da.max_blocks = max_blocks;
-        da.num_blocks = num_blocks;
-        da.s = s;
-        da.H = H;
-        da.B = B;
-        da.groups = groups;
-        // the decode kernel sets itself up while the plan runs, and the
-        // combine launches while the decode's last CTAs finish
-        cudaError_t e = launch_pdl(tc_decode64_kernel, dim3(ranges * groups), dim3(kD64Threads), kD64Smem, strm,
-                                   mkv, da);
-        count_launch();
-        if (e != cudaSuccess) return MLA_ERR_CUDA;
-        const int ctas = combine_ctas(B, s, H);
-        const int cgrid = ctas < 8 * sm_count() ? ctas : 8 * sm_count();
-        e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
-                       (const float *)da.part_o, (const float *)da.part_lse2, seq_lens, max_blocks, B, s, H,
-                       (bf16 *)out_latent, out_lse);
-        count_launch();
-        if (e != cudaSuccess) return MLA_ERR_CUDA;
+        const mla_status_t r = run_tc_decode<false>(dims, q_abs, cache, nullptr, num_blocks, block_table, max_blocks,
+                                                    seq_lens, B, s, out_latent, out_lse, ws, ws_bytes, flags, strm);
+        if (r != MLA_OK) return r;
     }
     if (flags & MLA_SYNC_CHECK) {
         uint32_t host = 0;
@@ -622,25 +647,26 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
     const long long cap_blocks = (long long)max_blocks * kBlock;
     const int l_cap = cap_blocks < max_seq_len ? (int)cap_blocks : max_seq_len;
 
-    // tensor maps: the expansion GEMMs (rows x U^K_i^T, rows x U^V_i^T, one
-    // activation matrix against per-head weights) and the attention
-    CUtensorMap ma, muk, muv, mkc, mvc;
+    // tensor maps: the expansions, one GEMM each over all heads,
+    // K^C [M][H*128] = rows [M][512] . [U^K_0; ..; U^K_{H-1}]^T (the stacked
+    // [H*128][512] weights are K-major as stored), and the attention
+    CUtensorMap ma, muk, muv, mkc, mvc, skc, svc;
     if (!tmap(&ma, rows, kDc, M, 1, kRow, 0, 64, 128) ||
-        !tmap(&muk, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128) ||
-        !tmap(&muv, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 128) ||
+        !tmap(&muk, w_uk, kDc, (uint64_t)H * kDh, 1, kDc, 0, 64, 256) ||
+        !tmap(&muv, w_uv, kDc, (uint64_t)H * kDh, 1, kDc, 0, 64, 256) ||
+        !make_tmap_3d(&skc, kc, (uint64_t)H * kDh, 1, M, (uint64_t)H * kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_3d(&svc, vc, (uint64_t)H * kDh, 1, M, (uint64_t)H * kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_3d(&mkc, kc, kDh, H, M, kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_3d(&mvc, vc, kDh, H, M, kDh * 2, (uint64_t)H * kDh * 2, 64, 1, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return MLA_ERR_CUDA;
     PrefillMaps pm;
     {
-        const uint64_t qdims[4] = {(uint64_t)kDh, (uint64_t)H, (uint64_t)s, (uint64_t)B};
-        const uint64_t qstr[3] = {(uint64_t)kDh * 2, (uint64_t)H * kDh * 2, (uint64_t)s * H * kDh * 2};
-        const uint64_t rdims[4] = {(uint64_t)kDr, (uint64_t)H, (uint64_t)s, (uint64_t)B};
-        const uint64_t rstr[3] = {(uint64_t)kDr * 2, (uint64_t)H * kDr * 2, (uint64_t)s * H * kDr * 2};
-        const uint32_t box[4] = {64, 1, 128, 1};
-        if (!make_tmap_4d(&pm.qc, q_nope, qdims, qstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap_4d(&pm.qr, q_rot, rdims, rstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap_4d(&pm.out, out, qdims, qstr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        const uint64_t odims[4] = {(uint64_t)kDh, (uint64_t)H, (uint64_t)s, (uint64_t)B};
+        const uint64_t ostr[3] = {(uint64_t)kDh * 2, (uint64_t)H * kDh * 2, (uint64_t)s * H * kDh * 2};
+        const uint32_t obox[4] = {64, 1, 128, 1};
+        if (!make_tmap_4d(&pm.out, out, odims, ostr, obox, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_tmap_3d(&pm.kr, rows, kRow, M, 1, kRow * 2, (uint64_t)M * kRow * 2, 64, 128, 1,
                           CU_TENSOR_MAP_SWIZZLE_128B))
             return MLA_ERR_CUDA;
@@ -649,7 +675,7 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
     }
     if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
     {
-        const long long work = rows_total * (kRow / 8) + (long long)B * s * H * (kDr / 2);
+        const long long work = rows_total * (kRow / 8) + (long long)B * s * (kDr / 2);
         long long blocks = (work + 255) / 256;
         if (blocks > 8ll * sm_count()) blocks = 8ll * sm_count();
         prefill_prepare_kernel<<<(int)blocks, 256, 0, strm>>>((const bf16 *)cache, num_blocks, block_table,
@@ -659,12 +685,14 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
         count_launch();
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
-    if (launch_tc_gemm<128, false, TcEpiTmaStore, true>(ma, muk, M, kDh, kDc, H, TcEpiTmaStore{}, err, strm,
-                                                         &mkc) != cudaSuccess ||
-        launch_tc_gemm<128, false, TcEpiTmaStore, true>(ma, muv, M, kDh, kDc, H, TcEpiTmaStore{}, err, strm,
-                                                         &mvc) != cudaSuccess)
+    if (launch_tc_gemm<256, false, TcEpiTmaStore>(ma, muk, M, H * kDh, kDc, 1, TcEpiTmaStore{}, err, strm, &skc) !=
+            cudaSuccess ||
+        launch_tc_gemm<256, false, TcEpiTmaStore>(ma, muv, M, H * kDh, kDc, 1, TcEpiTmaStore{}, err, strm, &svc) !=
+            cudaSuccess)
         return MLA_ERR_CUDA;
     PrefillArgs pa;
+    pa.q_nope = (const bf16 *)q_nope;
+    pa.q_rot = q_rot;
     pa.seq_lens = seq_lens;
     pa.s = s;
     pa.H = H;
@@ -676,7 +704,7 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
     pa.limit_ns = kWaitLimitNs;
     static std::atomic<bool> attr_set[kMaxDevices];
     if (ensure_smem_attr(tc_prefill_kernel, kPfSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
-    tc_prefill_kernel<<<dim3((s + 255) / 256, H, B), kPfThreads, kPfSmem, strm>>>(pm, pa);
+    tc_prefill_kernel<<<dim3((s + 127) / 128, H, B), kPfThreads, kPfSmem, strm>>>(pm, pa);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (flags & MLA_SYNC_CHECK) {
@@ -685,6 +713,58 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
             cudaStreamSynchronize(strm) != cudaSuccess)
             return MLA_ERR_CUDA;
         if (h) return MLA_ERR_DEVICE;
+    }
+    return MLA_OK;
+}
+
+mla_status_t mla_append_latent_fp8(const mla_dims_t *dims, const void *c_kv, const void *k_rope, int T,
+                                   const int32_t *seq_idx, const int32_t *pos, const int32_t *block_table,
+                                   int num_seqs, int max_blocks, void *codes, float *scales, int num_blocks,
+                                   const void *kv_norm_weight, float kv_norm_eps, uint32_t *err_word, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (T < 0 || num_seqs < 0 || max_blocks < 0 || num_blocks < 0) return MLA_ERR_INVALID_ARG;
+    if (T == 0) return MLA_OK;
+    if (!c_kv || !k_rope || !seq_idx || !pos || !block_table || !codes || !scales) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(c_kv) || !aligned16(codes) || ((uintptr_t)k_rope & 3u) || ((uintptr_t)scales & 7u))
+        return MLA_ERR_INVALID_ARG;
+    if (kv_norm_weight && (!aligned16(kv_norm_weight) || !(kv_norm_eps >= 0.f))) return MLA_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    append_latent_fp8_kernel<<<(T + 7) / 8, 256, 0, s>>>((const bf16 *)c_kv, (const bf16 *)k_rope, T, seq_idx, pos,
+                                                         block_table, num_seqs, max_blocks, (uint8_t *)codes, scales,
+                                                         num_blocks, rope_table(dims), (const bf16 *)kv_norm_weight,
+                                                         kv_norm_eps, err_word);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+mla_status_t mla_decode_fp8(const mla_dims_t *dims, const void *q_abs, const void *codes, const float *scales,
+                            int num_blocks, const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                            int B, int s, void *out_latent, float *out_lse, void *workspace, size_t ws_bytes,
+                            uint32_t flags, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (B < 0 || s <= 0 || num_blocks < 0 || max_blocks < 0) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    if (num_blocks == 0 || max_blocks == 0) return MLA_ERR_INVALID_ARG;
+    if (flags & MLA_FORCE_SIMPLE) return MLA_ERR_UNSUPPORTED;
+    if (!q_abs || !codes || !scales || !block_table || !seq_lens || !out_latent) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q_abs) || !aligned16(codes) || !aligned16(scales) || !aligned16(out_latent))
+        return MLA_ERR_INVALID_ARG;
+    if (!workspace) return MLA_ERR_WORKSPACE;
+    cudaStream_t strm = as_stream(stream);
+    char *ws = (char *)workspace;
+    const mla_status_t r = run_tc_decode<true>(dims, q_abs, codes, scales, num_blocks, block_table, max_blocks,
+                                               seq_lens, B, s, out_latent, out_lse, ws, ws_bytes, flags, strm);
+    if (r != MLA_OK) return r;
+    if (flags & MLA_SYNC_CHECK) {
+        uint32_t host = 0;
+        if (cudaMemcpyAsync(&host, ws, sizeof host, cudaMemcpyDeviceToHost, strm) != cudaSuccess ||
+            cudaStreamSynchronize(strm) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (host) return MLA_ERR_DEVICE;
     }
     return MLA_OK;
 }

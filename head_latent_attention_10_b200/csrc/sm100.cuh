@@ -136,6 +136,15 @@ __device__ __forceinline__ void tma_load_4d(const CUtensorMap *map, uint64_t *ba
         : "memory");
 }
 
+// Contiguous copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // Store a tile from shared memory (tensor-map layout and swizzle) to global
 // memory; rows of the box past the tensor's extent are not written.
 // Completion is tracked per thread with bulk groups (tma_store_commit /
@@ -346,6 +355,13 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr, uint32_t row_byt
 __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t chunk_stride)
 {
     return smem_desc(saddr, chunk_stride, 1024, kSw128);
+}
+
+// Instruction descriptor for kind::f16 with f16 A and B (formats 0), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major)
+{
+    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16: bf16 A and B, fp32 D, M x N,

@@ -56,9 +56,24 @@
 // log2-sum-exp), merged by dec_combine_kernel.  Every wait is bounded; a wait
 // that gives up sets MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own
 // copies in flight and frees its TMEM.
+//
+// FP8 cache (kFp8): a page is 576 E4M3 codes per token plus two fp32 scales
+// per token (csrc/fp8.cuh).  TMA lands the codes, one 64-column box per
+// chunk (4 KB each), in the upper half of the stage and the page's 512 B of
+// scales in a side slot; two extra warps (8-9) widen them in place into the
+// same f16 tile layout the bf16 path uses, with the token's larger scale
+// s_j = max(sc_c, sc_r) factored out: the f16 values are code * sc / s_j
+// (one part exact, the other scaled by <= 1), so the logits MMA gives l_j / s_j
+// and the softmax multiplies its logits by s_j, and P_j s_j is the A operand
+// of the latent sum.  Q and P are f16; the MMAs are kind::f16 with f16
+// operands.  Chunk j's codes sit at 36,864 + 4,096 j and its f16 output at
+// 8,192 j, so output chunk j overwrites the codes of chunks 2j-9 and 2j-8: the
+// converters go in four groups (0-3 | 4-5 | 6 | 7-8) with a named barrier
+// between groups, and chunk 8's codes are read before the last barrier.
 #pragma once
 
 #include "dec_common.cuh"
+#include "fp8.cuh"
 
 namespace mla {
 
@@ -75,14 +90,25 @@ constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-5
 constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
 constexpr uint32_t kD64TmS2 = 416;                // third logits buffer: lanes 0-15, columns 416-479
 constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
+// FP8 cache: 64 more threads (the converters), per-stage scale slots
+// ([64][2] fp32) and per-token factored scales s_j ([64] fp32) after the stages
+constexpr int kD64ThreadsFp8 = kD64Threads + 64;
+constexpr int kD64F8Codes = kT64 * kRow / 2;      // 36,864: where the codes land in the stage
+constexpr int kD64F8Box = kT64 * 64;              // one 64-column box of codes (4 KB)
+constexpr int kD64OffScale = kD64Stages * kD64Stage;              // [3][64][2] fp32
+constexpr int kD64OffSmax = kD64OffScale + kD64Stages * 512;      // [3][64] fp32
+constexpr int kD64OffBarFp8 = kD64OffSmax + kD64Stages * 256;
+constexpr int kD64SmemFp8 = kD64OffBarFp8 + 512 + 1024;
 
-__global__ void __launch_bounds__(kD64Threads, 1)
+template <bool kFp8>
+__global__ void __launch_bounds__(kFp8 ? kD64ThreadsFp8 : kD64Threads, 1)
 tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
 {
     extern __shared__ uint8_t d64_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(d64_smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kD64OffBar);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (kFp8 ? kD64OffBarFp8 : kD64OffBar));
+    uint64_t *cv_full = bars + 32;   // [3] FP8: the stage's codes widened to f16 (2 converter warps)
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
     uint64_t *kv_empty = bars + 21;  // [3] P.C MMAs of the stage done -> TMA, softmax
     // Q of segment n is in TMEM once q_cnt >= 4 (n + 1) (each softmax warp adds
@@ -113,6 +139,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             sm100::mbar_init(&s_free[i], 4);
         }
         for (int i = 0; i < kD64Stages; ++i) p_cnt[i] = 0;
+        if constexpr (kFp8)
+            for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&cv_full[i], 2);
         sm100::mbar_init(mma_done, 7);
         *abort_flag = 0;
         sm100::fence_mbar_init();
@@ -149,8 +177,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 if (ahead.ok) {
                     // warm L2 with a tile further ahead while this stage waits to be freed
                     const int pb = page_of(ahead);
-                    if (pb >= 0)
+                    if (pb >= 0) {
                         for (int j = 0; j < 9; ++j) sm100::tma_prefetch_3d(&map_kv, 64 * j, pb * kBlock, 0);
+                        if constexpr (kFp8)
+                            for (int e = 0; e < 4; ++e)
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(a.scales + (long long)pb * 128 + 32 * e));
+                    }
                     ahead.advance();
                 }
                 if (k >= kD64Stages)
@@ -170,9 +202,18 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     it.advance();
                     continue;
                 }
-                sm100::mbar_arrive_expect_tx(&kv_full[st], kD64Stage);
-                for (int j = 0; j < 9; ++j)
-                    sm100::tma_load_3d(&map_kv, &kv_full[st], dst + j * kD64Chunk, 64 * j, blk * kBlock, 0);
+                if constexpr (kFp8) {
+                    sm100::mbar_arrive_expect_tx(&kv_full[st], 9 * kD64F8Box + 512);
+                    for (int j = 0; j < 9; ++j)
+                        sm100::tma_load_3d(&map_kv, &kv_full[st], dst + kD64F8Codes + j * kD64F8Box, 64 * j,
+                                           blk * kBlock, 0);
+                    sm100::bulk_load(smem + kD64OffScale + st * 512, a.scales + (long long)blk * 128, 512,
+                                     &kv_full[st]);
+                } else {
+                    sm100::mbar_arrive_expect_tx(&kv_full[st], kD64Stage);
+                    for (int j = 0; j < 9; ++j)
+                        sm100::tma_load_3d(&map_kv, &kv_full[st], dst + j * kD64Chunk, 64 * j, blk * kBlock, 0);
+                }
                 issued_k = k + 1;
                 it.advance();
             }
@@ -189,7 +230,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // logits buffer, all 36 K steps
         const int b = warp - 1;
         const uint32_t scol = b < 2 ? 64u * b : kD64TmS2;
-        const uint32_t idesc_s = sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
+        const uint32_t idesc_s = kFp8 ? sm100::idesc_f16(kGroupRows, kT64, 0, 0) : sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
         is.init(seq_start, a.B, lo, hi);
         int q_seg = -1;
@@ -207,7 +248,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 q_seg = is.seg;
             }
             if (!ok) break;
-            ok = sm100::warp_wait(&kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
+            ok = sm100::warp_wait(kFp8 ? &cv_full[st] : &kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
             if (ok && kk >= 3) ok = sm100::warp_wait(&s_free[b], ((kk / 3) - 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
@@ -223,6 +264,90 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             }
             __syncwarp();
             is.advance();
+        }
+    } else if (kFp8 && warp >= 8) {
+        // ------------------------------------------------ FP8 -> f16 (warps 8-9)
+        // thread ct: rows rr_i = ct / 4 + 16 i (i = 0..3), 16-code segment g =
+        // ct % 4 of each 64-column chunk (a warp reads 512 contiguous bytes)
+        const int ct = threadIdx.x - kD64Threads, g = ct & 3;
+        TileIter it;
+        it.init(seq_start, a.B, lo, hi);
+        bool ok = true;
+        while (ok && it.ok) {
+            const int k = it.k, st = k % kD64Stages;
+            ok = sm100::warp_wait(&kv_full[st], (k / kD64Stages) & 1, abort_flag, a.err, lim);
+            // both converter warps go on only if both saw the page land: they
+            // meet at named barriers below, which neither may skip
+            {
+                uint32_t both;
+                asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+                             "bar.red.and.pred p, 3, 64, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                             : "=r"(both) : "r"((uint32_t)ok) : "memory");
+                ok = both != 0;
+            }
+            if (!ok) break;
+            uint8_t *stg = stages + st * kD64Stage;
+            const float2 *scl = reinterpret_cast<const float2 *>(smem + kD64OffScale + st * 512);
+            float *smax = reinterpret_cast<float *>(smem + kD64OffSmax + st * 256);
+            uint32_t rat_c[4], rat_r[4];   // f16x2 ratios sc / s_j of the thread's rows
+            bool one_c[4], one_r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = (ct >> 2) + 16 * i;
+                const float2 sc = scl[rr];
+                const float m = fmaxf(sc.x, sc.y);
+                const float fc = sc.x / m, fr = sc.y / m;
+                one_c[i] = fc == 1.f;
+                one_r[i] = fr == 1.f;
+                const __half2 hc = __float2half2_rn(fc), hr = __float2half2_rn(fr);
+                rat_c[i] = *reinterpret_cast<const uint32_t *>(&hc);
+                rat_r[i] = *reinterpret_cast<const uint32_t *>(&hr);
+                if (g == 0) smax[rr] = m;
+            }
+            auto read = [&](int j, uint4 *in) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    in[i] = *reinterpret_cast<const uint4 *>(stg + kD64F8Codes + j * kD64F8Box +
+                                                             64 * ((ct >> 2) + 16 * i) + 16 * g);
+            };
+            auto write = [&](int j, const uint4 *in, const uint32_t *rat, const bool *one) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = (ct >> 2) + 16 * i;
+                    const uint16_t *c = reinterpret_cast<const uint16_t *>(&in[i]);
+                    uint32_t h[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) h[e] = e4m3x2_to_f16x2(c[e]);
+                    if (!one[i]) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            __half2 v = *reinterpret_cast<__half2 *>(&h[e]);
+                            v = __hmul2(v, *reinterpret_cast<const __half2 *>(&rat[i]));
+                            h[e] = *reinterpret_cast<uint32_t *>(&v);
+                        }
+                    }
+                    uint8_t *rowp = stg + j * kD64Chunk + rr * 128;
+                    *reinterpret_cast<uint4 *>(rowp + (((2 * g) ^ (rr & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(rowp + (((2 * g + 1) ^ (rr & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+                }
+            };
+            auto group_sync = [] { asm volatile("bar.sync 3, 64;" ::: "memory"); };
+            uint4 in[4], in8[4];
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) { read(j, in); write(j, in, rat_c, one_c); }
+            group_sync();
+#pragma unroll 1
+            for (int j = 4; j < 6; ++j) { read(j, in); write(j, in, rat_c, one_c); }
+            group_sync();
+            read(6, in); write(6, in, rat_c, one_c);
+            group_sync();
+            read(7, in); read(8, in8); write(7, in, rat_c, one_c);
+            group_sync();
+            write(8, in8, rat_r, one_r);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(&cv_full[st]);
+            it.advance();
         }
     } else {
         // -------------------------------------------------------- softmax
@@ -252,6 +377,19 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
 #pragma unroll
                 for (int e = 0; e < 12; ++e)
                     v[e] = row_ok ? __ldg(q4 + 8 * (3 * g + (e >> 2)) + (e & 3)) : make_uint4(0, 0, 0, 0);
+                if constexpr (kFp8) {
+                    // the FP8 path's MMAs take f16 operands
+#pragma unroll
+                    for (int e = 0; e < 12; ++e) {
+                        uint32_t *w = reinterpret_cast<uint32_t *>(&v[e]);
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) {
+                            const __half2 hh = __float22half2_rn(
+                                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[f])));
+                            w[f] = *reinterpret_cast<const uint32_t *>(&hh);
+                        }
+                    }
+                }
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
                     sm100::tmem_st16x2_16(lane_base + kD64TmQ + 32 * (3 * g + j), reinterpret_cast<const uint32_t *>(v + 4 * j));
@@ -277,7 +415,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         it.init(seq_start, a.B, lo, hi);
         float m_run = -INFINITY, l_run = 0.f;
         int nvis = 0, nseq = 0;
-        const uint32_t idesc_o = sm100::idesc_bf16(kGroupRows, 256, 0, 1);
+        const uint32_t idesc_o = kFp8 ? sm100::idesc_f16(kGroupRows, 256, 0, 1) : sm100::idesc_bf16(kGroupRows, 256, 0, 1);
         bool ok = true;
         if (it.ok) write_q(it.seq);
         while (ok && it.ok) {
@@ -307,6 +445,16 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 if (lane == 0) sm100::mbar_arrive(&s_free[sb]);
             }
             const int tok0 = it.tt * kT64 + (srow ? 0 : 32);
+            // FP8: the factored per-token scales s_j of this thread's 32 columns,
+            // written by the converters before they released the stage
+            const float *smx = reinterpret_cast<const float *>(smem + kD64OffSmax + (k % kD64Stages) * 256) +
+                               (srow ? 0 : 32);
+            if constexpr (kFp8) {
+                ok = sm100::warp_wait(&cv_full[k % kD64Stages], (k / kD64Stages) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) x[c] *= smx[c];
+            }
             if (tok0 + 32 > nvis) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
@@ -352,7 +500,15 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             for (int c = 0; c < 16; ++c) {
                 const float p0 = ex2(fmaf(x[2 * c], a.scale_log2, -mu));
                 const float p1 = ex2(fmaf(x[2 * c + 1], a.scale_log2, -mu));
-                pw[c] = pack_bf162(p0, p1);
+                if constexpr (kFp8) {
+                    // a masked column has p = 0 and may sit past the sequence
+                    // end, where the scale can be NaN: keep its P exactly 0
+                    const float2 sj = *reinterpret_cast<const float2 *>(smx + 2 * c);
+                    const __half2 hh = __floats2half2_rn(p0 > 0.f ? p0 * sj.x : 0.f, p1 > 0.f ? p1 * sj.y : 0.f);
+                    pw[c] = *reinterpret_cast<const uint32_t *>(&hh);
+                } else {
+                    pw[c] = pack_bf162(p0, p1);
+                }
                 lsum += p0 + p1;
             }
             l_run += lsum;
@@ -465,7 +621,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     sm100::pdl_trigger();   // the combine may start launching
     sm100::tc_fence_before();
     __syncthreads();
-    if (warp >= 1) {
+    if (warp >= 1 && warp < 8) {
         // every MMA this CTA issued retires before its TMEM is released
         if (lane == 0) sm100::umma_commit(mma_done);
         __syncwarp();

@@ -9,10 +9,8 @@
 // with tcgen05.ld (one TMEM lane = one output row per thread) and hand 16
 // columns at a time to the epilogue functor.
 //
-// A is K-major (rows of K contiguous); with kAshared every batch entry z uses
-// batch entry 0 of A (one activation matrix against per-head weights).  B is
-// either K-major (B^T stored row-major, e.g. a weight [N][K]) or MN-major (B
-// stored [K][N]).
+// A is K-major (rows of K contiguous).  B is either K-major (B^T stored
+// row-major, e.g. a weight [N][K]) or MN-major (B stored [K][N]).
 // Tensor maps are 3-D: A {K, M, Z}, B K-major {K, N, Z}, B MN-major {N, K, Z}.
 #pragma once
 
@@ -33,7 +31,7 @@ struct GemmSmem {
     static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
 };
 
-template <int BN, bool kBmn, class Epi, bool kAshared = false>
+template <int BN, bool kBmn, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                const __grid_constant__ CUtensorMap mapC, int M, int N, int K, Epi epi, uint32_t *err,
@@ -85,7 +83,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 uint8_t *b = a + S::A;
                 sm100::mbar_arrive_expect_tx(&full[s], S::STAGE);
                 const int kx = kb * 64;
-                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, kAshared ? 0 : z);
+                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, z);
                 if (kBmn) {
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)

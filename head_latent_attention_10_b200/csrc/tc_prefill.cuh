@@ -12,51 +12,53 @@
 // With many queries per sequence the expanded form costs fewer flops than the
 // absorbed one (2 (192 + 128) per query, key and head against 2 (576 + 512)),
 // and the step is bound by the tensor cores: a FlashAttention-style loop on
-// tcgen05.  CTA (block, head i, sequence b) owns two 128-query tiles of head
-// i (MMA M = 128 each) and streams 128-key tiles of K = [K^C | k^R] and V^C:
-//   S_u(k) = Q_u K_k^T    N=128, K=192 (12 MMAs)   fp32 in TMEM
-//   P_u(k) = exp2(S_u(k) scale log2 e - m_u)       bf16, written over S_u(k)
-//   O_u   += P_u(k) V_k   N=128, K=128 (8 MMAs, P read from TMEM)
-// TMEM (512 columns): S_0/P_0 0-127, S_1/P_1 128-255, O_0 256-383, O_1
-// 384-511.  Each tile u has its own issuing thread (warp 1 + u) and softmax
-// warpgroup (warps 4-7, 8-11; thread = query row), so tile u's chain
-// S_u(k) -> softmax -> P_u(k) V_k -> S_u(k+1) runs while the other tile's
-// MMAs keep the tensor pipe busy.  S_u(k+1) overwrites P_u(k), so its issuer
-// waits for P_u(k) V_k to complete first; that also means O_u is idle while
-// the softmax rescales it.  Lazy rescaling as in the decode.
-// Shared memory: Q_0, Q_1 (three 64-column chunks each, [128 rows][128 B],
-// 128-byte swizzle: q^C 0-63, q^C 64-127, rotated q^R), two K slots (K^C
-// 0-63, 64-127, k^R) and one V slot (V^C 0-63, 64-127): 224 KB.  Warp 0
-// loads with TMA (no cluster multicast).  Every wait is bounded.
+// tcgen05.  CTA (128-query tile, head i, sequence b), the tile as MMA M = 128,
+// streams 128-key tiles of K = [K^C | k^R] and V^C:
+//   S(k) = Q K_k^T    N=128, K=192: 12 MMAs, Q read from TMEM
+//   P(k) = exp2(S(k) scale log2 e - m)           bf16, one thread per query row
+//   O   += P(k) V_k   N=128, K=128: 8 MMAs, P read from TMEM
+// TMEM (512 columns): S 0-127, P(k % 2) 128-191 / 192-255, O 256-383,
+// Q 384-479 (192 bf16 per row, written by the softmax warps at the start).
+// With Q and P in TMEM, shared memory holds only key and value tiles: a
+// 3-slot ring of K tiles (K^C 0-63, K^C 64-127, k^R; 48 KB each) and a 2-slot
+// ring of V tiles (V^C 0-63, 64-127; 32 KB each), 208 KB, each ring fed by
+// its own loader warp (0: K, 6: V) so that neither waits behind the other.
+// Warp 1 issues S(k+1) as soon as the softmax warps (2-5) have read S(k) out
+// of TMEM, so the logits of the next tile run while the softmax of this one
+// computes, then P(k) V_k once P(k) is written.  The causal mask applies to
+// the tiles that straddle the diagonal; lazy rescaling as in the decode (O
+// is rescaled in TMEM only when the running max grows by more than 8, after
+// the previous P V has retired).  Every wait is bounded; no TMA load uses
+// cluster multicast.
 #pragma once
 
 #include "dec_common.cuh"
 
 namespace mla {
 
-constexpr int kPfThreads = 384;
-constexpr int kPfChunk = 128 * 128;                    // [128 rows][64 bf16]: 16 KB
-constexpr int kPfOffQ = 0;                             // Q_u chunk c at (3u + c) * 16 KB
-constexpr int kPfOffK = 6 * kPfChunk;                  // K slot j chunk c at +(3j + c) * 16 KB
-constexpr int kPfOffV = 12 * kPfChunk;                 // V chunk c at +c * 16 KB
-constexpr int kPfOffBar = 14 * kPfChunk;               // 229,376
+constexpr int kPfThreads = 224;                        // warps: 0 K loads, 1 MMA, 2-5 softmax, 6 V loads
+constexpr int kPfChunk = 128 * 128;                    // [128 rows][64 bf16], 128-byte swizzle: 16 KB
+constexpr int kPfKSlots = 3, kPfVSlots = 2;
+constexpr int kPfOffK = 0;                             // K slot j: chunks 3j .. 3j+2
+constexpr int kPfOffV = kPfKSlots * 3 * kPfChunk;      // V slot j: 2 chunks
+constexpr int kPfOffBar = kPfOffV + kPfVSlots * 2 * kPfChunk;   // 212,992
 constexpr int kPfSmem = kPfOffBar + 256 + 1024;        // barriers, alignment slack
-constexpr uint32_t kPfTmS = 0, kPfTmO = 256;
+constexpr uint32_t kPfTmS = 0, kPfTmP = 128, kPfTmO = 256, kPfTmQ = 384;
 
 // Tensor maps of one call.  Rows of K^C, V^C and the gathered latents are
-// [B * Lpad] long (sequence b at rows b * Lpad ..); queries and outputs are
-// [B][s][H][.] with the sequence as the outermost dimension, so a 128-row
-// tile is clipped at the end of its own sequence.
+// [B * Lpad] long (sequence b at rows b * Lpad ..); outputs are [B][s][H][128]
+// with the sequence as the outermost dimension, so a 128-row tile is clipped
+// at the end of its own sequence.
 struct PrefillMaps {
-    CUtensorMap qc;    // q^C         {128, H, s, B}, box {64, 1, 128, 1}
-    CUtensorMap qr;    // rotated q^R {64, H, s, B},  box {64, 1, 128, 1}
-    CUtensorMap kc;    // K^C         {128, H, B Lpad}, box {64, 1, 128}
-    CUtensorMap vc;    // V^C         {128, H, B Lpad}, box {64, 1, 128}
+    CUtensorMap kc;    // K^C   {128, H, B Lpad}, box {64, 1, 128}
+    CUtensorMap vc;    // V^C   {128, H, B Lpad}, box {64, 1, 128}
     CUtensorMap kr;    // gathered rows {576, B Lpad, 1}, box {64, 128, 1}, read at x = 512
-    CUtensorMap out;   // out         {128, H, s, B}, box {64, 1, 128, 1}
+    CUtensorMap out;   // out   {128, H, s, B}, box {64, 1, 128, 1}
 };
 
 struct PrefillArgs {
+    const bf16 *q_nope;           // [B*s][H][128]
+    const bf16 *q_rot;            // [B*s][H][64], rotated
     const int32_t *seq_lens;
     int s, H, lpad, l_cap;        // l_cap: the largest valid sequence length
     float scale_log2;
@@ -82,41 +84,43 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
     extern __shared__ uint8_t pf_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kPfOffBar);
-    uint64_t *q_full = bars;            // Q_0 and Q_1 loaded
-    uint64_t *k_full = bars + 1;        // [2] K slot loaded
-    uint64_t *v_full = bars + 3;        // V buffer loaded
-    uint64_t *k_free = bars + 4;        // [2u + slot]: S_u of the slot's tile done
-    uint64_t *v_free = bars + 8;        // [u]: P_u V of the buffer's tile done
-    uint64_t *s_full = bars + 10;       // [u] S_u(k) in TMEM
-    uint64_t *p_full = bars + 12;       // [u] P_u(k) in TMEM, O_u rescaled (4 softmax warps arrive)
-    uint64_t *pv_done = bars + 14;      // [u] P_u(k) V_k done
-    uint64_t *done = bars + 16;         // both issuers' last MMAs done (teardown)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 17);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 18);
+    uint64_t *k_full = bars;            // [3] K slot loaded
+    uint64_t *k_free = bars + 3;        // [3] S of the slot's tile done
+    uint64_t *v_full = bars + 6;        // [2] V slot loaded
+    uint64_t *v_free = bars + 8;        // [2] P V of the slot's tile done
+    uint64_t *q_ready = bars + 10;      // Q in TMEM (4 softmax warps)
+    uint64_t *s_full = bars + 11;       // S(k) in TMEM
+    uint64_t *s_free = bars + 12;       // S(k) read out (4 softmax warps)
+    uint64_t *p_full = bars + 13;       // [2] P(k) in TMEM and O rescaled (4 softmax warps)
+    uint64_t *pv_done = bars + 15;      // [2] P(k) V_k done
+    uint64_t *done = bars + 17;         // the issuer's last MMAs done (teardown)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = gridDim.x - 1 - blockIdx.x;   // the longest rows of the causal triangle first
     const int head = blockIdx.y, b = blockIdx.z;
-    const int q0 = 256 * qb;
+    const int q0 = 128 * qb;
     const int L = a.seq_lens[b];
     const bool valid = prefill_valid(L, a.s, a.l_cap);
-    const int nk0 = valid ? prefill_tiles(q0, a.s, L) : 0;
-    const int nk1 = valid ? prefill_tiles(q0 + 128, a.s, L) : 0;
-    const int nkmax = nk0 > nk1 ? nk0 : nk1;
+    const int nk = valid ? prefill_tiles(q0, a.s, L) : 0;
     const int row0 = b * a.lpad;                 // this sequence's first key row
 
     if (threadIdx.x == 0) {
-        sm100::mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kPfKSlots; ++i) {
             sm100::mbar_init(&k_full[i], 1);
-            sm100::mbar_init(&s_full[i], 1);
+            sm100::mbar_init(&k_free[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            sm100::mbar_init(&v_full[i], 1);
+            sm100::mbar_init(&v_free[i], 1);
             sm100::mbar_init(&p_full[i], 4);
             sm100::mbar_init(&pv_done[i], 1);
-            sm100::mbar_init(&v_free[i], 1);
         }
-        for (int i = 0; i < 4; ++i) sm100::mbar_init(&k_free[i], 1);
-        sm100::mbar_init(v_full, 1);
-        sm100::mbar_init(done, 2);
+        sm100::mbar_init(q_ready, 4);
+        sm100::mbar_init(s_full, 1);
+        sm100::mbar_init(s_free, 4);
+        sm100::mbar_init(done, 1);
         *abort_flag = 0;
         sm100::fence_mbar_init();
         sm100::prefetch_tensormap(&maps.kc);
@@ -135,124 +139,136 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
     const unsigned long long drain = lim > 200000000ull ? lim : 200000000ull;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ loads
-        if (lane == 0 && nkmax > 0) {
-            auto load_k = [&](int k) {
-                uint8_t *dst = smem + kPfOffK + 3 * (k & 1) * kPfChunk;
+        // ----------------------------------------------------------- K loads
+        if (lane == 0 && nk > 0) {
+            int issued = 0;
+            for (int k = 0; k < nk; ++k) {
+                const int sl = k % kPfKSlots;
+                if (k >= kPfKSlots &&
+                    !sm100::mbar_wait(&k_free[sl], ((k / kPfKSlots) - 1) & 1, abort_flag, a.err, lim))
+                    break;
+                uint8_t *dst = smem + kPfOffK + 3 * sl * kPfChunk;
                 const int r = row0 + 128 * k;
-                sm100::mbar_arrive_expect_tx(&k_full[k & 1], 3 * kPfChunk);
-                sm100::tma_load_3d(&maps.kc, &k_full[k & 1], dst, 0, head, r);
-                sm100::tma_load_3d(&maps.kc, &k_full[k & 1], dst + kPfChunk, 64, head, r);
-                sm100::tma_load_3d(&maps.kr, &k_full[k & 1], dst + 2 * kPfChunk, kDc, r, 0);
-            };
-            auto load_v = [&](int k) {
-                const int r = row0 + 128 * k;
-                sm100::mbar_arrive_expect_tx(v_full, 2 * kPfChunk);
-                sm100::tma_load_3d(&maps.vc, v_full, smem + kPfOffV, 0, head, r);
-                sm100::tma_load_3d(&maps.vc, v_full, smem + kPfOffV + kPfChunk, 64, head, r);
-            };
-            // a K slot (or the V buffer) is free once every query tile that
-            // reads tile k is done with it; tile u reads the tiles [0, nk_u)
-            auto wait_free = [&](uint64_t *bar0, uint64_t *bar1, int k, uint32_t parity) -> bool {
-                if (k < nk0 && !sm100::mbar_wait(bar0, parity, abort_flag, a.err, lim)) return false;
-                if (k < nk1 && !sm100::mbar_wait(bar1, parity, abort_flag, a.err, lim)) return false;
-                return true;
-            };
-            sm100::mbar_arrive_expect_tx(q_full, 6 * kPfChunk);
-            for (int u = 0; u < 2; ++u) {
-                uint8_t *qd = smem + kPfOffQ + 3 * u * kPfChunk;
-                sm100::tma_load_4d(&maps.qc, q_full, qd, 0, head, q0 + 128 * u, b);
-                sm100::tma_load_4d(&maps.qc, q_full, qd + kPfChunk, 64, head, q0 + 128 * u, b);
-                sm100::tma_load_4d(&maps.qr, q_full, qd + 2 * kPfChunk, 0, head, q0 + 128 * u, b);
+                sm100::mbar_arrive_expect_tx(&k_full[sl], 3 * kPfChunk);
+                sm100::tma_load_3d(&maps.kc, &k_full[sl], dst, 0, head, r);
+                sm100::tma_load_3d(&maps.kc, &k_full[sl], dst + kPfChunk, 64, head, r);
+                sm100::tma_load_3d(&maps.kr, &k_full[sl], dst + 2 * kPfChunk, kDc, r, 0);
+                issued = k + 1;
             }
-            load_k(0);
-            int k_issued = 1, v_issued = 1;
-            if (nkmax > 1) {
-                load_k(1);
-                k_issued = 2;
-            }
-            load_v(0);
-            for (int k = 0; k < nkmax; ++k) {
-                // K slot of tile k -> tile k + 2, once the S MMAs of tile k are done
-                if (k + 2 < nkmax) {
-                    if (!wait_free(&k_free[k & 1], &k_free[2 + (k & 1)], k, (k >> 1) & 1)) break;
-                    load_k(k + 2);
-                    k_issued = k + 3;
-                }
-                // V buffer of tile k -> tile k + 1, once the P V MMAs of tile k are done
-                if (k + 1 < nkmax) {
-                    if (!wait_free(&v_free[0], &v_free[1], k, k & 1)) break;
-                    load_v(k + 1);
-                    v_issued = k + 2;
-                }
-            }
-            if (*abort_flag) {
-                // let the copies in flight land before the CTA can exit
+            if (*abort_flag) {   // let the copies in flight land before the CTA can exit
                 volatile int no_abort = 0;
-                sm100::mbar_wait(q_full, 0, &no_abort, a.err, drain);
-                for (int k = k_issued - 2 < 0 ? 0 : k_issued - 2; k < k_issued; ++k)
-                    sm100::mbar_wait(&k_full[k & 1], (k >> 1) & 1, &no_abort, a.err, drain);
-                sm100::mbar_wait(v_full, (v_issued - 1) & 1, &no_abort, a.err, drain);
+                for (int k = issued - kPfKSlots < 0 ? 0 : issued - kPfKSlots; k < issued; ++k)
+                    sm100::mbar_wait(&k_full[k % kPfKSlots], (k / kPfKSlots) & 1, &no_abort, a.err, drain);
             }
         }
-    } else if (warp == 1 || warp == 2) {
-        // ------------------------------------------- MMA issue, query tile u
-        const int u = warp - 1;
-        const int nk = u ? nk1 : nk0;
+    } else if (warp == 6) {
+        // ----------------------------------------------------------- V loads
+        if (lane == 0 && nk > 0) {
+            int issued = 0;
+            for (int k = 0; k < nk; ++k) {
+                const int sl = k & 1;
+                if (k >= 2 && !sm100::mbar_wait(&v_free[sl], ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
+                uint8_t *dst = smem + kPfOffV + 2 * sl * kPfChunk;
+                const int r = row0 + 128 * k;
+                sm100::mbar_arrive_expect_tx(&v_full[sl], 2 * kPfChunk);
+                sm100::tma_load_3d(&maps.vc, &v_full[sl], dst, 0, head, r);
+                sm100::tma_load_3d(&maps.vc, &v_full[sl], dst + kPfChunk, 64, head, r);
+                issued = k + 1;
+            }
+            if (*abort_flag) {
+                volatile int no_abort = 0;
+                for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
+                    sm100::mbar_wait(&v_full[k & 1], (k >> 1) & 1, &no_abort, a.err, drain);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issue
         if (lane == 0) {
             const uint32_t idesc_s = sm100::idesc_bf16(128, 128, 0, 0);
             const uint32_t idesc_o = sm100::idesc_bf16(128, 128, 0, 1);
-            const uint32_t tm_s = tmem + kPfTmS + 128 * u, tm_o = tmem + kPfTmO + 128 * u;
-            const uint32_t qa = sm100::smem_u32(smem + kPfOffQ + 3 * u * kPfChunk);
-            const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(smem + kPfOffV), kPfChunk);
-            bool ok = nk == 0 || sm100::mbar_wait(q_full, 0, abort_flag, a.err, lim);
-            for (int k = 0; ok && k < nk; ++k) {
-                ok = sm100::mbar_wait(&k_full[k & 1], (k >> 1) & 1, abort_flag, a.err, lim);
-                // S_u(k) overwrites P_u(k-1): its P V must have completed
-                if (ok && k > 0) ok = sm100::mbar_wait(&pv_done[u], (k - 1) & 1, abort_flag, a.err, lim);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                const uint32_t ka = sm100::smem_u32(smem + kPfOffK + 3 * (k & 1) * kPfChunk);
+            bool ok = nk == 0 || sm100::mbar_wait(q_ready, 0, abort_flag, a.err, lim);
+            // step k issues S(k), then P(k-1) V_{k-1}
+            for (int k = 0; ok && k <= nk; ++k) {
+                if (k < nk) {
+                    const int sl = k % kPfKSlots;
+                    ok = sm100::mbar_wait(&k_full[sl], (k / kPfKSlots) & 1, abort_flag, a.err, lim);
+                    // S(k) overwrites S(k-1): the softmax must have read it
+                    if (ok && k > 0) ok = sm100::mbar_wait(s_free, (k - 1) & 1, abort_flag, a.err, lim);
+                    if (!ok) break;
+                    sm100::tc_fence_after();
+                    const uint32_t ka = sm100::smem_u32(smem + kPfOffK + 3 * sl * kPfChunk);
 #pragma unroll
-                for (int step = 0; step < 12; ++step) {      // q^C 0-63, q^C 64-127, q^R
-                    const uint32_t off = (step >> 2) * kPfChunk + (step & 3) * 32;
-                    sm100::umma_ss(tm_s, sm100::desc_kmajor(qa + off, 128, sm100::kSw128),
-                                   sm100::desc_kmajor(ka + off, 128, sm100::kSw128), idesc_s, step > 0);
+                    for (int step = 0; step < 12; ++step)      // q^C 0-63, q^C 64-127, q^R
+                        sm100::umma_ts(tmem + kPfTmS, tmem + kPfTmQ + 8 * step,
+                                       sm100::desc_kmajor(ka + (step >> 2) * kPfChunk + (step & 3) * 32, 128,
+                                                          sm100::kSw128),
+                                       idesc_s, step > 0);
+                    sm100::umma_commit(s_full);
+                    sm100::umma_commit(&k_free[sl]);
                 }
-                sm100::umma_commit(&s_full[u]);
-                sm100::umma_commit(&k_free[2 * u + (k & 1)]);
-                ok = sm100::mbar_wait(&p_full[u], k & 1, abort_flag, a.err, lim) &&
-                     sm100::mbar_wait(v_full, k & 1, abort_flag, a.err, lim);
-                if (!ok) break;
-                sm100::tc_fence_after();
+                if (k > 0) {
+                    const int j = k - 1, pb = j & 1;
+                    ok = sm100::mbar_wait(&p_full[pb], (j >> 1) & 1, abort_flag, a.err, lim) &&
+                         sm100::mbar_wait(&v_full[pb], (j >> 1) & 1, abort_flag, a.err, lim);
+                    if (!ok) break;
+                    sm100::tc_fence_after();
+                    const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(smem + kPfOffV + 2 * pb * kPfChunk),
+                                                                  kPfChunk);
 #pragma unroll
-                for (int kq = 0; kq < 8; ++kq)               // 16 keys per MMA: 8 TMEM columns of P
-                    sm100::umma_ts(tm_o, tm_s + 8 * kq, vd + (uint64_t)((kq * 2048) >> 4), idesc_o,
-                                   (k > 0 || kq > 0) ? 1u : 0u);
-                sm100::umma_commit(&pv_done[u]);
-                sm100::umma_commit(&v_free[u]);
+                    for (int kq = 0; kq < 8; ++kq)           // 16 keys per MMA: 8 TMEM columns of P
+                        sm100::umma_ts(tmem + kPfTmO, tmem + kPfTmP + 64 * pb + 8 * kq,
+                                       vd + (uint64_t)((kq * 2048) >> 4), idesc_o, (j > 0 || kq > 0) ? 1u : 0u);
+                    sm100::umma_commit(&pv_done[pb]);
+                    sm100::umma_commit(&v_free[pb]);
+                }
             }
             sm100::umma_commit(done);
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ------------------------------------------- softmax of query tile u
-        const int u = (warp - 4) >> 2, qd = warp & 3;
-        const int nk = u ? nk1 : nk0;
-        const int r = 32 * qd + lane, t = q0 + 128 * u + r;
+    } else if (warp >= 2 && warp <= 5) {
+        // ------------------------------------------------------ softmax
+        // warp w owns TMEM lane quarter w % 4; thread = query row r
+        const int qd = warp & 3;
+        const int r = 32 * qd + lane, t = q0 + r;
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        const uint32_t tm_s = tmem + lane_off + kPfTmS + 128 * u, tm_o = tmem + lane_off + kPfTmO + 128 * u;
-        const int nvis = (t < a.s) ? L - a.s + t + 1 : 0;    // keys [0, nvis) visible to row t
-        float m_run = -INFINITY, l_run = 0.f;
+        const uint32_t tm_s = tmem + lane_off + kPfTmS, tm_p = tmem + lane_off + kPfTmP;
+        const uint32_t tm_o = tmem + lane_off + kPfTmO, tm_q = tmem + lane_off + kPfTmQ;
+        const bool has_row = t < a.s;
+        const int nvis = has_row ? L - a.s + t + 1 : 0;   // keys [0, nvis) visible to row t
         bool ok = true;
+        if (nk > 0) {
+            // this row's query [q^C | rotated q^R] into TMEM (192 bf16 = 96 columns)
+            const long long qrow = ((long long)b * a.s + (has_row ? t : 0)) * a.H + head;
+            const uint4 *qc = reinterpret_cast<const uint4 *>(a.q_nope + qrow * kDh);
+            const uint4 *qr = reinterpret_cast<const uint4 *>(a.q_rot + qrow * kDr);
+#pragma unroll
+            for (int c = 0; c < 3; ++c) {
+                uint4 v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int u = 8 * c + e;   // 16-byte unit of the 384-byte row
+                    v[e] = !has_row ? make_uint4(0, 0, 0, 0) : (u < 16 ? __ldg(qc + u) : __ldg(qr + (u - 16)));
+                }
+                sm100::tmem_st32(tm_q + 32 * c, reinterpret_cast<const uint32_t *>(v));
+            }
+            sm100::tmem_wait_st();
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(q_ready);
+        }
+        float m_run = -INFINITY, l_run = 0.f;
         for (int k = 0; ok && k < nk; ++k) {
-            ok = sm100::warp_wait(&s_full[u], k & 1, abort_flag, a.err, lim);
+            const int pb = k & 1;
+            ok = sm100::warp_wait(s_full, k & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
             uint32_t x[128];
 #pragma unroll
             for (int c = 0; c < 128; c += 32) sm100::tmem_ld32(tm_s + c, x + c);
             sm100::tmem_wait_ld();
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) sm100::mbar_arrive(s_free);      // S(k+1) may go in now
             const int key0 = 128 * k;
             if (key0 + 128 > nvis) {
 #pragma unroll
@@ -281,13 +297,20 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
                 x[c] = pack_bf162(p0, p1);
             }
             l_run += lsum;
-            // P_u(k) over the first 64 columns of S_u(k) (this thread's own
-            // lane, read above)
-            sm100::tmem_st32(tm_s, x);
-            sm100::tmem_st32(tm_s + 32, x + 32);
-            // O_u holds the tiles before k, whose P V completed before S_u(k)
-            // was issued: rescale this thread's row in place
+            // P(k) into buffer pb once P(k-2) V_{k-2}, its last reader, is done
+            if (k >= 2) {
+                ok = sm100::warp_wait(&pv_done[pb], ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
+            }
+            sm100::tmem_st32(tm_p + 64 * pb, x);
+            sm100::tmem_st32(tm_p + 64 * pb + 32, x + 32);
             if (__any_sync(0xffffffffu, rescale)) {
+                // O holds the tiles before k: let P(k-1) V_{k-1} retire, then
+                // scale this thread's row in place
+                ok = sm100::warp_wait(&pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < 128; c += 32) {
                     uint32_t ov[32];
@@ -301,20 +324,19 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
             __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(&p_full[u]);
+            if (lane == 0) sm100::mbar_arrive(&p_full[pb]);
         }
-        // epilogue: O_u / l as bf16, staged over Q_u's q^C chunks (free once
-        // the last P V completed, which follows the last S MMA) as [128
-        // rows][128 B] with 128-byte swizzle, stored with TMA
+        // epilogue: O / l as bf16, staged over K slot 0 (free once the last
+        // P V completed, which follows every S MMA) as two [128 rows][128 B]
+        // chunks with 128-byte swizzle, stored with TMA
         if (ok && nk > 0) {
-            ok = sm100::warp_wait(&pv_done[u], (nk - 1) & 1, abort_flag, a.err, lim);
+            ok = sm100::warp_wait(&pv_done[(nk - 1) & 1], ((nk - 1) >> 1) & 1, abort_flag, a.err, lim);
             sm100::tc_fence_after();
         }
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        uint8_t *stage = smem + kPfOffQ + 3 * u * kPfChunk;
-        const bool has_rows = q0 + 128 * u < a.s;      // else nothing to store (and Q_u may still be landing)
+        uint8_t *stage = smem + kPfOffK;
 #pragma unroll 1
-        for (int c = 0; c < (has_rows ? 128 : 0); c += 32) {
+        for (int c = 0; c < 128; c += 32) {
             uint32_t ov[32];
             if (ok && nk > 0) {
                 sm100::tmem_ld32(tm_o + c, ov);
@@ -334,17 +356,14 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
                                pack_bf162(__uint_as_float(ov[8 * q + 6]) * inv, __uint_as_float(ov[8 * q + 7]) * inv));
             }
         }
-        if (a.out_lse && t < a.s)
+        if (a.out_lse && has_row)
             a.out_lse[((long long)b * a.s + t) * a.H + head] =
                 l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
         fence_proxy_async_smem();
-        if (u == 0)
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-        else
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (qd == 0 && lane == 0 && has_rows) {
-            sm100::tma_store_4d(&maps.out, stage, 0, head, q0 + 128 * u, b);
-            sm100::tma_store_4d(&maps.out, stage + kPfChunk, 64, head, q0 + 128 * u, b);
+        asm volatile("bar.sync 1, 128;" ::: "memory");     // the 4 softmax warps
+        if (warp == 2 && lane == 0) {
+            sm100::tma_store_4d(&maps.out, stage, 0, head, q0, b);
+            sm100::tma_store_4d(&maps.out, stage + kPfChunk, 64, head, q0, b);
             sm100::tma_store_commit();
             sm100::tma_store_wait_read();
         }
@@ -394,18 +413,24 @@ prefill_prepare_kernel(const bf16 *__restrict__ cache, int num_blocks, const int
         }
         reinterpret_cast<uint4 *>(rows + row * kRow)[c] = v;
     }
-    const long long pairs = (long long)B * s * H * (kDr / 2);  // (token, head) rows x RoPE pairs
-    for (long long w = tid; w < pairs; w += nthreads) {
-        const long long qrow = w / (kDr / 2);
+    // RoPE pair k of every head of token tok: one angle per (token, pair),
+    // the rotation applied to the H heads (a warp covers one token's 32 pairs)
+    const long long units = (long long)B * s * (kDr / 2);
+    for (long long w = tid; w < units; w += nthreads) {
+        const long long tok = w / (kDr / 2);
         const int k = (int)(w % (kDr / 2));
-        const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(q_rope + qrow * kDr)[k];
-        __nv_bfloat162 y = x;
-        if (q_pos) {
-            float y0, y1;
-            rope_turn(__low2float(x), __high2float(x), q_pos[qrow / H], rope.theta[k], &y0, &y1);
-            y = __floats2bfloat162_rn(y0, y1);
+        double sn = 0.0, cs = 1.0;
+        if (q_pos) sincos((double)q_pos[tok] * rope.theta[k], &sn, &cs);
+        for (int h = 0; h < H; ++h) {
+            const long long qrow = tok * H + h;
+            const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(q_rope + qrow * kDr)[k];
+            __nv_bfloat162 y = x;
+            if (q_pos) {
+                const double x0 = __low2float(x), x1 = __high2float(x);
+                y = __floats2bfloat162_rn((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
+            }
+            reinterpret_cast<__nv_bfloat162 *>(q_rot + qrow * kDr)[k] = y;
         }
-        reinterpret_cast<__nv_bfloat162 *>(q_rot + qrow * kDr)[k] = y;
     }
 }
 

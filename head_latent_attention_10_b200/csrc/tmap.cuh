@@ -33,7 +33,7 @@ inline EncodeTiledFn encode_fn()
 
 struct TmapKey {
     const void *ptr;
-    uint32_t rank;
+    uint32_t rank, dtype;
     uint64_t dims[4], strides[3];
     uint32_t box[4];
     int swizzle;
@@ -46,11 +46,12 @@ inline CUtensorMapSwizzle swizzle_for(uint32_t inner_bytes)
                               : (inner_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-// bf16 tensor of rank 3 or 4: dims innermost first (elements), strides of
-// dims 1.. in bytes, box in elements.  Out-of-range elements read as zero and
-// are not written by stores.
+// Tensor of rank 1-4 (bf16 unless `dtype` says otherwise): dims innermost
+// first (elements), strides of dims 1.. in bytes, box in elements.
+// Out-of-range elements read as zero and are not written by stores.
 inline bool make_tmap_nd(CUtensorMap *out, const void *ptr, uint32_t rank, const uint64_t *dims,
-                         const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw)
+                         const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw,
+                         CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
 {
     static std::mutex mu;
     static TmapKey keys[64];
@@ -61,6 +62,7 @@ inline bool make_tmap_nd(CUtensorMap *out, const void *ptr, uint32_t rank, const
     memset(&k, 0, sizeof k);
     k.ptr = ptr;
     k.rank = rank;
+    k.dtype = (uint32_t)dtype;
     for (uint32_t i = 0; i < rank; ++i) {
         k.dims[i] = dims[i];
         k.box[i] = box[i];
@@ -85,7 +87,7 @@ inline bool make_tmap_nd(CUtensorMap *out, const void *ptr, uint32_t rank, const
         if (i + 1 < rank) gstr[i] = k.strides[i];
     }
     CUtensorMap m;
-    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), gdim, gstr, cbox, estr,
+    if (fn(&m, dtype, rank, const_cast<void *>(ptr), gdim, gstr, cbox, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
@@ -104,6 +106,15 @@ inline bool make_tmap_3d(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_
     const uint64_t dims[3] = {d0, d1, d2}, strides[2] = {s1, s2};
     const uint32_t box[3] = {b0, b1, b2};
     return make_tmap_nd(out, ptr, 3, dims, strides, box, sw);
+}
+
+// uint8 tensor of rank 3 (the FP8 cache), as make_tmap_3d.
+inline bool make_tmap_3d_u8(CUtensorMap *out, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                            uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw)
+{
+    const uint64_t dims[3] = {d0, d1, d2}, strides[2] = {s1, s2};
+    const uint32_t box[3] = {b0, b1, b2};
+    return make_tmap_nd(out, ptr, 3, dims, strides, box, sw, CU_TENSOR_MAP_DATA_TYPE_UINT8);
 }
 
 inline bool make_tmap_4d(CUtensorMap *out, const void *ptr, const uint64_t (&dims)[4], const uint64_t (&strides)[3],

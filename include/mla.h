@@ -313,6 +313,49 @@ mla_status_t mla_prefill(const mla_dims_t *dims, const void *q_nope, const void 
                          void *stream);
 
 /*
+ * FP8 latent cache [DeepSeek-V2 paper review, sections 4 and 9: the deployed
+ * model keeps its KV cache at about 6 bits per element; DeepSeek-V3 report
+ * summary, the FP8 framework: E4M3 values with fine-grained scaling factors].
+ * A token's row [c^KV (512) | k^R (64), rotated] is stored as 576 E4M3 codes
+ * (OCP: bias 7, no infinities, 448 the largest finite value) plus one fp32
+ * scale per part, scale = amax / 448 over the part (1 for an all-zero part),
+ * code = E4M3(x / scale), the quotient in fp32, nearest-even, saturated.  A
+ * code's value is E4M3(code) * scale.
+ *   codes  [num_blocks][block_size][d_c + d_rope] uint8   (16-byte aligned)
+ *   scales [num_blocks][block_size][2] fp32 (c^KV part, k^R part)
+ *
+ * mla_append_latent_fp8 -- mla_append_latent into the FP8 cache: forms the
+ * same bf16 row (copy or RMSNorm of c_kv, RoPE of k_rope at pos), quantizes it
+ * as above and writes codes and scales to the slot of (seq_idx[t], pos[t]).
+ * Arguments as for mla_append_latent, with `codes` and `scales` in place of
+ * `cache` (num_blocks pages of each); scales must be 8-byte aligned.
+ */
+mla_status_t mla_append_latent_fp8(const mla_dims_t *dims, const void *c_kv, const void *k_rope,
+                                   int T, const int32_t *seq_idx, const int32_t *pos,
+                                   const int32_t *block_table, int num_seqs, int max_blocks,
+                                   void *codes, float *scales, int num_blocks,
+                                   const void *kv_norm_weight, float kv_norm_eps,
+                                   uint32_t *err_word, void *stream);
+
+/*
+ * mla_decode_fp8 -- mla_decode over the FP8 cache: the same attention with
+ * each cache row taken as its codes' values times its scales.  The kernel
+ * widens each page to f16 in shared memory (exactly: every E4M3 value is an
+ * f16 value, one part of the row multiplied by the ratio of its scale to the
+ * larger of the two) and runs the logits and the latent sum on f16 tensor
+ * cores with fp32 accumulation; q_abs is read as bf16 and rounded to f16.
+ * Arguments, workspace (mla_decode_workspace_size), outputs and errors as for
+ * mla_decode, with `codes` and `scales` (16-byte aligned) in place of
+ * `cache`.  flags: MLA_SYNC_CHECK, MLA_DEBUG_STALL; MLA_FORCE_SIMPLE returns
+ * MLA_ERR_UNSUPPORTED.
+ */
+mla_status_t mla_decode_fp8(const mla_dims_t *dims, const void *q_abs, const void *codes,
+                            const float *scales, int num_blocks, const int32_t *block_table,
+                            int max_blocks, const int32_t *seq_lens, int B, int s,
+                            void *out_latent, float *out_lse, void *workspace, size_t ws_bytes,
+                            uint32_t flags, void *stream);
+
+/*
  * mla_decode_ctas -- number of CTAs (the persistent grid) the tensor-core
  * decode launches on the current device for these dims and s query tokens
  * per sequence, or 0 if it cannot run.  A measurement aid.

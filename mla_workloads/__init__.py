@@ -33,10 +33,11 @@ from typing import Dict, Optional, Sequence, Tuple, Union
 import numpy as np
 
 BF16_NAN = np.uint16(0x7FC0)
+E4M3_NAN = np.uint8(0x7F)
 D_C, D_R, D_H, BLOCK = 512, 64, 128, 64
 
 _STREAMS = ("w_uk", "w_uv", "c_kv", "k_rope", "q_nope", "q_rope", "block_perm", "seq_lens",
-            "h", "w_dkv", "w_kr", "w_o", "q_abs_nope", "q_abs_rope", "latent")
+            "h", "w_dkv", "w_kr", "w_o", "q_abs_nope", "q_abs_rope", "latent", "fp8_codes", "fp8_scales")
 
 
 @dataclass(frozen=True)
@@ -230,3 +231,28 @@ def sample_pairs(cfg: MLAConfig, seq_lens: np.ndarray, n_rows: int, n_heads: int
                 rows.append(b * cfg.s + t)
                 heads.append(int(h))
     return np.asarray(rows, np.int32), np.asarray(heads, np.int32)
+
+
+def make_fp8_cache(cfg: MLAConfig, table: np.ndarray, num_blocks: int, tok_seq, tok_pos):
+    """A random FP8 latent cache for testing the FP8 decode on its own, drawn
+    as bit patterns (no quantization here): every token's 576 E4M3 codes have
+    a random sign, an exponent field uniform in 5..9 (values 2^-2 .. 2^2 times
+    1 + m/8) and a uniform 3-bit mantissa; its two fp32 scales (c^KV part,
+    k^R part) are uniform in [0.1, 0.3].  Slots no token maps to hold the NaN
+    code 0x7F and NaN scales.  Returns (codes [num_blocks][64][576] uint8,
+    scales [num_blocks][64][2] float32)."""
+    st = _streams(cfg.seed)
+    D = cfg.d_c + cfg.d_r
+    N = tok_seq.size
+    g = st["fp8_codes"]
+    sign = g.integers(0, 2, size=(N, D), dtype=np.uint8) << np.uint8(7)
+    expo = g.integers(5, 10, size=(N, D), dtype=np.uint8) << np.uint8(3)
+    mant = g.integers(0, 8, size=(N, D), dtype=np.uint8)
+    rows = (sign | expo | mant).astype(np.uint8)
+    sc = st["fp8_scales"].uniform(0.1, 0.3, size=(N, 2)).astype(np.float32)
+    codes = np.full((num_blocks, cfg.block_size, D), E4M3_NAN, dtype=np.uint8)
+    scales = np.full((num_blocks, cfg.block_size, 2), np.nan, dtype=np.float32)
+    blk = table[tok_seq, tok_pos // cfg.block_size]
+    codes[blk, tok_pos % cfg.block_size] = rows
+    scales[blk, tok_pos % cfg.block_size] = sc
+    return codes, scales

@@ -239,3 +239,29 @@ def test_prefill_argument_errors_and_workspace(M):
     # K^C and V^C dominate: 2 x rows x H x 128 bf16
     assert a >= 2 * 1024 * 128 * 128 * 2
     assert lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 129, 128) == 0
+
+
+def test_fp8_argument_errors(M):
+    """The FP8 writer and decode reject bad arguments before any device work."""
+    lib = _raw(M)
+    d = M.dims(128)
+    p = ctypes.c_void_p(256)
+    n0 = lib.mla_kernel_launches()
+    # writer: negative T, misaligned codes or scales, bad norm arguments; T = 0 is a no-op
+    assert lib.mla_append_latent_fp8(ctypes.byref(d), p, p, -1, p, p, p, 1, 1, p, p, 1, None, 0.0, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_latent_fp8(ctypes.byref(d), p, p, 1, p, p, p, 1, 1, ctypes.c_void_p(264), p, 1, None, 0.0, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_latent_fp8(ctypes.byref(d), p, p, 1, p, p, p, 1, 1, p, ctypes.c_void_p(260), 1, None, 0.0, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_latent_fp8(ctypes.byref(d), p, p, 1, p, p, p, 1, 1, p, p, 1, p, -1.0, None, None) == M.MLA_ERR_INVALID_ARG
+    assert lib.mla_append_latent_fp8(ctypes.byref(d), p, p, 0, p, p, p, 1, 1, p, p, 1, None, 0.0, None, None) == M.MLA_OK
+    # decode: the CUDA-core path does not read FP8; bad sizes; misaligned scales; workspace
+    big = 1 << 40
+    dec = lambda flags=0, B=1, s=1, nb=1, mb=1, sc=p, ws=p, wsb=big: lib.mla_decode_fp8(
+        ctypes.byref(d), p, p, sc, nb, p, mb, p, B, s, p, None, ws, wsb, flags, None)
+    assert dec(flags=M.MLA_FORCE_SIMPLE) == M.MLA_ERR_UNSUPPORTED
+    assert dec(s=0) == M.MLA_ERR_INVALID_ARG
+    assert dec(nb=0) == M.MLA_ERR_INVALID_ARG
+    assert dec(sc=ctypes.c_void_p(264)) == M.MLA_ERR_INVALID_ARG
+    assert dec(ws=None) == M.MLA_ERR_WORKSPACE
+    assert dec(wsb=16) == M.MLA_ERR_WORKSPACE
+    assert dec(B=0) == M.MLA_OK
+    assert lib.mla_kernel_launches() == n0
