@@ -23,7 +23,8 @@ MLA_SYNC_CHECK, MLA_FORCE_SIMPLE, MLA_DEBUG_STALL = 0x1, 0x2, 0x100
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",
             "mla_kernel_launches", "mla_decode_ctas", "mla_decode_noalloc",
-            "mla_prefill_workspace_size", "mla_prefill", "mla_append_latent_fp8", "mla_decode_fp8")
+            "mla_prefill_workspace_size", "mla_prefill", "mla_append_latent_fp8", "mla_decode_fp8",
+            "mla_fold_weights", "mla_absorb_q_folded", "mla_up_out_folded")
 
 
 class MLAError(RuntimeError):
@@ -84,6 +85,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mla_append_latent_fp8.argtypes = [D, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _vp, _vp, _i, _vp, _f, _vp, _vp]
     lib.mla_decode_fp8.argtypes = [D, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _vp, _vp, _vp, ctypes.c_size_t,
                                    ctypes.c_uint32, _vp]
+    lib.mla_fold_weights.argtypes = [D, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp]
+    lib.mla_absorb_q_folded.argtypes = [D, _vp, _i, _vp, _vp, _vp, _i, _vp, _vp]
+    lib.mla_up_out_folded.argtypes = [D, _vp, _i, _vp, _i, _vp, _vp]
     lib.mla_kernel_launches.argtypes = []
     lib.mla_kernel_launches.restype = ctypes.c_uint64
     for name in EXPORTED:
@@ -228,6 +232,30 @@ def mla_decode_fp8(d, q_abs, codes, scales, block_table, seq_lens, s, out_latent
         ctypes.byref(d), _ptr(q_abs), _ptr(codes), _ptr(scales), codes.shape[0], _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), B, s, _ptr(out_latent), _ptr(out_lse), _ptr(workspace),
         workspace.numel() * workspace.element_size(), flags, _stream(stream)), "mla_decode_fp8")
+
+
+def mla_fold_weights(d, w_uq=None, w_uk=None, w_qk=None, w_o=None, w_uv=None, w_ov=None, stream=None):
+    """W^QK_i = (U^K_i)^T W^UQ_i into w_qk [H][512][d_q]; W^OV block i = O_i U^V_i
+    into w_ov [d_model][H*512].  Either group may be left out."""
+    d_q = 0 if w_uq is None else w_uq.shape[-1]
+    d_model = 0 if w_o is None else w_o.shape[0]
+    _check(load_library().mla_fold_weights(
+        ctypes.byref(d), d_q, _ptr(w_uq), _ptr(w_uk), _ptr(w_qk), d_model, _ptr(w_o), _ptr(w_uv), _ptr(w_ov),
+        _stream(stream)), "mla_fold_weights")
+
+
+def mla_absorb_q_folded(d, c_q, q_rope, q_pos, w_qk, q_abs, stream=None):
+    """q_abs = [W^QK_i c_q | RoPE(q^R_i, q_pos)]."""
+    _check(load_library().mla_absorb_q_folded(
+        ctypes.byref(d), _ptr(c_q), c_q.shape[1], _ptr(q_rope), _ptr(q_pos), _ptr(w_qk), c_q.shape[0],
+        _ptr(q_abs), _stream(stream)), "mla_absorb_q_folded")
+
+
+def mla_up_out_folded(d, latent, w_ov, out_model, stream=None):
+    """out_model = sum_i W^OV_i latent_i."""
+    _check(load_library().mla_up_out_folded(
+        ctypes.byref(d), _ptr(latent), latent.shape[0], _ptr(w_ov), w_ov.shape[0], _ptr(out_model),
+        _stream(stream)), "mla_up_out_folded")
 
 
 def mla_up_v(d, latent, w_uv, out_heads, w_o=None, out_model=None, stream=None):

@@ -49,6 +49,29 @@ __device__ __forceinline__ void rope_turn(float x0, float x1, int pos, double th
     *y1 = (float)((double)x0 * sn + (double)x1 * cs);
 }
 
+// RoPE pair k of every head of token tok: one angle per (token, pair), taken
+// and turned in double precision (the rotate of rope_turn), applied to the H
+// heads' rows q_rope[tok][h] (64 bf16 each) and written to dst at row
+// (tok * H + h) * dst_stride + dst_off; copied unturned when q_pos is null.
+// A warp of consecutive k covers one token's 32 pairs: coalesced per head.
+__device__ __forceinline__ void rope_heads(const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos,
+                                           long long tok, int k, int H, const RopeTable &rope, bf16 *__restrict__ dst,
+                                           int dst_stride, int dst_off)
+{
+    double sn = 0.0, cs = 1.0;
+    if (q_pos) sincos((double)q_pos[tok] * rope.theta[k], &sn, &cs);
+    for (int h = 0; h < H; ++h) {
+        const long long row = tok * H + h;
+        const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(q_rope + row * kDr)[k];
+        __nv_bfloat162 y = x;
+        if (q_pos) {
+            const double x0 = __low2float(x), x1 = __high2float(x);
+            y = __floats2bfloat162_rn((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
+        }
+        reinterpret_cast<__nv_bfloat162 *>(dst + row * dst_stride + dst_off)[k] = y;
+    }
+}
+
 // Root mean square normalisation factor of a latent row, from the sum of its
 // squares: 1 / sqrt(ss / d_c + eps).
 __device__ __forceinline__ float rms_inv(float ss, float eps)

@@ -104,6 +104,17 @@ append_latent_kernel(const bf16 *__restrict__ c_kv, const bf16 *__restrict__ k_r
     reinterpret_cast<__nv_bfloat162 *>(dst + kDc)[lane] = kr;
 }
 
+// RoPE of the query's RoPE part for every head, into rows of stride
+// dst_stride at offset dst_off (the folded absorption writes q_abs[.][512:576]).
+__global__ void __launch_bounds__(256)
+rope_q_kernel(const bf16 *__restrict__ q_rope, const int32_t *__restrict__ q_pos, int T, int H, bf16 *__restrict__ dst,
+              int dst_stride, int dst_off, const RopeTable rope)
+{
+    const long long units = (long long)T * (kDr / 2);
+    for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < units; w += (long long)gridDim.x * blockDim.x)
+        rope_heads(q_rope, q_pos, w / (kDr / 2), (int)(w % (kDr / 2)), H, rope, dst, dst_stride, dst_off);
+}
+
 // RMS normalisation, in place, of the latent part of the cache rows of T
 // tokens (the projection path writes the rows first): one warp per token.
 __global__ void __launch_bounds__(256)

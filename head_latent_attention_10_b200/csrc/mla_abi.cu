@@ -147,12 +147,12 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
 
 // C = A B on tcgen05; `c` is the output tensor map of the staged (TMA store)
 // epilogue, unused by the others.
-template <int BN, bool kBmn, class Epi>
+template <int BN, bool kBmn, class Epi, bool kAmn = false>
 cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
                            uint32_t *err, cudaStream_t st, const CUtensorMap *c = nullptr)
 {
     using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kAmn>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
     if (e != cudaSuccess) return e;
@@ -766,6 +766,101 @@ mla_status_t mla_decode_fp8(const mla_dims_t *dims, const void *q_abs, const voi
             return MLA_ERR_CUDA;
         if (host) return MLA_ERR_DEVICE;
     }
+    return MLA_OK;
+}
+
+mla_status_t mla_fold_weights(const mla_dims_t *dims, int d_q, const void *w_uq, const void *w_uk, void *w_qk,
+                              int d_model, const void *w_o, const void *w_uv, void *w_ov, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    const bool qk = w_uq || w_uk || w_qk, ov = w_o || w_uv || w_ov;
+    if (qk && (!w_uq || !w_uk || !w_qk || d_q <= 0 || d_q % 64 != 0)) return MLA_ERR_INVALID_ARG;
+    if (ov && (!w_o || !w_uv || !w_ov || d_model <= 0 || d_model % 64 != 0)) return MLA_ERR_INVALID_ARG;
+    if ((w_uq && !aligned16(w_uq)) || (w_uk && !aligned16(w_uk)) || (w_qk && !aligned16(w_qk)) ||
+        (w_o && !aligned16(w_o)) || (w_uv && !aligned16(w_uv)) || (w_ov && !aligned16(w_ov)))
+        return MLA_ERR_INVALID_ARG;
+    const int H = dims->num_heads;
+    cudaStream_t s = as_stream(stream);
+    if (qk) {
+        // W^QK_i [512][d_q] = (U^K_i)^T [512][128] . W^UQ_i [128][d_q]: A = U^K_i
+        // read MN-major (stored [128][512]), B = W^UQ_i MN-major (stored [128][d_q])
+        CUtensorMap ma, mb, mc;
+        if (!tmap(&ma, w_uk, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64) ||
+            !tmap(&mb, w_uq, d_q, kDh, H, d_q, (uint64_t)kDh * d_q, 64, 64) ||
+            !make_tmap_3d(&mc, w_qk, d_q, H, kDc, (uint64_t)kDc * d_q * 2, (uint64_t)d_q * 2, 64, 1, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+            return MLA_ERR_CUDA;
+        if (launch_tc_gemm<256, true, TcEpiTmaStore, true>(ma, mb, kDc, d_q, kDh, H, TcEpiTmaStore{}, nullptr, s,
+                                                           &mc) != cudaSuccess)
+            return MLA_ERR_CUDA;
+    }
+    if (ov) {
+        // W^OV [d_model][H*512], block i = O_i [d_model][128] . U^V_i [128][512]:
+        // A = the 128 columns of head i in W^O (K-major), B = U^V_i MN-major
+        CUtensorMap ma, mb, mc;
+        if (!tmap(&ma, w_o, kDh, d_model, H, (uint64_t)H * kDh, kDh, 64, 128) ||
+            !tmap(&mb, w_uv, kDc, kDh, H, kDc, (uint64_t)kDh * kDc, 64, 64) ||
+            !make_tmap_3d(&mc, w_ov, kDc, H, d_model, (uint64_t)kDc * 2, (uint64_t)H * kDc * 2, 64, 1, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+            return MLA_ERR_CUDA;
+        if (launch_tc_gemm<256, true, TcEpiTmaStore>(ma, mb, d_model, kDc, kDh, H, TcEpiTmaStore{}, nullptr, s, &mc) !=
+            cudaSuccess)
+            return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+mla_status_t mla_absorb_q_folded(const mla_dims_t *dims, const void *c_q, int d_q, const void *q_rope,
+                                 const int32_t *q_pos, const void *w_qk, int T, void *q_abs, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (T < 0 || d_q <= 0 || d_q % 64 != 0) return MLA_ERR_INVALID_ARG;
+    if (T == 0) return MLA_OK;
+    if (!c_q || !q_rope || !w_qk || !q_abs) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(c_q) || !aligned16(w_qk) || !aligned16(q_abs) || ((uintptr_t)q_rope & 3u))
+        return MLA_ERR_INVALID_ARG;
+    const int H = dims->num_heads;
+    cudaStream_t s = as_stream(stream);
+    // q_abs[t][i][0:512] = W^QK_i c_q[t]: one GEMM over all heads, C [T][H*512]
+    // = c_q [T][d_q] . W^QK^T (W^QK stored [H*512][d_q], K-major), each
+    // 512-column head block stored into its q_abs row
+    CUtensorMap ma, mb, mc;
+    if (!tmap(&ma, c_q, d_q, T, 1, d_q, 0, 64, 128) ||
+        !tmap(&mb, w_qk, d_q, (uint64_t)H * kDc, 1, d_q, 0, 64, 256) ||
+        !make_tmap_3d(&mc, q_abs, kDc, H, T, (uint64_t)kRow * 2, (uint64_t)H * kRow * 2, 64, 1, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return MLA_ERR_CUDA;
+    TcEpiTmaStore e;
+    e.split_n = kDc;
+    if (launch_tc_gemm<256, false, TcEpiTmaStore>(ma, mb, T, H * kDc, d_q, 1, e, nullptr, s, &mc) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    long long blocks = ((long long)T * (kDr / 2) + 255) / 256;
+    if (blocks > 8ll * sm_count()) blocks = 8ll * sm_count();
+    rope_q_kernel<<<(int)blocks, 256, 0, s>>>((const bf16 *)q_rope, q_pos, T, H, (bf16 *)q_abs, kRow, kDc,
+                                              rope_table(dims));
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+mla_status_t mla_up_out_folded(const mla_dims_t *dims, const void *latent, int T, const void *w_ov, int d_model,
+                               void *out_model, void *stream)
+{
+    mla_status_t st = check_dims(dims);
+    if (st != MLA_OK) return st;
+    if (T < 0 || d_model <= 0 || d_model % 64 != 0) return MLA_ERR_INVALID_ARG;
+    if (T == 0) return MLA_OK;
+    if (!latent || !w_ov || !out_model) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(latent) || !aligned16(w_ov) || !aligned16(out_model)) return MLA_ERR_INVALID_ARG;
+    const int K = dims->num_heads * kDc;
+    cudaStream_t s = as_stream(stream);
+    // out_model [T][d_model] = latent [T][H*512] . W^OV^T (W^OV [d_model][H*512], K-major)
+    CUtensorMap ma, mb;
+    if (!tmap(&ma, latent, K, T, 1, K, 0, 64, 128) || !tmap(&mb, w_ov, K, d_model, 1, K, 0, 64, 256))
+        return MLA_ERR_CUDA;
+    TcEpiStore e{(bf16 *)out_model, 0, d_model};
+    if (launch_tc_gemm<256, false>(ma, mb, T, d_model, K, 1, e, nullptr, s) != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
 }
 

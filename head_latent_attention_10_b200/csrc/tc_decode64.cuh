@@ -93,7 +93,7 @@ constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ah
 // FP8 cache: 64 more threads (the converters), per-stage scale slots
 // ([64][2] fp32) and per-token factored scales s_j ([64] fp32) after the stages
 constexpr int kD64ThreadsFp8 = kD64Threads + 64;
-constexpr int kD64F8Codes = kT64 * kRow / 2;      // 36,864: where the codes land in the stage
+constexpr int kD64F8Codes = kT64 * kRow;          // 36,864 (one code per value): where the codes land
 constexpr int kD64F8Box = kT64 * 64;              // one 64-column box of codes (4 KB)
 constexpr int kD64OffScale = kD64Stages * kD64Stage;              // [3][64][2] fp32
 constexpr int kD64OffSmax = kD64OffScale + kD64Stages * 512;      // [3][64] fp32

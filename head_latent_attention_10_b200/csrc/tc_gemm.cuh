@@ -9,9 +9,11 @@
 // with tcgen05.ld (one TMEM lane = one output row per thread) and hand 16
 // columns at a time to the epilogue functor.
 //
-// A is K-major (rows of K contiguous).  B is either K-major (B^T stored
-// row-major, e.g. a weight [N][K]) or MN-major (B stored [K][N]).
-// Tensor maps are 3-D: A {K, M, Z}, B K-major {K, N, Z}, B MN-major {N, K, Z}.
+// A is K-major (rows of K contiguous) or, with kAmn, MN-major (A stored
+// [K][M]); B is either K-major (B^T stored row-major, e.g. a weight [N][K])
+// or MN-major (B stored [K][N]).
+// Tensor maps are 3-D: A K-major {K, M, Z}, A MN-major {M, K, Z}, B K-major
+// {K, N, Z}, B MN-major {N, K, Z}.
 #pragma once
 
 #include "sm100.cuh"
@@ -31,7 +33,7 @@ struct GemmSmem {
     static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
 };
 
-template <int BN, bool kBmn, class Epi>
+template <int BN, bool kBmn, class Epi, bool kAmn = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                const __grid_constant__ CUtensorMap mapC, int M, int N, int K, Epi epi, uint32_t *err,
@@ -83,7 +85,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 uint8_t *b = a + S::A;
                 sm100::mbar_arrive_expect_tx(&full[s], S::STAGE);
                 const int kx = kb * 64;
-                sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, z);
+                if (kAmn) {
+                    sm100::tma_load_3d(&mapA, &full[s], a, m0, kx, z);
+                    sm100::tma_load_3d(&mapA, &full[s], a + 8192, m0 + 64, kx, z);
+                } else {
+                    sm100::tma_load_3d(&mapA, &full[s], a, kx, m0, z);
+                }
                 if (kBmn) {
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
@@ -102,7 +109,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
         }
     } else if (warp == 1) {
         if (sm100::elect_one()) {
-            const uint32_t idesc = sm100::idesc_bf16(128, BN, 0, kBmn ? 1 : 0);
+            const uint32_t idesc = sm100::idesc_bf16(128, BN, kAmn ? 1 : 0, kBmn ? 1 : 0);
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % kGemmStages;
@@ -111,11 +118,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
                 sm100::tc_fence_after();
                 const uint32_t a = sm100::smem_u32(smem + s * S::STAGE);
                 const uint32_t b = a + S::A;
-                const uint64_t ad = sm100::desc_kmajor(a, 128, sm100::kSw128);
+                const uint64_t ad = kAmn ? sm100::desc_mnmajor_sw128(a, 8192) : sm100::desc_kmajor(a, 128, sm100::kSw128);
                 const uint64_t bd = kBmn ? sm100::desc_mnmajor_sw128(b, 8192) : sm100::desc_kmajor(b, 128, sm100::kSw128);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    sm100::umma_ss(tmem, ad + (uint64_t)((kk * 32) >> 4),
+                    sm100::umma_ss(tmem, ad + (uint64_t)(((kAmn ? kk * 16 * 128 : kk * 32)) >> 4),
                                    bd + (uint64_t)(((kBmn ? kk * 16 * 128 : kk * 32)) >> 4), idesc, (kb | kk) != 0);
                 sm100::umma_commit(&empty[s]);
             }
@@ -157,7 +164,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("bar.sync 1, 128;" ::: "memory");   // the 4 epilogue warps
             if (warp == 2 && lane == 0) {
-                for (int c = 0; c < BN; c += 64) sm100::tma_store_3d(&mapC, smem + (c / 64) * 16384, n0 + c, z, m0);
+                for (int c = 0; c < BN; c += 64) {
+                    // with split_n the flat column n is (n % split_n) of batch entry n / split_n
+                    const int n = n0 + c;
+                    if (epi.split_n > 0)
+                        sm100::tma_store_3d(&mapC, smem + (c / 64) * 16384, n % epi.split_n, n / epi.split_n, m0);
+                    else
+                        sm100::tma_store_3d(&mapC, smem + (c / 64) * 16384, n, z, m0);
+                }
                 sm100::tma_store_commit();
                 sm100::tma_store_wait_read();
             }
@@ -186,9 +200,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 // ------------------------------------------------------------- epilogues
 // bf16 output stored with TMA from a staged tile through the kernel's output
 // tensor map, which covers the output as {N, Z, M} (columns, batch entry,
-// rows) with box {64, 1, 128}.
+// rows) with box {64, 1, 128}.  With split_n > 0 (Z = 1) the flat column n
+// goes to column n % split_n of entry n / split_n: one GEMM over all heads
+// writing a per-head output whose rows are interleaved with other data.
 struct TcEpiTmaStore {
     static constexpr bool kStaged = true;
+    int split_n = 0;
     __device__ void operator()(int, int, int, const float *) const {}
 };
 

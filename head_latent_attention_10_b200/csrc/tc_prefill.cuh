@@ -413,25 +413,9 @@ prefill_prepare_kernel(const bf16 *__restrict__ cache, int num_blocks, const int
         }
         reinterpret_cast<uint4 *>(rows + row * kRow)[c] = v;
     }
-    // RoPE pair k of every head of token tok: one angle per (token, pair),
-    // the rotation applied to the H heads (a warp covers one token's 32 pairs)
     const long long units = (long long)B * s * (kDr / 2);
-    for (long long w = tid; w < units; w += nthreads) {
-        const long long tok = w / (kDr / 2);
-        const int k = (int)(w % (kDr / 2));
-        double sn = 0.0, cs = 1.0;
-        if (q_pos) sincos((double)q_pos[tok] * rope.theta[k], &sn, &cs);
-        for (int h = 0; h < H; ++h) {
-            const long long qrow = tok * H + h;
-            const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162 *>(q_rope + qrow * kDr)[k];
-            __nv_bfloat162 y = x;
-            if (q_pos) {
-                const double x0 = __low2float(x), x1 = __high2float(x);
-                y = __floats2bfloat162_rn((float)(x0 * cs - x1 * sn), (float)(x0 * sn + x1 * cs));
-            }
-            reinterpret_cast<__nv_bfloat162 *>(q_rot + qrow * kDr)[k] = y;
-        }
-    }
+    for (long long w = tid; w < units; w += nthreads)
+        rope_heads(q_rope, q_pos, w / (kDr / 2), (int)(w % (kDr / 2)), H, rope, q_rot, kDr, 0);
 }
 
 }  // namespace mla

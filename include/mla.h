@@ -23,8 +23,7 @@
  *   - Every pointer is caller-owned DEVICE memory unless stated otherwise.
  *     No call allocates device memory (no cudaMalloc, no allocating library
  *     routine).  mla_decode and mla_prefill keep their scratch in the
- *     caller's workspace; mla_append_cache, mla_append_latent, mla_absorb_q
- *     and mla_up_v need none.  One call, mla_decode_noalloc, uses a fixed file-scope device
+ *     caller's workspace; the other calls need none.  One call, mla_decode_noalloc, uses a fixed file-scope device
  *     array inside the library instead (MLA_NOALLOC_SCRATCH_BYTES, one per
  *     device, held until the process exits); calls of it that may overlap on
  *     one device race on that array (see its notes).
@@ -354,6 +353,45 @@ mla_status_t mla_decode_fp8(const mla_dims_t *dims, const void *q_abs, const voi
                             int max_blocks, const int32_t *seq_lens, int B, int s,
                             void *out_latent, float *out_lse, void *workspace, size_t ws_bytes,
                             uint32_t flags, void *stream);
+
+/*
+ * Weight pre-absorption [DeepSeek-V2 paper review, section 2: at inference
+ * W^UK can be absorbed into the query up-projection W^UQ and W^UV into the
+ * output projection W^O; the query path compresses to c^Q = W^DQ h of width
+ * d_q (1536 in V2) and q^C_i = W^UQ_i c^Q].
+ *
+ * mla_fold_weights -- one-time weight transform on the GPU (tensor cores,
+ * fp32 accumulation, bf16 results):
+ *   w_qk [H][d_c][d_q]       W^QK_i = (U^K_i)^T W^UQ_i
+ *   w_ov [d_model][H*d_c]    block i (columns i*d_c ..) = O_i U^V_i
+ * from w_uq [H][d_head][d_q], w_uk and w_uv [H][d_head][d_c] (as for
+ * mla_absorb_q / mla_up_v) and w_o [d_model][H*d_head].  Either group
+ * (w_uq, w_uk, w_qk) or (w_o, w_uv, w_ov) may be all NULL to skip it.
+ * d_q and d_model must be positive multiples of 64.
+ *
+ * mla_absorb_q_folded -- step a2 from the compressed query:
+ *   q_abs[t][i] = [ W^QK_i c_q[t] , RoPE(q_rope[t][i], q_pos[t]) ]
+ * c_q [T][d_q] bf16, q_rope / q_pos / q_abs as for mla_absorb_q.  Equal to
+ * mla_absorb_q on q^C_i = W^UQ_i c^Q up to rounding.
+ *
+ * mla_up_out_folded -- step a7 with the folded output weights:
+ *   out_model[t] = sum_i W^OV_i latent[t][i]
+ * latent [T][H][d_c] bf16 (mla_decode's output), out_model [T][d_model].
+ * Equal to mla_up_v with w_o up to rounding.
+ *
+ * The folded forms trade memory traffic for fewer launches: at decode batch
+ * sizes both steps read their weights once per call, and W^QK (H*d_c*d_q)
+ * and W^OV (d_model*H*d_c) are larger than U^K + W^UQ and U^V + W^O
+ * (for V2: 201 MB against 67 MB, and 671 MB against 185 MB).
+ */
+mla_status_t mla_fold_weights(const mla_dims_t *dims, int d_q, const void *w_uq, const void *w_uk,
+                              void *w_qk, int d_model, const void *w_o, const void *w_uv,
+                              void *w_ov, void *stream);
+mla_status_t mla_absorb_q_folded(const mla_dims_t *dims, const void *c_q, int d_q,
+                                 const void *q_rope, const int32_t *q_pos, const void *w_qk,
+                                 int T, void *q_abs, void *stream);
+mla_status_t mla_up_out_folded(const mla_dims_t *dims, const void *latent, int T,
+                               const void *w_ov, int d_model, void *out_model, void *stream);
 
 /*
  * mla_decode_ctas -- number of CTAs (the persistent grid) the tensor-core

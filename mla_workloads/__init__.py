@@ -37,7 +37,8 @@ E4M3_NAN = np.uint8(0x7F)
 D_C, D_R, D_H, BLOCK = 512, 64, 128, 64
 
 _STREAMS = ("w_uk", "w_uv", "c_kv", "k_rope", "q_nope", "q_rope", "block_perm", "seq_lens",
-            "h", "w_dkv", "w_kr", "w_o", "q_abs_nope", "q_abs_rope", "latent", "fp8_codes", "fp8_scales")
+            "h", "w_dkv", "w_kr", "w_o", "q_abs_nope", "q_abs_rope", "latent", "fp8_codes", "fp8_scales",
+            "w_uq", "c_q")
 
 
 @dataclass(frozen=True)
@@ -206,6 +207,15 @@ def make_append_inputs(cfg: MLAConfig, T: int) -> dict:
     return dict(h=_normal_bf16(st["h"], (T, d), 1.0),
                 w_dkv=_normal_bf16(st["w_dkv"], (cfg.d_c, d), (1.0 / d) ** 0.5),
                 w_kr=_normal_bf16(st["w_kr"], (cfg.d_r, d), (1.0 / d) ** 0.5))
+
+
+def make_query_latent_inputs(cfg: MLAConfig, T: int, d_q: int = 1536) -> dict:
+    """The compressed query path: c^Q [T][d_q] N(0,1) and W^UQ [H][d_h][d_q]
+    N(0, 1/d_q), so that q^C = W^UQ c^Q is about N(0,1) like q^C above
+    (bf16 bits).  d_q = 1536 is DeepSeek-V2's query latent width."""
+    st = _streams(cfg.seed)
+    return dict(c_q=_normal_bf16(st["c_q"], (T, d_q), 1.0),
+                w_uq=_normal_bf16(st["w_uq"], (cfg.H, cfg.d_h, d_q), (1.0 / d_q) ** 0.5))
 
 
 def make_w_o(cfg: MLAConfig) -> np.ndarray:

@@ -45,7 +45,11 @@ tests/test_oracle_pins.py, none is "parity unpinned":
     invariance, the constant-row closed form;
   * yarn_theta, rope_rows_theta: scale 1 gives the plain RoPE frequencies and
     rotations, pairs far below the ramp are divided by s and pairs far above
-    it are unchanged, the ramp is continuous, the rotation preserves norms.
+    it are unchanged, the ramp is continuous, the rotation preserves norms;
+  * fold_qk, fold_ov: identity W^UQ (or W^O) returning (U^K)^T (or the U^V
+    blocks) exactly, and brute-force dot products on tiny integer inputs;
+  * absorb_q_folded, up_out_folded: equal to the pinned two-step path
+    (absorb_q of W^UQ c^Q; out_proj of up_v) on the same inputs.
 """
 from __future__ import annotations
 
@@ -101,6 +105,11 @@ def load(path: str):
     lib.mla_oracle_rope_rows_theta.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _i32p, _f64p, _f64p]
     lib.mla_oracle_up_v.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     lib.mla_oracle_out_proj.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
+    lib.mla_oracle_fold_qk.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
+    lib.mla_oracle_fold_ov.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
+    lib.mla_oracle_absorb_q_folded.argtypes = [ctypes.c_int] * 5 + [_f64p, _f64p, _i32p, _f64p, ctypes.c_double,
+                                                                   _f64p]
+    lib.mla_oracle_up_out_folded.argtypes = [ctypes.c_int] * 4 + [_f64p, _f64p, _f64p]
     return lib
 
 
@@ -371,4 +380,48 @@ def out_proj(heads, w_o) -> np.ndarray:
     d_model = w_o.shape[0]
     u = np.empty((T, d_model))
     _lib().mla_oracle_out_proj(T, H, d_h, d_model, _p(heads, _f64p), _p(w_o, _f64p), _p(u, _f64p))
+    return u
+
+
+# ------------------------------------------------ weight pre-absorption (f3)
+def fold_qk(w_uq, w_uk) -> np.ndarray:
+    """W^QK [H][d_c][d_q], W^QK_i = (U^K_i)^T W^UQ_i."""
+    w_uq, w_uk = _f64(w_uq), _f64(w_uk)
+    H, d_h, d_q = w_uq.shape
+    d_c = w_uk.shape[-1]
+    out = np.empty((H, d_c, d_q))
+    _lib().mla_oracle_fold_qk(H, d_h, d_c, d_q, _p(w_uq, _f64p), _p(w_uk, _f64p), _p(out, _f64p))
+    return out
+
+
+def fold_ov(w_o, w_uv) -> np.ndarray:
+    """W^OV [d_model][H*d_c], block i = O_i U^V_i."""
+    w_o, w_uv = _f64(w_o), _f64(w_uv)
+    H, d_h, d_c = w_uv.shape
+    d_model = w_o.shape[0]
+    out = np.empty((d_model, H * d_c))
+    _lib().mla_oracle_fold_ov(H, d_h, d_c, d_model, _p(w_o, _f64p), _p(w_uv, _f64p), _p(out, _f64p))
+    return out
+
+
+def absorb_q_folded(c_q, q_rope, w_qk, q_pos=None, base: float = 10000.0) -> np.ndarray:
+    """q_abs [T][H][d_c+d_r] = [W^QK_i c_q[t] | RoPE(q^R_{t,i}, q_pos[t])]."""
+    c_q, q_rope, w_qk = _f64(c_q), _f64(q_rope), _f64(w_qk)
+    T, d_q = c_q.shape
+    H, d_c, _ = w_qk.shape
+    d_r = q_rope.shape[-1]
+    qp = None if q_pos is None else _i32(q_pos)
+    out = np.empty((T, H, d_c + d_r))
+    _lib().mla_oracle_absorb_q_folded(T, H, d_c, d_q, d_r, _p(c_q, _f64p), _p(q_rope, _f64p), _p(qp, _i32p),
+                                      _p(w_qk, _f64p), float(base), _p(out, _f64p))
+    return out
+
+
+def up_out_folded(latent, w_ov) -> np.ndarray:
+    """u [T][d_model] = sum_i W^OV_i latent[t][i]."""
+    latent, w_ov = _f64(latent), _f64(w_ov)
+    T, H, d_c = latent.shape
+    d_model = w_ov.shape[0]
+    u = np.empty((T, d_model))
+    _lib().mla_oracle_up_out_folded(T, H, d_c, d_model, _p(latent, _f64p), _p(w_ov, _f64p), _p(u, _f64p))
     return u

@@ -662,3 +662,84 @@ void mla_oracle_out_proj(int T, int H, int d_h, int d_model, const double *heads
         u[td] = acc;
     }
 }
+
+/* ------------------------------------------------- weight pre-absorption (f3)
+ * DeepSeek-V2 paper review, section 2: at inference W^UK can be absorbed into
+ * the query's up-projection and W^UV into the output projection, so that the
+ * attention runs on the latent directly; the query path compresses to
+ * c^Q = W^DQ h (width d_q, 1536 in V2) and q^C_i = W^UQ_i c^Q.
+ *   W^QK_i = (U^K_i)^T W^UQ_i     [d_c][d_q]: q~_i = W^QK_i c^Q
+ *   W^OV[:, i d_c : (i+1) d_c] = O_i U^V_i     [d_model][H d_c]:
+ *                                  u = sum_i W^OV_i o~_i
+ * w_uq [H][d_h][d_q], w_uk, w_uv [H][d_h][d_c], w_o [d_model][H d_h]. */
+void mla_oracle_fold_qk(int H, int d_h, int d_c, int d_q, const double *w_uq, const double *w_uk, double *w_qk)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int i = 0; i < H; ++i)
+        for (int c = 0; c < d_c; ++c) {
+            double *out = w_qk + ((size_t)i * d_c + c) * d_q;
+            for (int q = 0; q < d_q; ++q) out[q] = 0.0;
+            for (int k = 0; k < d_h; ++k) {
+                const double u = w_uk[((size_t)i * d_h + k) * d_c + c];
+                const double *row = w_uq + ((size_t)i * d_h + k) * d_q;
+                for (int q = 0; q < d_q; ++q) out[q] += u * row[q];
+            }
+        }
+}
+
+void mla_oracle_fold_ov(int H, int d_h, int d_c, int d_model, const double *w_o, const double *w_uv, double *w_ov)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int m = 0; m < d_model; ++m)
+        for (int i = 0; i < H; ++i) {
+            double *out = w_ov + (size_t)m * H * d_c + (size_t)i * d_c;
+            for (int c = 0; c < d_c; ++c) out[c] = 0.0;
+            for (int k = 0; k < d_h; ++k) {
+                const double o = w_o[(size_t)m * H * d_h + (size_t)i * d_h + k];
+                const double *row = w_uv + ((size_t)i * d_h + k) * d_c;
+                for (int c = 0; c < d_c; ++c) out[c] += o * row[c];
+            }
+        }
+}
+
+/* Absorbed query from the compressed query latent with the folded weights:
+ * q_abs[t][i] = [W^QK_i c_q[t] | RoPE(q_rope[t][i], q_pos[t])] (copied if
+ * q_pos is NULL).  c_q [T][d_q], q_rope [T][H][d_r], w_qk [H][d_c][d_q]. */
+void mla_oracle_absorb_q_folded(int T, int H, int d_c, int d_q, int d_r, const double *c_q, const double *q_rope,
+                                const int32_t *q_pos, const double *w_qk, double base, double *q_abs)
+{
+    const int D = d_c + d_r;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int i = 0; i < H; ++i) {
+            double *o = q_abs + ((size_t)t * H + i) * D;
+            const double *x = c_q + (size_t)t * d_q;
+            for (int c = 0; c < d_c; ++c) {
+                const double *w = w_qk + ((size_t)i * d_c + c) * d_q;
+                double acc = 0.0;
+                for (int q = 0; q < d_q; ++q) acc += w[q] * x[q];
+                o[c] = acc;
+            }
+            const double *r = q_rope + ((size_t)t * H + i) * d_r;
+            if (q_pos)
+                mla_oracle_rope(r, d_r, (double)q_pos[t], base, o + d_c);
+            else
+                for (int m = 0; m < d_r; ++m) o[d_c + m] = r[m];
+        }
+}
+
+/* Output projection with the folded weights: u[t] = sum_i W^OV_i latent[t][i],
+ * latent [T][H][d_c], w_ov [d_model][H d_c]. */
+void mla_oracle_up_out_folded(int T, int H, int d_c, int d_model, const double *latent, const double *w_ov,
+                              double *u)
+{
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int m = 0; m < d_model; ++m) {
+            const double *w = w_ov + (size_t)m * H * d_c;
+            const double *x = latent + (size_t)t * H * d_c;
+            double acc = 0.0;
+            for (int j = 0; j < H * d_c; ++j) acc += w[j] * x[j];
+            u[(size_t)t * d_model + m] = acc;
+        }
+}

@@ -795,3 +795,109 @@ def test_rope_rows_theta_matches_plain_rope_and_preserves_norms(oracle_mod):
     a = oracle_mod.rope_rows_theta(q, np.array([7], np.int32), th) @ oracle_mod.rope_rows_theta(k, np.array([900], np.int32), th).T
     b = oracle_mod.rope_rows_theta(q, np.array([7007], np.int32), th) @ oracle_mod.rope_rows_theta(k, np.array([7900], np.int32), th).T
     assert abs(a - b) < 1e-10
+
+
+# ------------------------------------------------ weight pre-absorption pins
+def test_fold_identities_return_the_factors_exactly(oracle_mod):
+    """W^UQ_i = I (d_q = d_h) makes W^QK_i = (U^K_i)^T; W^O = I (d_model =
+    H d_h) makes the blocks of W^OV the U^V_i, placed block-diagonally."""
+    rng = np.random.default_rng(31)
+    H, d_h, d_c = 3, 8, 12
+    w_uk = rng.standard_normal((H, d_h, d_c))
+    w_uv = rng.standard_normal((H, d_h, d_c))
+    eye = np.broadcast_to(np.eye(d_h), (H, d_h, d_h)).copy()
+    got = oracle_mod.fold_qk(eye, w_uk)
+    assert np.array_equal(got, np.transpose(w_uk, (0, 2, 1)))
+    got = oracle_mod.fold_ov(np.eye(H * d_h), w_uv)
+    want = np.zeros((H * d_h, H * d_c))
+    for i in range(H):
+        want[i * d_h:(i + 1) * d_h, i * d_c:(i + 1) * d_c] = w_uv[i]
+    assert np.array_equal(got, want)
+
+
+def test_fold_brute_force_tiny_integers(oracle_mod):
+    """Each entry of W^QK and W^OV is one dot product, checked one by one on
+    small integers (exact in fp64)."""
+    rng = np.random.default_rng(32)
+    H, d_h, d_c, d_q, d_model = 2, 3, 4, 5, 6
+    w_uq = rng.integers(-3, 4, (H, d_h, d_q)).astype(np.float64)
+    w_uk = rng.integers(-3, 4, (H, d_h, d_c)).astype(np.float64)
+    w_uv = rng.integers(-3, 4, (H, d_h, d_c)).astype(np.float64)
+    w_o = rng.integers(-3, 4, (d_model, H * d_h)).astype(np.float64)
+    qk = oracle_mod.fold_qk(w_uq, w_uk)
+    ov = oracle_mod.fold_ov(w_o, w_uv)
+    for i in range(H):
+        for c in range(d_c):
+            for q in range(d_q):
+                assert qk[i, c, q] == sum(w_uk[i, k, c] * w_uq[i, k, q] for k in range(d_h))
+    for m in range(d_model):
+        for i in range(H):
+            for c in range(d_c):
+                assert ov[m, i * d_c + c] == sum(w_o[m, i * d_h + k] * w_uv[i, k, c] for k in range(d_h))
+
+
+def test_folded_paths_equal_the_two_step_paths(oracle_mod):
+    """The identities the folding rests on, against the pinned routines:
+    absorb_q_folded(c^Q) = absorb_q(q^C = W^UQ c^Q) and up_out_folded(õ) =
+    out_proj(up_v(õ))."""
+    rng = np.random.default_rng(33)
+    T, H, d_h, d_c, d_r, d_q, d_model = 3, 4, 8, 16, 8, 24, 20
+    w_uq = rng.standard_normal((H, d_h, d_q))
+    w_uk = rng.standard_normal((H, d_h, d_c))
+    w_uv = rng.standard_normal((H, d_h, d_c))
+    w_o = rng.standard_normal((d_model, H * d_h))
+    c_q = rng.standard_normal((T, d_q))
+    q_rope = rng.standard_normal((T, H, d_r))
+    q_pos = np.array([0, 7, 300], np.int32)
+    q_c = np.einsum("ikq,tq->tik", w_uq, c_q)
+    want = oracle_mod.absorb_q(q_c, q_rope, w_uk, q_pos=q_pos)
+    got = oracle_mod.absorb_q_folded(c_q, q_rope, oracle_mod.fold_qk(w_uq, w_uk), q_pos=q_pos)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(got[..., d_c:],
+                                  oracle_mod.absorb_q_folded(c_q, q_rope, np.zeros((H, d_c, d_q)),
+                                                             q_pos=q_pos)[..., d_c:])
+    lat = rng.standard_normal((T, H, d_c))
+    want = oracle_mod.out_proj(oracle_mod.up_v(lat, w_uv), w_o)
+    got = oracle_mod.up_out_folded(lat, oracle_mod.fold_ov(w_o, w_uv))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+FOLD_MUTATIONS = {
+    "qk_untransposed": ("const double u = w_uk[((size_t)i * d_h + k) * d_c + c];",
+                        "const double u = w_uk[((size_t)i * d_h + c % d_h) * d_c + k];"),
+    "ov_wrong_head_block": ("const double o = w_o[(size_t)m * H * d_h + (size_t)i * d_h + k];",
+                            "const double o = w_o[(size_t)m * H * d_h + (size_t)((i + 1) % H) * d_h + k];"),
+    "absorb_folded_drops_rope": ("mla_oracle_rope(r, d_r, (double)q_pos[t], base, o + d_c);",
+                                 "for (int m = 0; m < d_r; ++m) o[d_c + m] = r[m];"),
+    "up_out_folded_skips_last_head": ("for (int j = 0; j < H * d_c; ++j) acc += w[j] * x[j];",
+                                      "for (int j = 0; j < (H - 1) * d_c; ++j) acc += w[j] * x[j];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FOLD_MUTATIONS))
+def test_planted_fold_mistakes_are_caught(oracle_mod, tmp_path, name):
+    """One plausible mistake in the folding routines of a copy of the oracle
+    must make one of the folding pins fail."""
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle_mod.__file__), "mla_oracle.c")).read()
+    old, new = FOLD_MUTATIONS[name]
+    assert src.count(old) == 1, name
+    mutant = tmp_path / "m.c"
+    mutant.write_text(src.replace(old, new, 1))
+    so = tmp_path / "m.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(mutant), "-lm"], check=True)
+    saved = oracle_mod._LIB
+    oracle_mod._LIB = oracle_mod.load(str(so))
+    pins = (test_fold_identities_return_the_factors_exactly, test_fold_brute_force_tiny_integers,
+            test_folded_paths_equal_the_two_step_paths)
+    try:
+        caught = False
+        for pin in pins:
+            try:
+                pin(oracle_mod)
+            except AssertionError:
+                caught = True
+                break
+        assert caught, f"mutation {name} was not caught"
+    finally:
+        oracle_mod._LIB = saved
