@@ -412,6 +412,7 @@ def run_ours(args):
         line["per_config_fp8"] = per_config(M, [n for n in ("v2lite", "v2", "longctx", "mtp")], fp8=True)
     if not args.no_prefill and world == 1:
         line["prefill"] = prefill_bench(M)
+        line["folded_weights"] = fold_bench(M)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     print(json.dumps(line), flush=True)
@@ -586,6 +587,63 @@ def prefill_bench(M, names=tuple(PREFILL_WORKLOADS), iters=10):
     return out
 
 
+# ------------------------------------------------- weight pre-absorption
+def fold_bench(M, T=128, H=128, d_q=1536, d_model=5120, iters=20):
+    """The query absorption and output projection of one decode step of the
+    V2 shape (T tokens), two-step (mla_absorb_q from q^C, mla_up_v with W^O)
+    against folded (mla_absorb_q_folded from c^Q, mla_up_out_folded), each
+    call's CUDA-event time (mean of `iters` after 3 warm-ups, 256 MB L2 flush
+    before each call) and the weight bytes it reads.  The two-step absorb
+    takes q^C as given, so its time leaves out the W^UQ projection that
+    produces q^C (a further 50 MB of weights at this shape)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3001)
+    dev = dict(device="cuda")
+    rnd = lambda *shape, std=1.0: (torch.randn(shape, generator=g, **dev) * std).to(torch.bfloat16)
+    dims = M.dims(H)
+    c_q, q_c, q_r = rnd(T, d_q), rnd(T, H, 128), rnd(T, H, 64)
+    q_pos = torch.arange(T, dtype=torch.int32, **dev)
+    w_uq, w_uk, w_uv = rnd(H, 128, d_q, std=d_q ** -0.5), rnd(H, 128, 512, std=512 ** -0.5), rnd(H, 128, 512, std=512 ** -0.5)
+    w_o = rnd(d_model, H * 128, std=(H * 128) ** -0.5)
+    w_qk = torch.empty(H, 512, d_q, dtype=torch.bfloat16, **dev)
+    w_ov = torch.empty(d_model, H * 512, dtype=torch.bfloat16, **dev)
+    M.mla_fold_weights(dims, w_uq, w_uk, w_qk, w_o, w_uv, w_ov)
+    lat = rnd(T, H, 512, std=0.125)
+    q_abs = torch.empty(T, H, 576, dtype=torch.bfloat16, **dev)
+    heads = torch.empty(T, H, 128, dtype=torch.bfloat16, **dev)
+    u = torch.empty(T, d_model, dtype=torch.bfloat16, **dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, **dev)
+    E = torch.cuda.Event
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        ts = []
+        for _ in range(iters):
+            flush.fill_(1)
+            a, b = E(enable_timing=True), E(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return float(np.mean([x.elapsed_time(y) for x, y in ts])) * 1e3
+
+    out = {"workload": f"V2-shaped decode step: T={T}, H={H}, d_q={d_q}, d_model={d_model}",
+           "absorb_two_step_us": timed(lambda: M.mla_absorb_q(dims, q_c, q_r, q_pos, w_uk, q_abs)),
+           "absorb_folded_us": timed(lambda: M.mla_absorb_q_folded(dims, c_q, q_r, q_pos, w_qk, q_abs)),
+           "out_two_step_us": timed(lambda: M.mla_up_v(dims, lat, w_uv, heads, w_o=w_o, out_model=u)),
+           "out_folded_us": timed(lambda: M.mla_up_out_folded(dims, lat, w_ov, u)),
+           "fold_weights_us": timed(lambda: M.mla_fold_weights(dims, w_uq, w_uk, w_qk, w_o, w_uv, w_ov)),
+           "weight_bytes": {"U^K": H * 128 * 512 * 2, "W^UQ": H * 128 * d_q * 2, "W^QK": H * 512 * d_q * 2,
+                            "U^V": H * 128 * 512 * 2, "W^O": d_model * H * 128 * 2, "W^OV": d_model * H * 512 * 2},
+           "l2": "flushed before each call"}
+    del flush, w_qk, w_ov, w_o
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------- CPU oracle (baseline)
 def cpu_baseline(cfg: W.MLAConfig, budget_s: float = 10.0):
     """The fp64 expanded-form oracle, as it stands, on a bounded sample of the
@@ -705,7 +763,7 @@ def main():
         import head_latent_attention_10_b200 as M
         M.load_library()
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        print(json.dumps({"prefill": prefill_bench(M)}), flush=True)
+        print(json.dumps({"prefill": prefill_bench(M), "folded_weights": fold_bench(M)}), flush=True)
     else:
         run_ours(args)
 

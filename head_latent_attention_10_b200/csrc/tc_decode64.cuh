@@ -60,7 +60,7 @@
 // FP8 cache (kFp8): a page is 576 E4M3 codes per token plus two fp32 scales
 // per token (csrc/fp8.cuh).  TMA lands the codes, one 64-column box per
 // chunk (4 KB each), in the upper half of the stage and the page's 512 B of
-// scales in a side slot; two extra warps (8-9) widen them in place into the
+// scales in a side slot; four extra warps (8-11) widen them in place into the
 // same f16 tile layout the bf16 path uses, with the token's larger scale
 // s_j = max(sc_c, sc_r) factored out: the f16 values are code * sc / s_j
 // (one part exact, the other scaled by <= 1), so the logits MMA gives l_j / s_j
@@ -90,9 +90,11 @@ constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-5
 constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
 constexpr uint32_t kD64TmS2 = 416;                // third logits buffer: lanes 0-15, columns 416-479
 constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
-// FP8 cache: 64 more threads (the converters), per-stage scale slots
+// FP8 cache: 128 more threads (the converters), per-stage scale slots
 // ([64][2] fp32) and per-token factored scales s_j ([64] fp32) after the stages
-constexpr int kD64ThreadsFp8 = kD64Threads + 64;
+constexpr int kD64Cvt = 128;                       // converter threads (warps 8-11)
+constexpr int kD64ThreadsFp8 = kD64Threads + kD64Cvt;
+constexpr int kD64CvtRows = kT64 * 4 / kD64Cvt;    // rows per converter thread (4 threads per row)
 constexpr int kD64F8Codes = kT64 * kRow;          // 36,864 (one code per value): where the codes land
 constexpr int kD64F8Box = kT64 * 64;              // one 64-column box of codes (4 KB)
 constexpr int kD64OffScale = kD64Stages * kD64Stage;              // [3][64][2] fp32
@@ -108,7 +110,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(d64_smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (kFp8 ? kD64OffBarFp8 : kD64OffBar));
-    uint64_t *cv_full = bars + 32;   // [3] FP8: the stage's codes widened to f16 (2 converter warps)
+    uint64_t *cv_full = bars + 32;   // [3] FP8: the stage's codes widened to f16 (the converter warps)
     uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
     uint64_t *kv_empty = bars + 21;  // [3] P.C MMAs of the stage done -> TMA, softmax
     // Q of segment n is in TMEM once q_cnt >= 4 (n + 1) (each softmax warp adds
@@ -140,7 +142,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         }
         for (int i = 0; i < kD64Stages; ++i) p_cnt[i] = 0;
         if constexpr (kFp8)
-            for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&cv_full[i], 2);
+            for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&cv_full[i], kD64Cvt / 32);
         sm100::mbar_init(mma_done, 7);
         *abort_flag = 0;
         sm100::fence_mbar_init();
@@ -266,8 +268,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             is.advance();
         }
     } else if (kFp8 && warp >= 8) {
-        // ------------------------------------------------ FP8 -> f16 (warps 8-9)
-        // thread ct: rows rr_i = ct / 4 + 16 i (i = 0..3), 16-code segment g =
+        // ----------------------------------------------- FP8 -> f16 (warps 8-11)
+        // thread ct: rows rr_i = ct / 4 + 32 i (i = 0, 1), 16-code segment g =
         // ct % 4 of each 64-column chunk (a warp reads 512 contiguous bytes)
         const int ct = threadIdx.x - kD64Threads, g = ct & 3;
         TileIter it;
@@ -276,12 +278,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         while (ok && it.ok) {
             const int k = it.k, st = k % kD64Stages;
             ok = sm100::warp_wait(&kv_full[st], (k / kD64Stages) & 1, abort_flag, a.err, lim);
-            // both converter warps go on only if both saw the page land: they
-            // meet at named barriers below, which neither may skip
+            // the converter warps go on only if all saw the page land: they
+            // meet at named barriers below, which none may skip
             {
                 uint32_t both;
                 asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-                             "bar.red.and.pred p, 3, 64, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                             "bar.red.and.pred p, 3, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
                              : "=r"(both) : "r"((uint32_t)ok) : "memory");
                 ok = both != 0;
             }
@@ -289,11 +291,11 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             uint8_t *stg = stages + st * kD64Stage;
             const float2 *scl = reinterpret_cast<const float2 *>(smem + kD64OffScale + st * 512);
             float *smax = reinterpret_cast<float *>(smem + kD64OffSmax + st * 256);
-            uint32_t rat_c[4], rat_r[4];   // f16x2 ratios sc / s_j of the thread's rows
-            bool one_c[4], one_r[4];
+            uint32_t rat_c[kD64CvtRows], rat_r[kD64CvtRows];   // f16x2 ratios sc / s_j of the thread's rows
+            bool one_c[kD64CvtRows], one_r[kD64CvtRows];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int rr = (ct >> 2) + 16 * i;
+            for (int i = 0; i < kD64CvtRows; ++i) {
+                const int rr = (ct >> 2) + 32 * i;
                 const float2 sc = scl[rr];
                 const float m = fmaxf(sc.x, sc.y);
                 const float fc = sc.x / m, fr = sc.y / m;
@@ -306,14 +308,14 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             }
             auto read = [&](int j, uint4 *in) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < kD64CvtRows; ++i)
                     in[i] = *reinterpret_cast<const uint4 *>(stg + kD64F8Codes + j * kD64F8Box +
-                                                             64 * ((ct >> 2) + 16 * i) + 16 * g);
+                                                             64 * ((ct >> 2) + 32 * i) + 16 * g);
             };
             auto write = [&](int j, const uint4 *in, const uint32_t *rat, const bool *one) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int rr = (ct >> 2) + 16 * i;
+                for (int i = 0; i < kD64CvtRows; ++i) {
+                    const int rr = (ct >> 2) + 32 * i;
                     const uint16_t *c = reinterpret_cast<const uint16_t *>(&in[i]);
                     uint32_t h[8];
 #pragma unroll
@@ -331,8 +333,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     *reinterpret_cast<uint4 *>(rowp + (((2 * g + 1) ^ (rr & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
                 }
             };
-            auto group_sync = [] { asm volatile("bar.sync 3, 64;" ::: "memory"); };
-            uint4 in[4], in8[4];
+            auto group_sync = [] { asm volatile("bar.sync 3, 128;" ::: "memory"); };
+            uint4 in[kD64CvtRows], in8[kD64CvtRows];
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) { read(j, in); write(j, in, rat_c, one_c); }
             group_sync();

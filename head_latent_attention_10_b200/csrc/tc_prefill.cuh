@@ -17,15 +17,19 @@
 //   S(k) = Q K_k^T    N=128, K=192: 12 MMAs, Q read from TMEM
 //   P(k) = exp2(S(k) scale log2 e - m)           bf16, one thread per query row
 //   O   += P(k) V_k   N=128, K=128: 8 MMAs, P read from TMEM
-// TMEM (512 columns): S 0-127, P(k % 2) 128-191 / 192-255, O 256-383,
-// Q 384-479 (192 bf16 per row, written by the softmax warps at the start).
+// TMEM (512 columns): S(k) in buffer k % 2 (columns 0-127, 128-255), P(k)
+// written over the first 64 columns of its S buffer, O 256-383, Q 384-479
+// (192 bf16 per row, written by the softmax warps at the start).
 // With Q and P in TMEM, shared memory holds only key and value tiles: a
 // 3-slot ring of K tiles (K^C 0-63, K^C 64-127, k^R; 48 KB each) and a 2-slot
 // ring of V tiles (V^C 0-63, 64-127; 32 KB each), 208 KB, each ring fed by
 // its own loader warp (0: K, 6: V) so that neither waits behind the other.
-// Warp 1 issues S(k+1) as soon as the softmax warps (2-5) have read S(k) out
-// of TMEM, so the logits of the next tile run while the softmax of this one
-// computes, then P(k) V_k once P(k) is written.  The causal mask applies to
+// Warp 1 keeps the logits one tile ahead: S(0), S(1), then S(k+2) into
+// buffer k % 2 once P(k) V_k has completed (S(k+2) overwrites P(k)), so the
+// softmax warps (2-5) find the next tile's logits ready when they finish this
+// one; warp 7 issues P(k) V_k as soon as P(k) is written.  Two issuing
+// threads, because a thread's tcgen05.mma issue blocks while the tensor pipe
+// is busy, and one thread would hold P(k+1) V back behind S(k+2).  The causal mask applies to
 // the tiles that straddle the diagonal; lazy rescaling as in the decode (O
 // is rescaled in TMEM only when the running max grows by more than 8, after
 // the previous P V has retired).  Every wait is bounded; no TMA load uses
@@ -36,14 +40,14 @@
 
 namespace mla {
 
-constexpr int kPfThreads = 224;                        // warps: 0 K loads, 1 MMA, 2-5 softmax, 6 V loads
+constexpr int kPfThreads = 256;                        // warps: 0 K loads, 1 S MMAs, 2-5 softmax, 6 V loads, 7 P V MMAs
 constexpr int kPfChunk = 128 * 128;                    // [128 rows][64 bf16], 128-byte swizzle: 16 KB
 constexpr int kPfKSlots = 3, kPfVSlots = 2;
 constexpr int kPfOffK = 0;                             // K slot j: chunks 3j .. 3j+2
 constexpr int kPfOffV = kPfKSlots * 3 * kPfChunk;      // V slot j: 2 chunks
 constexpr int kPfOffBar = kPfOffV + kPfVSlots * 2 * kPfChunk;   // 212,992
 constexpr int kPfSmem = kPfOffBar + 256 + 1024;        // barriers, alignment slack
-constexpr uint32_t kPfTmS = 0, kPfTmP = 128, kPfTmO = 256, kPfTmQ = 384;
+constexpr uint32_t kPfTmS = 0, kPfTmO = 256, kPfTmQ = 384;   // S/P buffers at 0 and 128
 
 // Tensor maps of one call.  Rows of K^C, V^C and the gathered latents are
 // [B * Lpad] long (sequence b at rows b * Lpad ..); outputs are [B][s][H][128]
@@ -89,11 +93,10 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
     uint64_t *v_full = bars + 6;        // [2] V slot loaded
     uint64_t *v_free = bars + 8;        // [2] P V of the slot's tile done
     uint64_t *q_ready = bars + 10;      // Q in TMEM (4 softmax warps)
-    uint64_t *s_full = bars + 11;       // S(k) in TMEM
-    uint64_t *s_free = bars + 12;       // S(k) read out (4 softmax warps)
+    uint64_t *s_full = bars + 11;       // [2] S(k) in buffer k % 2
     uint64_t *p_full = bars + 13;       // [2] P(k) in TMEM and O rescaled (4 softmax warps)
     uint64_t *pv_done = bars + 15;      // [2] P(k) V_k done
-    uint64_t *done = bars + 17;         // the issuer's last MMAs done (teardown)
+    uint64_t *done = bars + 17;         // both issuers' last MMAs done (teardown)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 19);
 
@@ -118,9 +121,9 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
             sm100::mbar_init(&pv_done[i], 1);
         }
         sm100::mbar_init(q_ready, 4);
-        sm100::mbar_init(s_full, 1);
-        sm100::mbar_init(s_free, 4);
-        sm100::mbar_init(done, 1);
+        sm100::mbar_init(&s_full[0], 1);
+        sm100::mbar_init(&s_full[1], 1);
+        sm100::mbar_init(done, 2);
         *abort_flag = 0;
         sm100::fence_mbar_init();
         sm100::prefetch_tensormap(&maps.kc);
@@ -181,43 +184,47 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
                     sm100::mbar_wait(&v_full[k & 1], (k >> 1) & 1, &no_abort, a.err, drain);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 7) {
         // ------------------------------------------------------ MMA issue
         if (lane == 0) {
             const uint32_t idesc_s = sm100::idesc_bf16(128, 128, 0, 0);
             const uint32_t idesc_o = sm100::idesc_bf16(128, 128, 0, 1);
             bool ok = nk == 0 || sm100::mbar_wait(q_ready, 0, abort_flag, a.err, lim);
-            // step k issues S(k), then P(k-1) V_{k-1}
-            for (int k = 0; ok && k <= nk; ++k) {
-                if (k < nk) {
+            if (warp == 1) {
+                // S(k) into buffer k % 2
+                auto issue_s = [&](int k) -> bool {
                     const int sl = k % kPfKSlots;
-                    ok = sm100::mbar_wait(&k_full[sl], (k / kPfKSlots) & 1, abort_flag, a.err, lim);
-                    // S(k) overwrites S(k-1): the softmax must have read it
-                    if (ok && k > 0) ok = sm100::mbar_wait(s_free, (k - 1) & 1, abort_flag, a.err, lim);
-                    if (!ok) break;
+                    if (!sm100::mbar_wait(&k_full[sl], (k / kPfKSlots) & 1, abort_flag, a.err, lim)) return false;
                     sm100::tc_fence_after();
                     const uint32_t ka = sm100::smem_u32(smem + kPfOffK + 3 * sl * kPfChunk);
 #pragma unroll
                     for (int step = 0; step < 12; ++step)      // q^C 0-63, q^C 64-127, q^R
-                        sm100::umma_ts(tmem + kPfTmS, tmem + kPfTmQ + 8 * step,
+                        sm100::umma_ts(tmem + kPfTmS + 128 * (k & 1), tmem + kPfTmQ + 8 * step,
                                        sm100::desc_kmajor(ka + (step >> 2) * kPfChunk + (step & 3) * 32, 128,
                                                           sm100::kSw128),
                                        idesc_s, step > 0);
-                    sm100::umma_commit(s_full);
+                    sm100::umma_commit(&s_full[k & 1]);
                     sm100::umma_commit(&k_free[sl]);
-                }
-                if (k > 0) {
-                    const int j = k - 1, pb = j & 1;
-                    ok = sm100::mbar_wait(&p_full[pb], (j >> 1) & 1, abort_flag, a.err, lim) &&
-                         sm100::mbar_wait(&v_full[pb], (j >> 1) & 1, abort_flag, a.err, lim);
+                    return true;
+                };
+                if (ok && nk > 0) ok = issue_s(0);
+                if (ok && nk > 1) ok = issue_s(1);
+                // S(k+2) overwrites P(k): that P V must have completed
+                for (int k = 0; ok && k + 2 < nk; ++k)
+                    ok = sm100::mbar_wait(&pv_done[k & 1], (k >> 1) & 1, abort_flag, a.err, lim) && issue_s(k + 2);
+            } else {
+                for (int k = 0; ok && k < nk; ++k) {
+                    const int pb = k & 1;
+                    ok = sm100::mbar_wait(&p_full[pb], (k >> 1) & 1, abort_flag, a.err, lim) &&
+                         sm100::mbar_wait(&v_full[pb], (k >> 1) & 1, abort_flag, a.err, lim);
                     if (!ok) break;
                     sm100::tc_fence_after();
-                    const uint64_t vd = sm100::desc_mnmajor_sw128(sm100::smem_u32(smem + kPfOffV + 2 * pb * kPfChunk),
-                                                                  kPfChunk);
+                    const uint64_t vd =
+                        sm100::desc_mnmajor_sw128(sm100::smem_u32(smem + kPfOffV + 2 * pb * kPfChunk), kPfChunk);
 #pragma unroll
                     for (int kq = 0; kq < 8; ++kq)           // 16 keys per MMA: 8 TMEM columns of P
-                        sm100::umma_ts(tmem + kPfTmO, tmem + kPfTmP + 64 * pb + 8 * kq,
-                                       vd + (uint64_t)((kq * 2048) >> 4), idesc_o, (j > 0 || kq > 0) ? 1u : 0u);
+                        sm100::umma_ts(tmem + kPfTmO, tmem + kPfTmS + 128 * pb + 8 * kq,
+                                       vd + (uint64_t)((kq * 2048) >> 4), idesc_o, (k > 0 || kq > 0) ? 1u : 0u);
                     sm100::umma_commit(&pv_done[pb]);
                     sm100::umma_commit(&v_free[pb]);
                 }
@@ -231,7 +238,7 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
         const int qd = warp & 3;
         const int r = 32 * qd + lane, t = q0 + r;
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        const uint32_t tm_s = tmem + lane_off + kPfTmS, tm_p = tmem + lane_off + kPfTmP;
+        const uint32_t tm_s = tmem + lane_off + kPfTmS;
         const uint32_t tm_o = tmem + lane_off + kPfTmO, tm_q = tmem + lane_off + kPfTmQ;
         const bool has_row = t < a.s;
         const int nvis = has_row ? L - a.s + t + 1 : 0;   // keys [0, nvis) visible to row t
@@ -259,16 +266,13 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
         float m_run = -INFINITY, l_run = 0.f;
         for (int k = 0; ok && k < nk; ++k) {
             const int pb = k & 1;
-            ok = sm100::warp_wait(s_full, k & 1, abort_flag, a.err, lim);
+            ok = sm100::warp_wait(&s_full[pb], (k >> 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
             uint32_t x[128];
 #pragma unroll
-            for (int c = 0; c < 128; c += 32) sm100::tmem_ld32(tm_s + c, x + c);
+            for (int c = 0; c < 128; c += 32) sm100::tmem_ld32(tm_s + 128 * pb + c, x + c);
             sm100::tmem_wait_ld();
-            sm100::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) sm100::mbar_arrive(s_free);      // S(k+1) may go in now
             const int key0 = 128 * k;
             if (key0 + 128 > nvis) {
 #pragma unroll
@@ -297,14 +301,9 @@ tc_prefill_kernel(const __grid_constant__ PrefillMaps maps, const PrefillArgs a)
                 x[c] = pack_bf162(p0, p1);
             }
             l_run += lsum;
-            // P(k) into buffer pb once P(k-2) V_{k-2}, its last reader, is done
-            if (k >= 2) {
-                ok = sm100::warp_wait(&pv_done[pb], ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
-                if (!ok) break;
-                sm100::tc_fence_after();
-            }
-            sm100::tmem_st32(tm_p + 64 * pb, x);
-            sm100::tmem_st32(tm_p + 64 * pb + 32, x + 32);
+            // P(k) over the first 64 columns of S(k), already read by this thread
+            sm100::tmem_st32(tm_s + 128 * pb, x);
+            sm100::tmem_st32(tm_s + 128 * pb + 32, x + 32);
             if (__any_sync(0xffffffffu, rescale)) {
                 // O holds the tiles before k: let P(k-1) V_{k-1} retire, then
                 // scale this thread's row in place
