@@ -396,15 +396,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 for (int j = 0; j < 3; ++j)
                     sm100::tmem_st16x2_16(lane_base + kD64TmQ + 32 * (3 * g + j), reinterpret_cast<const uint32_t *>(v + 4 * j));
             }
-            // warm L2 with the following sequence's row, the next one a range moving on reads
-            if (row_ok && seq + 1 < a.B) {
-                // the row's nine 128-byte lines: five by thread i, four by thread 16+i
-                const char *nq = reinterpret_cast<const char *>(
-                    a.q_abs + ((long long)(seq + 1) * rows_per_seq + grow_row) * kRow);
-#pragma unroll
-                for (int e = 0; e < 5; ++e)
-                    if (srow || e < 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * (srow ? e : 5 + e)));
-            }
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
             __syncwarp();
@@ -412,6 +403,17 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 __threadfence_block();
                 atomicAdd(const_cast<int *>(q_cnt), 1);
             }
+        };
+        // warm L2 with the row of the sequence a range moves on to, a few
+        // tiles before the switch (earlier, the streaming cache pages would
+        // evict it again): the row's nine 128-byte lines, five by thread i,
+        // four by thread 16+i
+        auto prefetch_q = [&](int seq) {
+            if (!row_ok || seq >= a.B) return;
+            const char *nq = reinterpret_cast<const char *>(a.q_abs + ((long long)seq * rows_per_seq + grow_row) * kRow);
+#pragma unroll
+            for (int e = 0; e < 5; ++e)
+                if (srow || e < 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * (srow ? e : 5 + e)));
         };
         TileIter it;
         it.init(seq_start, a.B, lo, hi);
@@ -422,6 +424,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         if (it.ok) write_q(it.seq);
         while (ok && it.ok) {
             const int k = it.k;
+            if (it.tt + 4 == it.t1 || (it.first() && it.t1 - it.t0 < 4)) prefetch_q(it.seq + 1);
             if (it.first()) {
                 m_run = -INFINITY;
                 l_run = 0.f;
