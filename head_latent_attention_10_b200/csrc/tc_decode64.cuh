@@ -111,7 +111,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (kFp8 ? kD64OffBarFp8 : kD64OffBar));
     uint64_t *cv_full = bars + 32;   // [3] FP8: the stage's codes widened to f16 (the converter warps)
-    uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA
+    uint64_t *kv_full = bars + 18;   // [3] TMA -> MMA (bf16: chunks 5-8 of the page)
+    uint64_t *kv_half = bars + 35;   // [3] bf16: chunks 0-4 of the page landed
     uint64_t *kv_empty = bars + 21;  // [3] P.C MMAs of the stage done -> TMA, softmax
     // Q of segment n is in TMEM once q_cnt >= 4 (n + 1) (each softmax warp adds
     // 1 per segment): a count rather than a barrier phase, so that an issuer
@@ -134,7 +135,11 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     const int rows_per_seq = a.s * a.H;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kD64Stages; ++i) { sm100::mbar_init(&kv_full[i], 1); sm100::mbar_init(&kv_empty[i], 1); }
+        for (int i = 0; i < kD64Stages; ++i) {
+            sm100::mbar_init(&kv_full[i], 1);
+            sm100::mbar_init(&kv_empty[i], 1);
+            sm100::mbar_init(&kv_half[i], 1);
+        }
         *q_cnt = 0;
         for (int i = 0; i < 3; ++i) {
             sm100::mbar_init(&s_full[i], 1);
@@ -212,9 +217,12 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     sm100::bulk_load(smem + kD64OffScale + st * 512, a.scales + (long long)blk * 128, 512,
                                      &kv_full[st]);
                 } else {
-                    sm100::mbar_arrive_expect_tx(&kv_full[st], kD64Stage);
+                    // two halves, so the logits can start on chunks 0-4 while 5-8 land
+                    sm100::mbar_arrive_expect_tx(&kv_half[st], 5 * kD64Chunk);
+                    sm100::mbar_arrive_expect_tx(&kv_full[st], 4 * kD64Chunk);
                     for (int j = 0; j < 9; ++j)
-                        sm100::tma_load_3d(&map_kv, &kv_full[st], dst + j * kD64Chunk, 64 * j, blk * kBlock, 0);
+                        sm100::tma_load_3d(&map_kv, j < 5 ? &kv_half[st] : &kv_full[st], dst + j * kD64Chunk, 64 * j,
+                                           blk * kBlock, 0);
                 }
                 issued_k = k + 1;
                 it.advance();
@@ -222,8 +230,11 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             if (*abort_flag) {  // wait for the copies still in flight
                 volatile int no_abort = 0;
                 for (int kk = issued_k - kD64Stages < 0 ? 0 : issued_k - kD64Stages; kk < issued_k; ++kk)
-                    if (kk != a.stall_tile)
+                    if (kk != a.stall_tile) {
                         sm100::mbar_wait(&kv_full[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
+                        if (!kFp8)
+                            sm100::mbar_wait(&kv_half[kk % kD64Stages], (kk / kD64Stages) & 1, &no_abort, a.err, drain);
+                    }
             }
         }
     } else if (warp >= 1 && warp <= 3) {
@@ -250,20 +261,30 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 q_seg = is.seg;
             }
             if (!ok) break;
-            ok = sm100::warp_wait(kFp8 ? &cv_full[st] : &kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
+            ok = sm100::warp_wait(kFp8 ? &cv_full[st] : &kv_half[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim);
             if (ok && kk >= 3) ok = sm100::warp_wait(&s_free[b], ((kk / 3) - 1) & 1, abort_flag, a.err, lim);
             if (!ok) break;
             sm100::tc_fence_after();
+            int ok2 = 1;
             if (lane == 0) {
                 const uint64_t kd = sm100::desc_kmajor(sm100::smem_u32(stages + st * kD64Stage), 128, sm100::kSw128);
                 const uint32_t d = tmem + scol;
 #pragma unroll
                 for (int step = 0; step < 36; ++step) {          // 16-column K steps
+                    if (!kFp8 && step == 20) {
+                        // chunks 5-8 (the bf16 page's second half)
+                        if (!sm100::mbar_wait(&kv_full[st], (kk / kD64Stages) & 1, abort_flag, a.err, lim)) {
+                            ok2 = 0;
+                            break;
+                        }
+                        sm100::tc_fence_after();
+                    }
                     const uint32_t off = (step >> 2) * kD64Chunk + (step & 3) * 32;
                     sm100::umma_ts(d, tmem + kD64TmQ + 8 * step, kd + (uint64_t)(off >> 4), idesc_s, step > 0);
                 }
-                sm100::umma_commit(&s_full[b]);
+                if (ok2) sm100::umma_commit(&s_full[b]);
             }
+            ok = __shfl_sync(0xffffffffu, ok2, 0) != 0;
             __syncwarp();
             is.advance();
         }
