@@ -3,6 +3,8 @@
 // and the plan kernel that cuts the batch's tiles into equal ranges.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace mla {
@@ -15,7 +17,8 @@ struct DecArgs {
     const bf16 *q_abs;    // [B*s][H][576]
     const int32_t *block_table;
     const int32_t *seq_lens;
-    const int32_t *plan;  // [0]=tiles per range, [1]=total tiles, [2]=ranges, [4..4+B] sequence tile starts
+    const int32_t *plan;  // [0]=tiles per range, [1]=total tiles, [2]=ranges, [4..4+B] sequence tile starts,
+                          // [5+B+r] first sequence of range r
     bf16 *out;
     float *out_lse;
     float *part_o;        // [2*ranges][s*H][512] fp32
@@ -41,17 +44,6 @@ __device__ __forceinline__ int seq_len_clamped(const int32_t *seq_lens, int b, i
     return L < 0 ? 0 : min(L, max_blocks * kBlock);
 }
 
-// Largest r in [0, n] with start[r] <= x.
-__device__ __forceinline__ int find_seq(const int32_t *start, int n, int x)
-{
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (start[mid] <= x) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
 // Walks a range of the (sequence, tile) list one tile at a time.
 struct TileIter {
     const int32_t *rs;
@@ -69,10 +61,12 @@ struct TileIter {
         pos = end; ++r; ++seg;
         return true;
     }
-    __device__ void init(const int32_t *start, int n_, int lo, int hi_)
+    // r0: the sequence holding tile lo (find_seq(start, n, lo)), which the
+    // plan kernel stores for every range
+    __device__ void init(const int32_t *start, int n_, int lo, int hi_, int r0)
     {
         rs = start; n = n_; pos = lo; hi = hi_; seg = -1; k = 0;
-        r = find_seq(rs, n, lo);
+        r = r0;
         ok = next_seg();
         tt = t0;
     }
@@ -127,16 +121,29 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 // -------------------------------------------------------------------- plan
 // One CTA: `tile`-token tiles of every sequence (its last query sees all L
-// tokens), their prefix sums, and the per-range quota.
+// tokens), their prefix sums, the per-range quota, and the sequence each range
+// starts in (so that no decode warp searches the prefix sums at its start).
 // plan[0] = tiles per range, plan[1] = total tiles, plan[2] = ranges,
-// plan[4 + b] = first tile of sequence b (b = 0..B).
+// plan[4 + b] = first tile of sequence b (b = 0..B),
+// plan[5 + B + r] = sequence holding tile r * plan[0] (ranges r that start
+// before the end of the list).
+constexpr int kPlanInts = 5 + kMaxRanges;   // + B: ints of the plan
 __global__ void __launch_bounds__(1024)
 dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int tile,
                 int32_t *__restrict__ plan, uint32_t *err)
 {
     __shared__ int part[1024];
+    __shared__ int quota;
     sm100::pdl_trigger();   // the decode kernel may set itself up meanwhile
     const int per = (B + 1023) / 1024;
     const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
@@ -158,19 +165,26 @@ dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_bloc
         part[threadIdx.x] += v;
         __syncthreads();
     }
+    if (threadIdx.x == 1023) {
+        const int total = part[1023];
+        const int q = total > 0 ? (total + ranges - 1) / ranges : 1;
+        plan[4 + B] = total;
+        plan[1] = total;
+        plan[2] = ranges;
+        plan[0] = q;
+        quota = q;
+    }
+    __syncthreads();
+    const int q = quota;
     int run = part[threadIdx.x] - sum;
     for (int b = b0; b < b1; ++b) {
         plan[4 + b] = run;
         int L = seq_lens[b];
         L = L < 0 ? 0 : min(L, max_blocks * kBlock);
-        run += (L + tile - 1) / tile;
-    }
-    if (threadIdx.x == 1023) {
-        const int total = part[1023];
-        plan[4 + B] = total;
-        plan[1] = total;
-        plan[2] = ranges;
-        plan[0] = total > 0 ? (total + ranges - 1) / ranges : 1;
+        const int e = run + (L + tile - 1) / tile;
+        // ranges whose first tile lies in [run, e)
+        for (int r = (run + q - 1) / q; r < ranges && r * q < e; ++r) plan[5 + B + r] = b;
+        run = e;
     }
 }
 

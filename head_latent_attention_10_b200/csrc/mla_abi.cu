@@ -212,7 +212,7 @@ TcWs tc_ws(int H, int s, int B)
     const int groups = dec_groups(H, s);
     const int ranges = kMaxRanges / groups > 0 ? kMaxRanges / groups : 1;
     w.off_plan = kWsAlign;
-    w.off_o = align_up(w.off_plan + (size_t)(4 + B + 1) * sizeof(int32_t), kWsAlign);
+    w.off_o = align_up(w.off_plan + (size_t)(kPlanInts + B) * sizeof(int32_t), kWsAlign);
     const size_t slots = 2 * (size_t)ranges * s * H;
     w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
     w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);

@@ -85,7 +85,11 @@ constexpr int kD64Stage = 9 * kD64Chunk;          // 73728
 constexpr int kD64OffStage = 0;
 constexpr int kD64OffBar = kD64OffStage + kD64Stages * kD64Stage;  // 221184
 constexpr int kD64PChunk = 8 * kD64Chunk;         // P of a tile goes where its RoPE chunk was
-constexpr int kD64Smem = kD64OffBar + 512 + 1024;                // + alignment slack
+// epilogue staging: per softmax warp 16 rows of kD64EpiRow bytes, so that the
+// output rows leave in whole 128-byte lines (FP8 kernel: 64-byte rows)
+constexpr int kD64EpiRow = 128, kD64EpiRowFp8 = 64;
+constexpr int kD64OffEpi = kD64OffBar + 512;
+constexpr int kD64Smem = kD64OffEpi + 4 * 16 * kD64EpiRow + 1024;  // + alignment slack
 constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-511
 constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
 constexpr uint32_t kD64TmS2 = 416;                // third logits buffer: lanes 0-15, columns 416-479
@@ -100,7 +104,8 @@ constexpr int kD64F8Box = kT64 * 64;              // one 64-column box of codes 
 constexpr int kD64OffScale = kD64Stages * kD64Stage;              // [3][64][2] fp32
 constexpr int kD64OffSmax = kD64OffScale + kD64Stages * 512;      // [3][64] fp32
 constexpr int kD64OffBarFp8 = kD64OffSmax + kD64Stages * 256;
-constexpr int kD64SmemFp8 = kD64OffBarFp8 + 512 + 1024;
+constexpr int kD64OffEpiFp8 = kD64OffBarFp8 + 512;
+constexpr int kD64SmemFp8 = kD64OffEpiFp8 + 4 * 16 * kD64EpiRowFp8 + 1024;
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kFp8 ? kD64ThreadsFp8 : kD64Threads, 1)
@@ -132,6 +137,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     const int q_per = a.plan[0], total = a.plan[1];
     const int lo = rng * q_per, hi = min(lo + q_per, total);
     if (lo >= hi) return;
+    const int seq0 = a.plan[5 + a.B + rng];   // the sequence holding tile lo
     const int rows_per_seq = a.s * a.H;
 
     if (threadIdx.x == 0) {
@@ -174,15 +180,21 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             TileIter it, ahead;
-            it.init(seq_start, a.B, lo, hi);
+            it.init(seq_start, a.B, lo, hi, seq0);
             ahead = it;
             for (int i = 0; i < kD64Ahead && ahead.ok; ++i) ahead.advance();
-            int issued_k = 0;
-            bool ok = true;
-            while (ok && it.ok) {
-                const int k = it.k, st = k % kD64Stages;
+            // warm L2 with the page kD64Ahead tiles further on (and, when that tile
+            // starts a segment, with the segment's Q rows, which the softmax warps
+            // read at the switch: 64 rows of 1152 B at most); issued after each
+            // page load, so the first loads of the range go out first
+            auto prefetch_ahead = [&]() {
                 if (ahead.ok) {
-                    // warm L2 with a tile further ahead while this stage waits to be freed
+                    if (ahead.first() && ahead.seg > 0) {
+                        const int r0 = group * kGroupRows, nr = min(kGroupRows, rows_per_seq - r0);
+                        const char *q0 = reinterpret_cast<const char *>(a.q_abs + ((long long)ahead.seq * rows_per_seq + r0) * kRow);
+                        for (int r = 0; r < nr; r += 8)
+                            sm100::bulk_prefetch_l2(q0 + (long long)r * kRow * 2, min(8, nr - r) * kRow * 2);
+                    }
                     const int pb = page_of(ahead);
                     if (pb >= 0) {
                         for (int j = 0; j < 9; ++j) sm100::tma_prefetch_3d(&map_kv, 64 * j, pb * kBlock, 0);
@@ -192,6 +204,11 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                     }
                     ahead.advance();
                 }
+            };
+            int issued_k = 0;
+            bool ok = true;
+            while (ok && it.ok) {
+                const int k = it.k, st = k % kD64Stages;
                 if (k >= kD64Stages)
                     ok = sm100::mbar_wait(&kv_empty[st], ((k / kD64Stages) - 1) & 1, abort_flag, a.err, lim);
                 if (!ok) break;
@@ -206,6 +223,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 if (k == a.stall_tile) {
                     // test hook for failure detection: this page never arrives, so the
                     // first wait on it runs out and the CTA unwinds
+                    prefetch_ahead();
                     it.advance();
                     continue;
                 }
@@ -225,6 +243,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                            blk * kBlock, 0);
                 }
                 issued_k = k + 1;
+                prefetch_ahead();
                 it.advance();
             }
             if (*abort_flag) {  // wait for the copies still in flight
@@ -245,7 +264,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         const uint32_t scol = b < 2 ? 64u * b : kD64TmS2;
         const uint32_t idesc_s = kFp8 ? sm100::idesc_f16(kGroupRows, kT64, 0, 0) : sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
-        is.init(seq_start, a.B, lo, hi);
+        is.init(seq_start, a.B, lo, hi, seq0);
         int q_seg = -1;
         bool ok = true;
         while (ok && is.ok) {
@@ -294,7 +313,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ct % 4 of each 64-column chunk (a warp reads 512 contiguous bytes)
         const int ct = threadIdx.x - kD64Threads, g = ct & 3;
         TileIter it;
-        it.init(seq_start, a.B, lo, hi);
+        it.init(seq_start, a.B, lo, hi, seq0);
         bool ok = true;
         while (ok && it.ok) {
             const int k = it.k, st = k % kD64Stages;
@@ -394,29 +413,27 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         auto write_q = [&](int seq) {
             const uint4 *q4 = reinterpret_cast<const uint4 *>(
                 a.q_abs + ((long long)seq * rows_per_seq + (row_ok ? grow_row : 0)) * kRow) + (srow ? 0 : 4);
+            // all 36 loads in flight at once (one memory latency per switch)
+            uint4 v[36];
 #pragma unroll
-            for (int g = 0; g < 3; ++g) {  // 3 rounds of 3 blocks, loads batched per round
-                uint4 v[12];
+            for (int e = 0; e < 36; ++e)
+                v[e] = row_ok ? __ldg(q4 + 8 * (e >> 2) + (e & 3)) : make_uint4(0, 0, 0, 0);
+            if constexpr (kFp8) {
+                // the FP8 path's MMAs take f16 operands
 #pragma unroll
-                for (int e = 0; e < 12; ++e)
-                    v[e] = row_ok ? __ldg(q4 + 8 * (3 * g + (e >> 2)) + (e & 3)) : make_uint4(0, 0, 0, 0);
-                if constexpr (kFp8) {
-                    // the FP8 path's MMAs take f16 operands
+                for (int e = 0; e < 36; ++e) {
+                    uint32_t *w = reinterpret_cast<uint32_t *>(&v[e]);
 #pragma unroll
-                    for (int e = 0; e < 12; ++e) {
-                        uint32_t *w = reinterpret_cast<uint32_t *>(&v[e]);
-#pragma unroll
-                        for (int f = 0; f < 4; ++f) {
-                            const __half2 hh = __float22half2_rn(
-                                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[f])));
-                            w[f] = *reinterpret_cast<const uint32_t *>(&hh);
-                        }
+                    for (int f = 0; f < 4; ++f) {
+                        const __half2 hh = __float22half2_rn(
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[f])));
+                        w[f] = *reinterpret_cast<const uint32_t *>(&hh);
                     }
                 }
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    sm100::tmem_st16x2_16(lane_base + kD64TmQ + 32 * (3 * g + j), reinterpret_cast<const uint32_t *>(v + 4 * j));
             }
+#pragma unroll
+            for (int j = 0; j < 9; ++j)
+                sm100::tmem_st16x2_16(lane_base + kD64TmQ + 32 * j, reinterpret_cast<const uint32_t *>(v + 4 * j));
             sm100::tmem_wait_st();
             sm100::tc_fence_before();
             __syncwarp();
@@ -425,19 +442,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 atomicAdd(const_cast<int *>(q_cnt), 1);
             }
         };
-        // warm L2 with the row of the sequence a range moves on to, a few
-        // tiles before the switch (earlier, the streaming cache pages would
-        // evict it again): the row's nine 128-byte lines, five by thread i,
-        // four by thread 16+i
-        auto prefetch_q = [&](int seq) {
-            if (!row_ok || seq >= a.B) return;
-            const char *nq = reinterpret_cast<const char *>(a.q_abs + ((long long)seq * rows_per_seq + grow_row) * kRow);
-#pragma unroll
-            for (int e = 0; e < 5; ++e)
-                if (srow || e < 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * (srow ? e : 5 + e)));
-        };
         TileIter it;
-        it.init(seq_start, a.B, lo, hi);
+        it.init(seq_start, a.B, lo, hi, seq0);
         float m_run = -INFINITY, l_run = 0.f;
         int nvis = 0, nseq = 0;
         const uint32_t idesc_o = kFp8 ? sm100::idesc_f16(kGroupRows, 256, 0, 1) : sm100::idesc_bf16(kGroupRows, 256, 0, 1);
@@ -445,7 +451,6 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         if (it.ok) write_q(it.seq);
         while (ok && it.ok) {
             const int k = it.k;
-            if (it.tt + 4 == it.t1 || (it.first() && it.t1 - it.t0 < 4)) prefetch_q(it.seq + 1);
             if (it.first()) {
                 m_run = -INFINITY;
                 l_run = 0.f;
@@ -608,28 +613,76 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 const float lse2 = l_tot > 0.f ? m_fin + __log2f(l_tot) : -INFINITY;
                 const long long orow = (long long)(it.seq * a.s + tq) * a.H + head;
                 const long long slot = 2LL * rng + (it.seg == 0 ? 0 : 1);
-                const int hc = srow ? 0 : 32;
-                for (int c = 0; c < 512; c += 64) {
-                    uint32_t ov[32];
-                    sm100::tmem_ld16x2_32(o_base + c, ov);
-                    sm100::tmem_wait_ld();
-                    if (!row_ok) continue;
-                    if (it.complete) {
-                        uint4 *d = reinterpret_cast<uint4 *>(a.out + orow * kDc + c + hc);
+                // O row r leaves through the warp's staging rows: per 64-column
+                // block, thread i / 16+i put their halves of row r in shared
+                // memory (16-byte chunks XOR-swizzled by row), then each store
+                // instruction of the warp writes whole rows of the block
+                constexpr int RB = kFp8 ? kD64EpiRowFp8 : kD64EpiRow;
+                constexpr int CPR = RB / 16;
+                const uint32_t stg = sm100::smem_u32(smem + (kFp8 ? kD64OffEpiFp8 : kD64OffEpi)) + qd * 16 * RB;
+                const int lr_me = lane & 15, hh = srow ? 0 : 1;
+                auto swz = [](int row) { return (row * RB / 128) & (CPR - 1); };
+                auto drain = [&](auto f32_tag) {
+                    constexpr bool F32 = decltype(f32_tag)::value;
+                    constexpr int EB = F32 ? 4 : 2;          // output element bytes
+                    constexpr int HB = 32 * EB;              // a thread's half of a row's block
+                    constexpr int NR = 2 * HB / RB;          // staging rounds per block
+                    char *base = F32 ? reinterpret_cast<char *>(a.part_o + slot * rows_per_seq * kDc)
+                                     : reinterpret_cast<char *>(a.out + (long long)it.seq * rows_per_seq * kDc);
+                    for (int c = 0; c < 512; c += 64) {
+                        uint32_t ov[32];
+                        sm100::tmem_ld16x2_32(o_base + c, ov);
+                        sm100::tmem_wait_ld();
+                        uint4 pk[HB / 16];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            d[e] = make_uint4(pack_bf162(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
-                                              pack_bf162(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
-                                              pack_bf162(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
-                                              pack_bf162(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
-                    } else {
-                        float4 *d4 = reinterpret_cast<float4 *>(a.part_o + (slot * rows_per_seq + grow_row) * kDc + c + hc);
+                        for (int j = 0; j < HB / 16; ++j) {
+                            if constexpr (F32) {
+                                pk[j] = make_uint4(__float_as_uint(__uint_as_float(ov[4 * j]) * inv),
+                                                   __float_as_uint(__uint_as_float(ov[4 * j + 1]) * inv),
+                                                   __float_as_uint(__uint_as_float(ov[4 * j + 2]) * inv),
+                                                   __float_as_uint(__uint_as_float(ov[4 * j + 3]) * inv));
+                            } else {
+                                pk[j] = make_uint4(pack_bf162(__uint_as_float(ov[8 * j]) * inv, __uint_as_float(ov[8 * j + 1]) * inv),
+                                                   pack_bf162(__uint_as_float(ov[8 * j + 2]) * inv, __uint_as_float(ov[8 * j + 3]) * inv),
+                                                   pack_bf162(__uint_as_float(ov[8 * j + 4]) * inv, __uint_as_float(ov[8 * j + 5]) * inv),
+                                                   pack_bf162(__uint_as_float(ov[8 * j + 6]) * inv, __uint_as_float(ov[8 * j + 7]) * inv));
+                            }
+                        }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                                __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+                        for (int q = 0; q < NR; ++q) {
+                            // round q stages bytes [q RB, (q+1) RB) of the 16 rows' block
+                            if constexpr (RB >= HB) {
+                                if ((hh * HB) / RB == q) {
+                                    const int c0 = (hh * HB - q * RB) >> 4;
+#pragma unroll
+                                    for (int j = 0; j < HB / 16; ++j)
+                                        st_shared_v4(stg + lr_me * RB + (((c0 + j) ^ swz(lr_me)) << 4), pk[j]);
+                                }
+                            } else {
+                                constexpr int W = HB / RB;   // rounds per half
+                                if (q / W == hh) {
+#pragma unroll
+                                    for (int j = 0; j < CPR; ++j)
+                                        st_shared_v4(stg + lr_me * RB + ((j ^ swz(lr_me)) << 4), pk[(q % W) * CPR + j]);
+                                }
+                            }
+                            __syncwarp();
+#pragma unroll
+                            for (int e = 0; e < RB / 32; ++e) {
+                                const int f = e * 32 + lane, lr = f / CPR, ch = f % CPR;
+                                const uint4 v = ld_shared_v4(stg + lr * RB + ((ch ^ swz(lr)) << 4));
+                                const int grow = group * kGroupRows + 16 * qd + lr;
+                                if (grow < rows_per_seq)
+                                    *reinterpret_cast<uint4 *>(base + ((long long)grow * kDc + c) * EB + q * RB + 16 * ch) = v;
+                            }
+                            __syncwarp();
+                        }
                     }
-                }
+                };
+                if (it.complete)
+                    drain(std::false_type{});
+                else
+                    drain(std::true_type{});
                 if (row_ok && srow) {
                     if (it.complete) {
                         if (a.out_lse) a.out_lse[orow] = lse2 * kLn2;

@@ -96,3 +96,39 @@ def test_combine_rows_bound_at_sixteen_rows():
     assert max(r for _, r in rows_seen) == 15
     # the empty sequence's rows are zeroed (written) though it has no partial
     assert {(3, r) for r in range(16)} <= rows_seen
+
+
+def range_starts(start, q, ranges, B):
+    """dec_plan_kernel's per-range table: sequence b writes its index for the
+    ranges r with r*q in [start[b], start[b+1])."""
+    table = {}
+    for b in range(B):
+        run, e = int(start[b]), int(start[b + 1])
+        r = (run + q - 1) // q
+        while r < ranges and r * q < e:
+            assert r not in table          # one writer per range
+            table[r] = b
+            r += 1
+    return table
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("ranges", [1, 3, 74, 148])
+def test_range_start_table_matches_the_search(seed, ranges):
+    """Each range's first sequence (written by the plan kernel in place of a
+    binary search in every decode warp) is the largest b with start[b] <= lo,
+    empty sequences included, and every range with work gets one."""
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 300))
+    sl = rng.integers(0, 3000, size=B).astype(np.int32)
+    sl[rng.random(B) < 0.2] = 0
+    q, total, start = plan(sl, 1, 64, ranges)
+    table = range_starts(start, q, ranges, B)
+    for r in range(ranges):
+        lo = r * q
+        if lo >= total:
+            assert r not in table
+            continue
+        want = int(np.nonzero(start <= lo)[0].max())   # largest index with start <= lo
+        assert table[r] == want and start[want] <= lo < start[want + 1]
+    assert 5 + 148 + B >= 5 + B + ranges              # kPlanInts + B ints hold the table
