@@ -17,8 +17,8 @@ struct DecArgs {
     const bf16 *q_abs;    // [B*s][H][576]
     const int32_t *block_table;
     const int32_t *seq_lens;
-    const int32_t *plan;  // [0]=tiles per range, [1]=total tiles, [2]=ranges, [4..4+B] sequence tile starts,
-                          // [5+B+r] first sequence of range r
+    int32_t *plan;        // written by CTA 0 for the combine: [0]=tiles per range, [1]=total tiles,
+                          // [2]=ranges, [4..4+B] sequence tile starts
     bf16 *out;
     float *out_lse;
     float *part_o;        // [2*ranges][s*H][512] fp32
@@ -44,29 +44,42 @@ __device__ __forceinline__ int seq_len_clamped(const int32_t *seq_lens, int b, i
     return L < 0 ? 0 : min(L, max_blocks * kBlock);
 }
 
-// Walks a range of the (sequence, tile) list one tile at a time.
+// Walks a range of the (sequence, tile) list one tile at a time.  Sequence
+// r holds tiles [a_r, a_r + ceil(L_r / 64)); the walk starts in sequence r0,
+// whose first tile a0 the range's plan gives, and takes the later starts from
+// the sequence lengths.
 struct TileIter {
-    const int32_t *rs;
-    int n, pos, hi, r;
+    const int32_t *sl;
+    int max_tok, n, pos, hi, r, ar;
     int seq, t0, t1, seg, tt, k;
     bool complete, ok;
+    __device__ int tiles(int b) const
+    {
+        int L = sl[b];
+        L = L < 0 ? 0 : min(L, max_tok);
+        return (L + kBlock - 1) / kBlock;
+    }
     __device__ bool next_seg()
     {
-        while (pos < hi && r < n && rs[r + 1] <= pos) ++r;
-        if (pos >= hi || r >= n) return false;
-        const int a = rs[r], e = rs[r + 1];
+        if (pos >= hi) return false;
+        int e;
+        for (;;) {
+            if (r >= n) return false;
+            e = ar + tiles(r);
+            if (e > pos) break;
+            ar = e;   // an empty sequence, or one that ends before pos
+            ++r;
+        }
         const int end = min(hi, e);
-        seq = r; t0 = pos - a; t1 = end - a;
-        complete = (pos == a) && (end == e);
-        pos = end; ++r; ++seg;
+        seq = r; t0 = pos - ar; t1 = end - ar;
+        complete = (pos == ar) && (end == e);
+        pos = end; ar = e; ++r; ++seg;
         return true;
     }
-    // r0: the sequence holding tile lo (find_seq(start, n, lo)), which the
-    // plan kernel stores for every range
-    __device__ void init(const int32_t *start, int n_, int lo, int hi_, int r0)
+    __device__ void init(const int32_t *seq_lens, int max_blocks, int n_, int lo, int hi_, int r0, int a0)
     {
-        rs = start; n = n_; pos = lo; hi = hi_; seg = -1; k = 0;
-        r = r0;
+        sl = seq_lens; max_tok = max_blocks * kBlock; n = n_; pos = lo; hi = hi_; seg = -1; k = 0;
+        r = r0; ar = a0;
         ok = next_seg();
         tt = t0;
     }
@@ -130,61 +143,61 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 }
 
 // -------------------------------------------------------------------- plan
-// One CTA: `tile`-token tiles of every sequence (its last query sees all L
-// tokens), their prefix sums, the per-range quota, and the sequence each range
-// starts in (so that no decode warp searches the prefix sums at its start).
-// plan[0] = tiles per range, plan[1] = total tiles, plan[2] = ranges,
-// plan[4 + b] = first tile of sequence b (b = 0..B),
-// plan[5 + B + r] = sequence holding tile r * plan[0] (ranges r that start
-// before the end of the list).
-constexpr int kPlanInts = 5 + kMaxRanges;   // + B: ints of the plan
-__global__ void __launch_bounds__(1024)
-dec_plan_kernel(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int tile,
-                int32_t *__restrict__ plan, uint32_t *err)
+// One warp of every decode CTA: the CTA's range of the batch's (sequence,
+// tile) list.  The list holds the ceil(L_b / 64) tiles of every sequence b
+// (its last query sees all L_b tokens) in sequence order; `ranges` contiguous
+// ranges of ceil(total / ranges) tiles cover it.  Lane l takes sequences
+// [l per, (l+1) per); a shuffle scan gives the prefix sums.
+// out = {tiles per range, total tiles, the sequence holding tile rng * quota,
+// that sequence's first tile} (the last two only when rng * quota < total).
+// With `publish` (CTA 0 of the grid), the warp also stores the plan the
+// combine kernel reads (plan[0] = quota, plan[1] = total, plan[2] = ranges,
+// plan[4 + b] = first tile of sequence b, b = 0..B) and flags invalid lengths.
+__device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int rng,
+                           bool publish, int32_t *plan, uint32_t *err, int *out)
 {
-    __shared__ int part[1024];
-    __shared__ int quota;
-    sm100::pdl_trigger();   // the decode kernel may set itself up meanwhile
-    const int per = (B + 1023) / 1024;
-    const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
+    const int lane = threadIdx.x & 31;
+    const int max_tok = max_blocks * kBlock;
+    const int per = (B + 31) / 32;
+    const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
     int sum = 0;
     for (int b = b0; b < b1; ++b) {
         int L = seq_lens[b];
-        if (L < 0 || L > max_blocks * kBlock) {
-            set_error(err, MLA_DEVERR_SEQ_LEN);
-            L = L < 0 ? 0 : max_blocks * kBlock;
-        }
-        if (L < s) set_error(err, MLA_DEVERR_SEQ_LEN);  // some query sees no key
-        sum += (L + tile - 1) / tile;
+        // out of range, or some query sees no key
+        if (publish && (L < 0 || L > max_tok || L < s)) set_error(err, MLA_DEVERR_SEQ_LEN);
+        L = L < 0 ? 0 : min(L, max_tok);
+        sum += (L + kBlock - 1) / kBlock;
     }
-    part[threadIdx.x] = sum;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-        const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
-        __syncthreads();
-        part[threadIdx.x] += v;
-        __syncthreads();
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
     }
-    if (threadIdx.x == 1023) {
-        const int total = part[1023];
-        const int q = total > 0 ? (total + ranges - 1) / ranges : 1;
-        plan[4 + B] = total;
-        plan[1] = total;
-        plan[2] = ranges;
-        plan[0] = q;
-        quota = q;
-    }
-    __syncthreads();
-    const int q = quota;
-    int run = part[threadIdx.x] - sum;
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    const int q = total > 0 ? (total + ranges - 1) / ranges : 1;
+    const int lo = rng * q;
+    int run = inc - sum;
     for (int b = b0; b < b1; ++b) {
-        plan[4 + b] = run;
         int L = seq_lens[b];
-        L = L < 0 ? 0 : min(L, max_blocks * kBlock);
-        const int e = run + (L + tile - 1) / tile;
-        // ranges whose first tile lies in [run, e)
-        for (int r = (run + q - 1) / q; r < ranges && r * q < e; ++r) plan[5 + B + r] = b;
-        run = e;
+        L = L < 0 ? 0 : min(L, max_tok);
+        const int t = (L + kBlock - 1) / kBlock;
+        if (publish) plan[4 + b] = run;
+        if (run <= lo && lo < run + t) {
+            out[2] = b;
+            out[3] = run;
+        }
+        run += t;
+    }
+    if (lane == 0) {
+        out[0] = q;
+        out[1] = total;
+        if (publish) {
+            plan[0] = q;
+            plan[1] = total;
+            plan[2] = ranges;
+            plan[4 + B] = total;
+        }
     }
 }
 

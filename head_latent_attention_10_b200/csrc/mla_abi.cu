@@ -212,7 +212,7 @@ TcWs tc_ws(int H, int s, int B)
     const int groups = dec_groups(H, s);
     const int ranges = kMaxRanges / groups > 0 ? kMaxRanges / groups : 1;
     w.off_plan = kWsAlign;
-    w.off_o = align_up(w.off_plan + (size_t)(kPlanInts + B) * sizeof(int32_t), kWsAlign);
+    w.off_o = align_up(w.off_plan + (size_t)(4 + B + 1) * sizeof(int32_t), kWsAlign);
     const size_t slots = 2 * (size_t)ranges * s * H;
     w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
     w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
@@ -293,9 +293,6 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     }
     if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
     int32_t *plan = (int32_t *)(ws + w.off_plan);
-    dec_plan_kernel<<<1, 1024, 0, strm>>>(seq_lens, B, s, max_blocks, ranges, kT64, plan, err);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     DecArgs da;
     da.q_abs = (const bf16 *)q_abs;
     da.block_table = block_table;
@@ -316,8 +313,8 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     da.H = H;
     da.B = B;
     da.groups = groups;
-    // the decode kernel sets itself up while the plan runs, and the
-    // combine launches while the decode's last CTAs finish
+    // the decode kernel sets itself up while the kernel before it ends, and
+    // the combine launches while the decode's last CTAs finish
     cudaError_t e = launch_pdl(tc_decode64_kernel<kFp8>, dim3(ranges * groups),
                                dim3(kFp8 ? kD64ThreadsFp8 : kD64Threads), kFp8 ? kD64SmemFp8 : kD64Smem, strm, mkv,
                                da);

@@ -50,7 +50,7 @@
 // only when the running max grows by more than 8, a factor 256).
 //
 // Work split: the (sequence, tile) list of the batch is cut into equal
-// contiguous ranges per row group (dec_plan_kernel).  A sequence a range covers
+// contiguous ranges per row group (plan_range, one warp of every CTA).  A sequence a range covers
 // completely is normalized and written straight to the output.  A sequence cut
 // by range ends leaves one fp32 partial per piece (normalized, with its
 // log2-sum-exp), merged by dec_combine_kernel.  Every wait is bounded; a wait
@@ -130,14 +130,10 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
 
+    int *rplan = reinterpret_cast<int *>(bars + 40);   // this CTA's range (plan_range's out)
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = blockIdx.x % a.groups, rng = blockIdx.x / a.groups;
-    sm100::pdl_wait();  // the plan is complete
-    const int32_t *seq_start = a.plan + 4;
-    const int q_per = a.plan[0], total = a.plan[1];
-    const int lo = rng * q_per, hi = min(lo + q_per, total);
-    if (lo >= hi) return;
-    const int seq0 = a.plan[5 + a.B + rng];   // the sequence holding tile lo
     const int rows_per_seq = a.s * a.H;
 
     if (threadIdx.x == 0) {
@@ -163,10 +159,22 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         sm100::tmem_alloc(tmem_slot, 512);
         sm100::tmem_relinquish();
     }
+    // the sequence lengths and queries may come from the kernel before this one
+    sm100::pdl_wait();
+    if (warp == 2)
+        plan_range(a.seq_lens, a.B, a.s, a.max_blocks, gridDim.x / a.groups, rng, blockIdx.x == 0, a.plan, a.err,
+                   rplan);
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int q_per = rplan[0], total = rplan[1];
+    const int lo = rng * q_per, hi = min(lo + q_per, total);
+    if (lo >= hi) {   // no tile for this CTA
+        if (warp == 1) sm100::tmem_dealloc(tmem, 512);
+        return;
+    }
+    const int seq0 = rplan[2], start0 = rplan[3];   // the sequence holding tile lo, its first tile
     const unsigned long long lim = a.limit_ns;
     const unsigned long long drain = lim > 200000000ull ? lim : 200000000ull;
     uint8_t *stages = smem + kD64OffStage;
@@ -180,7 +188,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             TileIter it, ahead;
-            it.init(seq_start, a.B, lo, hi, seq0);
+            it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
             ahead = it;
             for (int i = 0; i < kD64Ahead && ahead.ok; ++i) ahead.advance();
             // warm L2 with the page kD64Ahead tiles further on (and, when that tile
@@ -264,7 +272,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         const uint32_t scol = b < 2 ? 64u * b : kD64TmS2;
         const uint32_t idesc_s = kFp8 ? sm100::idesc_f16(kGroupRows, kT64, 0, 0) : sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
-        is.init(seq_start, a.B, lo, hi, seq0);
+        is.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
         int q_seg = -1;
         bool ok = true;
         while (ok && is.ok) {
@@ -313,7 +321,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ct % 4 of each 64-column chunk (a warp reads 512 contiguous bytes)
         const int ct = threadIdx.x - kD64Threads, g = ct & 3;
         TileIter it;
-        it.init(seq_start, a.B, lo, hi, seq0);
+        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
         bool ok = true;
         while (ok && it.ok) {
             const int k = it.k, st = k % kD64Stages;
@@ -443,7 +451,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             }
         };
         TileIter it;
-        it.init(seq_start, a.B, lo, hi, seq0);
+        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
         float m_run = -INFINITY, l_run = 0.f;
         int nvis = 0, nseq = 0;
         const uint32_t idesc_o = kFp8 ? sm100::idesc_f16(kGroupRows, 256, 0, 1) : sm100::idesc_bf16(kGroupRows, 256, 0, 1);

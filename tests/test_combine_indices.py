@@ -2,7 +2,7 @@
 the CPU for every workload (s*H from 16 to 256) and several SM counts: every
 partial slot the combine reads lies inside the workspace's partial area,
 every row it forms is below s*H, every output element it writes lies inside
-the output, and every row of every cut sequence is written once.  The emulation restates the loops of dec_plan_kernel and
+the output, and every row of every cut sequence is written once.  The emulation restates the loops of plan_range and
 dec_combine_kernel (csrc/dec_common.cuh) index for index; the GPU tests then
 check the values."""
 import numpy as np
@@ -98,37 +98,42 @@ def test_combine_rows_bound_at_sixteen_rows():
     assert {(3, r) for r in range(16)} <= rows_seen
 
 
-def range_starts(start, q, ranges, B):
-    """dec_plan_kernel's per-range table: sequence b writes its index for the
-    ranges r with r*q in [start[b], start[b+1])."""
-    table = {}
-    for b in range(B):
-        run, e = int(start[b]), int(start[b + 1])
-        r = (run + q - 1) // q
-        while r < ranges and r * q < e:
-            assert r not in table          # one writer per range
-            table[r] = b
-            r += 1
-    return table
+def range_start(seq_lens, ranges, rng, max_blocks=64, lanes=32):
+    """plan_range for one CTA: lane l sums the tiles of sequences
+    [l per, (l+1) per), a scan over lanes gives each lane's first tile, and
+    the lane whose chunk holds tile rng*q names the sequence and its start."""
+    B = len(seq_lens)
+    per = (B + lanes - 1) // lanes
+    tiles = [(min(max(int(L), 0), max_blocks * 64) + 63) // 64 for L in seq_lens]
+    sums = [sum(tiles[min(B, l * per):min(B, l * per + per)]) for l in range(lanes)]
+    total = sum(sums)
+    q = (total + ranges - 1) // ranges if total > 0 else 1
+    lo, found, run = rng * q, [], 0
+    for l in range(lanes):
+        for b in range(min(B, l * per), min(B, l * per + per)):
+            if run <= lo < run + tiles[b]:
+                found.append((b, run))
+            run += tiles[b]
+    return q, total, found
 
 
 @pytest.mark.parametrize("seed", range(6))
 @pytest.mark.parametrize("ranges", [1, 3, 74, 148])
-def test_range_start_table_matches_the_search(seed, ranges):
-    """Each range's first sequence (written by the plan kernel in place of a
-    binary search in every decode warp) is the largest b with start[b] <= lo,
-    empty sequences included, and every range with work gets one."""
+def test_range_start_matches_the_search(seed, ranges):
+    """Each CTA's first sequence (plan_range) is the largest b with
+    start[b] <= lo, empty sequences included; exactly one lane finds it when
+    the range has work, none when it has not."""
     rng = np.random.default_rng(seed)
     B = int(rng.integers(1, 300))
     sl = rng.integers(0, 3000, size=B).astype(np.int32)
     sl[rng.random(B) < 0.2] = 0
     q, total, start = plan(sl, 1, 64, ranges)
-    table = range_starts(start, q, ranges, B)
     for r in range(ranges):
+        q2, total2, found = range_start(sl, ranges, r)
+        assert (q2, total2) == (q, total)
         lo = r * q
         if lo >= total:
-            assert r not in table
+            assert found == []
             continue
         want = int(np.nonzero(start <= lo)[0].max())   # largest index with start <= lo
-        assert table[r] == want and start[want] <= lo < start[want + 1]
-    assert 5 + 148 + B >= 5 + B + ranges              # kPlanInts + B ints hold the table
+        assert found == [(want, int(start[want]))] and start[want] <= lo < start[want + 1]
