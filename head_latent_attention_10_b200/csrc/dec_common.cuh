@@ -17,8 +17,7 @@ struct DecArgs {
     const bf16 *q_abs;    // [B*s][H][576]
     const int32_t *block_table;
     const int32_t *seq_lens;
-    int32_t *plan;        // written by CTA 0 for the combine: [0]=tiles per range, [1]=total tiles,
-                          // [2]=ranges, [4..4+B] sequence tile starts
+    int32_t *plan;        // written by CTA 0 for the combine (plan_range)
     bf16 *out;
     float *out_lse;
     float *part_o;        // [2*ranges][s*H][512] fp32
@@ -123,6 +122,13 @@ __device__ __forceinline__ bool wait_count(volatile int *cnt, int target, volati
 }
 
 
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -151,8 +157,15 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 // out = {tiles per range, total tiles, the sequence holding tile rng * quota,
 // that sequence's first tile} (the last two only when rng * quota < total).
 // With `publish` (CTA 0 of the grid), the warp also stores the plan the
-// combine kernel reads (plan[0] = quota, plan[1] = total, plan[2] = ranges,
-// plan[4 + b] = first tile of sequence b, b = 0..B) and flags invalid lengths.
+// combine kernel reads and flags invalid lengths:
+//   plan[0] = quota, plan[1] = total, plan[2] = ranges,
+//   plan[4 + b] = first tile of sequence b (b = 0..B),
+//   plan[5 + B] = n, the number of sequences the combine finishes (those cut
+//   by a range end, and those with no tile), listed in sequence order as
+//   int4 {b, first tile, end tile, clamped length} from int plan_list_off(B).
+__host__ __device__ inline int plan_list_off(int B) { return (B + 9) & ~3; }   // 16-byte aligned, after plan[5 + B]
+__host__ __device__ inline int plan_ints(int B) { return plan_list_off(B) + 4 * B; }
+
 __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int rng,
                            bool publish, int32_t *plan, uint32_t *err, int *out)
 {
@@ -199,20 +212,53 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
             plan[4 + B] = total;
         }
     }
+    if (publish) {
+        // the combine's list: sequences cut by a range end, or with no tile
+        auto listed = [&](int a0, int a1) { return a1 == a0 || a0 / q != (a1 - 1) / q; };
+        int cnt = 0;
+        run = inc - sum;
+        for (int b = b0; b < b1; ++b) {
+            int L = seq_lens[b];
+            L = L < 0 ? 0 : min(L, max_tok);
+            const int e = run + (L + kBlock - 1) / kBlock;
+            cnt += listed(run, e) ? 1 : 0;
+            run = e;
+        }
+        int ci = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, ci, o);
+            if (lane >= o) ci += v;
+        }
+        int4 *list = reinterpret_cast<int4 *>(plan + plan_list_off(B));
+        int at = ci - cnt;
+        run = inc - sum;
+        for (int b = b0; b < b1; ++b) {
+            int L = seq_lens[b];
+            L = L < 0 ? 0 : min(L, max_tok);
+            const int e = run + (L + kBlock - 1) / kBlock;
+            if (listed(run, e)) list[at++] = make_int4(b, run, e, L);
+            run = e;
+        }
+        if (lane == 31) plan[5 + B] = ci;
+    }
 }
 
 
 // ------------------------------------------------------------------ combine
 // Sequences cut by range ends are merged by log-sum-exp; sequences one range
 // finished are already in place; queries with no visible key get a zero
-// latent and lse = -inf.  One warp per (sequence b, row rr < s*H), CTAs of 8
-// warps over consecutive rows; lane l owns latent columns [16l, 16l+16).  The
-// pieces of a cut sequence are the ranges c0..c1 it spans; lane i reads the
-// log2-sum-exp of piece i (and i + 32, ...), and the partial rows are read
-// four pieces at a time so that 16 loads per lane are in flight.  Every
-// partial slot lies in [2 c0, 2 c1 + 1] with c1 < ranges.
+// latent and lse = -inf.  Only the sequences plan_range lists (cut by a range
+// end, or with no tile) are visited: one warp per (listed sequence, row
+// rr < s*H), lane l owning latent columns [16l, 16l+16).  The pieces of a cut
+// sequence are the ranges c0..c1 it spans; lane i reads the log2-sum-exp of
+// piece i (pieces past 32 only enter the max), and the partial rows are read
+// two pieces at a time, the first two in the same round as the log2-sum-exps.
+// Pieces are summed in range order.  Every partial slot lies in
+// [2 c0, 2 c1 + 1] with c1 < ranges.
 constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
+constexpr int kCombineCtasPerSm = 3;   // <= 85 registers a thread: the whole grid is resident at once
 
 __host__ __device__ inline int combine_ctas(int B, int s, int H)
 {
@@ -225,22 +271,31 @@ __device__ __forceinline__ int piece_slot(int c, int c0, int a0, int q)
     return 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
 }
 
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm)
 dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
-                   const float *__restrict__ part_lse2, const int32_t *__restrict__ seq_lens, int max_blocks,
-                   int B, int s, int H, bf16 *__restrict__ out, float *__restrict__ out_lse)
+                   const float *__restrict__ part_lse2, size_t part_bytes, int B, int s, int H,
+                   bf16 *__restrict__ out, float *__restrict__ out_lse)
 {
+    if (threadIdx.x == 0) {
+        // CTAs that start while the decode's last CTAs run bring the partial
+        // area back into L2 (the pieces written early in the decode have long
+        // been evicted by the streaming pages); a hint only: the values are
+        // read after the wait below
+        const size_t per = (part_bytes / gridDim.x + 255) & ~size_t(255);
+        const size_t o0 = (size_t)blockIdx.x * per, o1 = min(part_bytes, o0 + per);
+        for (size_t o = o0; o < o1; o += 16384)
+            sm100::bulk_prefetch_l2(reinterpret_cast<const char *>(part_o) + o, (uint32_t)min((size_t)16384, o1 - o));
+    }
     sm100::pdl_wait();      // the decode kernel's partials and outputs are complete
     const int rows = s * H;
-    const long long items = (long long)B * rows;
     const int q = plan[0];
+    const int items = plan[5 + B] * rows;   // rows of the listed sequences
+    const int4 *list = reinterpret_cast<const int4 *>(plan + plan_list_off(B));
     const int lane = threadIdx.x & 31;
-    for (long long w = (long long)blockIdx.x * kCombineWarps + (threadIdx.x >> 5); w < items;
-         w += (long long)gridDim.x * kCombineWarps) {
-        const int b = (int)(w / rows), rr = (int)(w % rows);
-        const int a0 = plan[4 + b], a1 = plan[4 + b + 1];
-        int L = seq_lens[b];
-        L = L < 0 ? 0 : min(L, max_blocks * kBlock);
+    for (int w = blockIdx.x * kCombineWarps + (threadIdx.x >> 5); w < items; w += gridDim.x * kCombineWarps) {
+        const int li = w / rows, rr = w - li * rows;
+        const int4 seq = list[li];
+        const int b = seq.x, a0 = seq.y, a1 = seq.z, L = seq.w;
         const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
         const bool split = a1 > a0 && c0 != c1;
         if (!split && L >= s) continue;  // written by the decode kernel
@@ -255,40 +310,54 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
         }
         if (!split) continue;
         const int n = c1 - c0 + 1;
-        float M = -INFINITY;
-        for (int i = lane; i < n; i += 32)
-            M = fmaxf(M, part_lse2[(long long)piece_slot(c0 + i, c0, a0, q) * rows + rr]);
+        // the log2-sum-exp of piece i sits in lane i (pieces past 32 are only
+        // folded into the max), and the partial rows of the first two pieces
+        // are loaded in the same round
+        const float *pbase = part_o + (long long)rr * kDc + 16 * lane;   // + slot * rows * 512
+        const float *lbase = part_lse2 + rr;                              // + slot * rows
+        auto row_of = [&](int i) {
+            return reinterpret_cast<const float4 *>(pbase + (long long)piece_slot(c0 + i, c0, a0, q) * rows * kDc);
+        };
+        auto lse_of = [&](int i) { return lbase[(long long)piece_slot(c0 + i, c0, a0, q) * rows]; };
+        const float l2_lane = lane < n ? lse_of(lane) : -INFINITY;
+        float4 v[2][4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        for (int u = 0; u < 2; ++u)
+            if (u < n) {
+                const float4 *src = row_of(u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[u][e] = src[e];
+            }
+        float M = l2_lane;
+        for (int i = lane + 32; i < n; i += 32) M = fmaxf(M, lse_of(i));
+        M = warp_max(M);
         float acc[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         float den = 0.f;
-        for (int i0 = 0; i0 < n; i0 += 4) {
-            float4 v[4][4];
-            float wgt[4];
+        for (int i0 = 0; i0 < n; i0 += 2) {
+            if (i0 > 0) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                wgt[u] = 0.f;
-                if (i0 + u < n) {
-                    const int slot = piece_slot(c0 + i0 + u, c0, a0, q);
-                    const float l2 = part_lse2[(long long)slot * rows + rr];
-                    wgt[u] = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
-                    const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)slot * rows + rr) * kDc + 16 * lane);
+                for (int u = 0; u < 2; ++u)
+                    if (i0 + u < n) {
+                        const float4 *src = row_of(i0 + u);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) v[u][e] = src[e];
-                }
+                        for (int e = 0; e < 4; ++e) v[u][e] = src[e];
+                    }
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (i0 + u >= n) break;
-                den += wgt[u];
+            for (int u = 0; u < 2; ++u) {
+                const int i = i0 + u;
+                if (i >= n) break;
+                const float l2 = i < 32 ? __shfl_sync(0xffffffffu, l2_lane, i) : lse_of(i);
+                const float wgt = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
+                den += wgt;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    acc[4 * e] = fmaf(wgt[u], v[u][e].x, acc[4 * e]);
-                    acc[4 * e + 1] = fmaf(wgt[u], v[u][e].y, acc[4 * e + 1]);
-                    acc[4 * e + 2] = fmaf(wgt[u], v[u][e].z, acc[4 * e + 2]);
-                    acc[4 * e + 3] = fmaf(wgt[u], v[u][e].w, acc[4 * e + 3]);
+                    acc[4 * e] = fmaf(wgt, v[u][e].x, acc[4 * e]);
+                    acc[4 * e + 1] = fmaf(wgt, v[u][e].y, acc[4 * e + 1]);
+                    acc[4 * e + 2] = fmaf(wgt, v[u][e].z, acc[4 * e + 2]);
+                    acc[4 * e + 3] = fmaf(wgt, v[u][e].w, acc[4 * e + 3]);
                 }
             }
         }

@@ -15,6 +15,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include "dec_common.cuh"
 #include "k_simple.cuh"
 
 namespace mla {
@@ -33,13 +34,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes)
 {
     const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)codes, __NV_E4M3);
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-__device__ __forceinline__ float warp_max(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
 }
 
 // One warp per token: the token's bf16 row exactly as the bf16 cache writer

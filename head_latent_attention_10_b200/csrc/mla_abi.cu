@@ -212,7 +212,7 @@ TcWs tc_ws(int H, int s, int B)
     const int groups = dec_groups(H, s);
     const int ranges = kMaxRanges / groups > 0 ? kMaxRanges / groups : 1;
     w.off_plan = kWsAlign;
-    w.off_o = align_up(w.off_plan + (size_t)(4 + B + 1) * sizeof(int32_t), kWsAlign);
+    w.off_o = align_up(w.off_plan + (size_t)plan_ints(B) * sizeof(int32_t), kWsAlign);
     const size_t slots = 2 * (size_t)ranges * s * H;
     w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
     w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
@@ -321,10 +321,11 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     count_launch();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     const int ctas = combine_ctas(B, s, H);
-    const int cgrid = ctas < 8 * sm_count() ? ctas : 8 * sm_count();
+    const int cgrid = ctas < kCombineCtasPerSm * sm_count() ? ctas : kCombineCtasPerSm * sm_count();
+    const size_t part_bytes = 2 * (size_t)ranges * s * H * kDc * sizeof(float);
     e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
-                   (const float *)da.part_o, (const float *)da.part_lse2, seq_lens, max_blocks, B, s, H,
-                   (bf16 *)out_latent, out_lse);
+                   (const float *)da.part_o, (const float *)da.part_lse2, part_bytes, B, s, H, (bf16 *)out_latent,
+                   out_lse);
     count_launch();
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

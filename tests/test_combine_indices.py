@@ -34,18 +34,29 @@ def workspace_slots(s, H):
     return 2 * max(1, 148 // groups)
 
 
+def combine_list(seq_lens, max_blocks, q, start):
+    """plan_range's list: sequences cut by a range end or with no tile, as
+    (b, first tile, end tile, clamped length)."""
+    out = []
+    for b in range(len(seq_lens)):
+        a0, a1 = int(start[b]), int(start[b + 1])
+        if a1 == a0 or a0 // q != (a1 - 1) // q:
+            out.append((b, a0, a1, min(max(int(seq_lens[b]), 0), max_blocks * BLOCK)))
+    return out
+
+
 def emulate_combine(B, s, H, seq_lens, max_blocks, q, start, grid):
-    """The combine's loops: warp w of CTA blk takes rows blk*8 + w, then
-    strides by grid*8 over the B*s*H (sequence, row) items."""
+    """The combine's loops: warp w of CTA blk takes item blk*8 + w, then
+    strides by grid*8 over the (listed sequence, row) items."""
     rows = s * H
-    items = B * rows
+    lst = combine_list(seq_lens, max_blocks, q, start)
+    items = len(lst) * rows
     reads, writes, rows_seen = [], [], set()
     for blk in range(grid):
         for warp in range(COMBINE_WARPS):
             for w in range(blk * COMBINE_WARPS + warp, items, grid * COMBINE_WARPS):
-                b, rr = divmod(w, rows)
-                a0, a1 = int(start[b]), int(start[b + 1])
-                L = min(max(int(seq_lens[b]), 0), max_blocks * BLOCK)
+                li, rr = divmod(w, rows)
+                b, a0, a1, L = lst[li]
                 c0 = a0 // q if a1 > a0 else 0
                 c1 = (a1 - 1) // q if a1 > a0 else 0
                 split = a1 > a0 and c0 != c1
@@ -73,7 +84,7 @@ def test_combine_indices_stay_in_bounds(name, sms):
     ranges, groups = ranges_of(sms, cfg.s, cfg.H)
     q, total, start = plan(sl, cfg.s, max_blocks, ranges)
     assert q * ranges >= total                      # every tile lies in some range
-    grid = min((cfg.B * cfg.s * cfg.H + COMBINE_WARPS - 1) // COMBINE_WARPS, 8 * sms)
+    grid = min((cfg.B * cfg.s * cfg.H + COMBINE_WARPS - 1) // COMBINE_WARPS, 3 * sms)
     reads, writes, rows_seen = emulate_combine(cfg.B, cfg.s, cfg.H, sl, max_blocks, q, start, grid)
     rows = cfg.s * cfg.H
     nslot = workspace_slots(cfg.s, cfg.H)
@@ -84,6 +95,10 @@ def test_combine_indices_stay_in_bounds(name, sms):
     # every row of every cut sequence is written exactly by one warp of one item
     cut = [b for b in range(cfg.B) if start[b + 1] > start[b] and start[b] // q != (start[b + 1] - 1) // q]
     assert rows_seen == {(b, r) for b in cut for r in range(rows)}
+    # the list fits the plan area (plan_list_off(B) + 4 B ints) and every listed
+    # sequence is cut or empty
+    lst = combine_list(sl, max_blocks, q, start)
+    assert len(lst) <= cfg.B and ((cfg.B + 9) & ~3) % 4 == 0 and (cfg.B + 9) & ~3 >= 6 + cfg.B
 
 
 def test_combine_rows_bound_at_sixteen_rows():
