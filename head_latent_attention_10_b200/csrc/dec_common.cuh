@@ -249,21 +249,26 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
 // Sequences cut by range ends are merged by log-sum-exp; sequences one range
 // finished are already in place; queries with no visible key get a zero
 // latent and lse = -inf.  Only the sequences plan_range lists (cut by a range
-// end, or with no tile) are visited: one warp per (listed sequence, row
-// rr < s*H), lane l owning latent columns [16l, 16l+16).  The pieces of a cut
-// sequence are the ranges c0..c1 it spans; lane i reads the log2-sum-exp of
-// piece i (pieces past 32 only enter the max), and the partial rows are read
-// two pieces at a time, the first two in the same round as the log2-sum-exps.
+// end, or with no tile) are visited, in blocks of 8 rows: a CTA takes one
+// block of one listed sequence at a time.  Thread 0 copies the block's partial
+// rows into shared memory, up to 4 pieces per round (the 8 rows of a piece
+// are contiguous: one bulk copy of 16 KB), while each warp loads the
+// log2-sum-exps of its row (lane i: piece i; pieces past 32 only enter the
+// max).  Warp w then merges row 8 blk + w from shared memory, lane l owning
+// the float4 columns l, 32 + l, 64 + l and 96 + l, so that the shared-memory
+// reads are conflict-free and the output stores contiguous across the warp.
 // Pieces are summed in range order.  Every partial slot lies in
 // [2 c0, 2 c1 + 1] with c1 < ranges.
-constexpr int kCombineWarps = 8;
+constexpr int kCombineWarps = 8;                  // rows per block
 constexpr int kCombineThreads = 32 * kCombineWarps;
-constexpr int kCombineCtasPerSm = 3;   // <= 85 registers a thread: the whole grid is resident at once
+constexpr int kCombinePieces = 4;                 // pieces per bulk round
+constexpr int kCombineBuf = kCombinePieces * kCombineWarps * kDc * 4;   // 64 KB
+constexpr int kCombineSmem = kCombineBuf + 16;
+constexpr int kCombineCtasPerSm = 3;
 
-__host__ __device__ inline int combine_ctas(int B, int s, int H)
+__host__ __device__ inline int combine_blocks(int B, int s, int H)
 {
-    const long long rows = (long long)B * s * H;
-    return (int)((rows + kCombineWarps - 1) / kCombineWarps);
+    return B * ((s * H + kCombineWarps - 1) / kCombineWarps);
 }
 
 __device__ __forceinline__ int piece_slot(int c, int c0, int a0, int q)
@@ -274,8 +279,11 @@ __device__ __forceinline__ int piece_slot(int c, int c0, int a0, int q)
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm)
 dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
                    const float *__restrict__ part_lse2, size_t part_bytes, int B, int s, int H,
-                   bf16 *__restrict__ out, float *__restrict__ out_lse)
+                   bf16 *__restrict__ out, float *__restrict__ out_lse, uint32_t *err, unsigned long long limit_ns)
 {
+    extern __shared__ __align__(128) uint8_t cb_smem[];
+    const float4 *buf = reinterpret_cast<const float4 *>(cb_smem);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(cb_smem + kCombineBuf);
     if (threadIdx.x == 0) {
         // CTAs that start while the decode's last CTAs run bring the partial
         // area back into L2 (the pieces written early in the decode have long
@@ -285,88 +293,99 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
         const size_t o0 = (size_t)blockIdx.x * per, o1 = min(part_bytes, o0 + per);
         for (size_t o = o0; o < o1; o += 16384)
             sm100::bulk_prefetch_l2(reinterpret_cast<const char *>(part_o) + o, (uint32_t)min((size_t)16384, o1 - o));
+        sm100::mbar_init(bar, 1);
+        sm100::fence_mbar_init();
     }
-    sm100::pdl_wait();      // the decode kernel's partials and outputs are complete
-    const int rows = s * H;
+    __syncthreads();
+    sm100::pdl_wait();      // the decode kernel's partials, outputs and plan are complete
+    const int rows = s * H, nbr = (rows + kCombineWarps - 1) / kCombineWarps;
     const int q = plan[0];
-    const int items = plan[5 + B] * rows;   // rows of the listed sequences
+    const int nblk = plan[5 + B] * nbr;
     const int4 *list = reinterpret_cast<const int4 *>(plan + plan_list_off(B));
-    const int lane = threadIdx.x & 31;
-    for (int w = blockIdx.x * kCombineWarps + (threadIdx.x >> 5); w < items; w += gridDim.x * kCombineWarps) {
-        const int li = w / rows, rr = w - li * rows;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int no_abort = 0;
+    uint32_t phase = 0;
+    for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+        const int li = blk / nbr, rb = blk - li * nbr;
         const int4 seq = list[li];
         const int b = seq.x, a0 = seq.y, a1 = seq.z, L = seq.w;
         const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
         const bool split = a1 > a0 && c0 != c1;
-        if (!split && L >= s) continue;  // written by the decode kernel
-        const int t = rr / H;
+        const int rr0 = rb * kCombineWarps, nr = min(kCombineWarps, rows - rr0);
+        const int rr = rr0 + warp;
+        const bool row_ok = warp < nr;
+        const bool visible = L - s + rr / H + 1 > 0;   // query rr / H sees some key
         const long long orow = (long long)b * rows + rr;
-        uint4 *dst = reinterpret_cast<uint4 *>(out + orow * kDc + 16 * lane);
-        if (L - s + t + 1 <= 0) {
-            dst[0] = make_uint4(0, 0, 0, 0);
-            dst[1] = make_uint4(0, 0, 0, 0);
-            if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
-            continue;
-        }
-        if (!split) continue;
-        const int n = c1 - c0 + 1;
-        // the log2-sum-exp of piece i sits in lane i (pieces past 32 are only
-        // folded into the max), and the partial rows of the first two pieces
-        // are loaded in the same round
-        const float *pbase = part_o + (long long)rr * kDc + 16 * lane;   // + slot * rows * 512
-        const float *lbase = part_lse2 + rr;                              // + slot * rows
-        auto row_of = [&](int i) {
-            return reinterpret_cast<const float4 *>(pbase + (long long)piece_slot(c0 + i, c0, a0, q) * rows * kDc);
-        };
-        auto lse_of = [&](int i) { return lbase[(long long)piece_slot(c0 + i, c0, a0, q) * rows]; };
-        const float l2_lane = lane < n ? lse_of(lane) : -INFINITY;
-        float4 v[2][4];
+        uint2 *dst = reinterpret_cast<uint2 *>(out + orow * kDc) + lane;   // + 32 e: columns 4 (32 e + lane) ..
+        if (!split) {
+            // a sequence with no tile: every query row is zero
+            if (row_ok && !visible) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-            if (u < n) {
-                const float4 *src = row_of(u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) v[u][e] = src[e];
+                for (int e = 0; e < 4; ++e) dst[32 * e] = make_uint2(0, 0);
+                if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
             }
+            continue;   // uniform: the whole block belongs to one sequence
+        }
+        const int n = c1 - c0 + 1;
+        auto lse_of = [&](int i) { return part_lse2[(long long)piece_slot(c0 + i, c0, a0, q) * rows + rr]; };
+        const bool merge = row_ok && visible;
+        const float l2_lane = (merge && lane < n) ? lse_of(lane) : -INFINITY;
         float M = l2_lane;
-        for (int i = lane + 32; i < n; i += 32) M = fmaxf(M, lse_of(i));
+        if (merge)
+            for (int i = lane + 32; i < n; i += 32) M = fmaxf(M, lse_of(i));
         M = warp_max(M);
         float acc[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         float den = 0.f;
-        for (int i0 = 0; i0 < n; i0 += 2) {
-            if (i0 > 0) {
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    if (i0 + u < n) {
-                        const float4 *src = row_of(i0 + u);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) v[u][e] = src[e];
-                    }
+        for (int i0 = 0; i0 < n; i0 += kCombinePieces) {
+            const int np = min(kCombinePieces, n - i0);
+            __syncthreads();   // every warp is done with the previous round's rows
+            if (threadIdx.x == 0) {
+                sm100::mbar_arrive_expect_tx(bar, (uint32_t)(np * nr * kDc * 4));
+                for (int u = 0; u < np; ++u)
+                    sm100::bulk_load(cb_smem + u * (kCombineWarps * kDc * 4),
+                                     part_o + ((long long)piece_slot(c0 + i0 + u, c0, a0, q) * rows + rr0) * kDc,
+                                     (uint32_t)(nr * kDc * 4), bar);
             }
+            bool ok = sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns);
+            if (!__syncthreads_and(ok)) {
+                // a copy that never lands: let the copies in flight finish
+                // before the CTA leaves, and give up
+                sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns > 200000000ull ? limit_ns : 200000000ull);
+                return;
+            }
+            phase ^= 1;
+            if (merge) {
+                for (int u = 0; u < np; ++u) {
+                    const int i = i0 + u;
+                    const float l2 = i < 32 ? __shfl_sync(0xffffffffu, l2_lane, i) : lse_of(i);
+                    const float wgt = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
+                    den += wgt;
+                    const float4 *row = buf + (u * kCombineWarps + warp) * (kDc / 4) + lane;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int i = i0 + u;
-                if (i >= n) break;
-                const float l2 = i < 32 ? __shfl_sync(0xffffffffu, l2_lane, i) : lse_of(i);
-                const float wgt = (l2 == -INFINITY) ? 0.f : exp2f(l2 - M);
-                den += wgt;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc[4 * e] = fmaf(wgt, v[u][e].x, acc[4 * e]);
-                    acc[4 * e + 1] = fmaf(wgt, v[u][e].y, acc[4 * e + 1]);
-                    acc[4 * e + 2] = fmaf(wgt, v[u][e].z, acc[4 * e + 2]);
-                    acc[4 * e + 3] = fmaf(wgt, v[u][e].w, acc[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float4 v = row[32 * e];
+                        acc[4 * e] = fmaf(wgt, v.x, acc[4 * e]);
+                        acc[4 * e + 1] = fmaf(wgt, v.y, acc[4 * e + 1]);
+                        acc[4 * e + 2] = fmaf(wgt, v.z, acc[4 * e + 2]);
+                        acc[4 * e + 3] = fmaf(wgt, v.w, acc[4 * e + 3]);
+                    }
                 }
             }
         }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        uint32_t pk[8];
+        if (!row_ok) continue;
+        if (!visible) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) pk[e] = pack_bf162(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int e = 0; e < 4; ++e) dst[32 * e] = make_uint2(0, 0);
+            if (lane == 0 && out_lse) out_lse[orow] = -INFINITY;
+            continue;
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            dst[32 * e] = make_uint2(pack_bf162(acc[4 * e] * inv, acc[4 * e + 1] * inv),
+                                     pack_bf162(acc[4 * e + 2] * inv, acc[4 * e + 3] * inv));
         if (lane == 0 && out_lse) out_lse[orow] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
     }
 }

@@ -320,12 +320,14 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
                                da);
     count_launch();
     if (e != cudaSuccess) return MLA_ERR_CUDA;
-    const int ctas = combine_ctas(B, s, H);
-    const int cgrid = ctas < kCombineCtasPerSm * sm_count() ? ctas : kCombineCtasPerSm * sm_count();
+    static std::atomic<bool> attr_cb[kMaxDevices];
+    if (ensure_smem_attr(dec_combine_kernel, kCombineSmem, attr_cb) != cudaSuccess) return MLA_ERR_CUDA;
+    const int blocks = combine_blocks(B, s, H);
+    const int cgrid = blocks < kCombineCtasPerSm * sm_count() ? blocks : kCombineCtasPerSm * sm_count();
     const size_t part_bytes = 2 * (size_t)ranges * s * H * kDc * sizeof(float);
-    e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), 0, strm, (const int32_t *)plan,
+    e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), kCombineSmem, strm, (const int32_t *)plan,
                    (const float *)da.part_o, (const float *)da.part_lse2, part_bytes, B, s, H, (bf16 *)out_latent,
-                   out_lse);
+                   out_lse, err, da.limit_ns);
     count_launch();
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

@@ -46,33 +46,44 @@ def combine_list(seq_lens, max_blocks, q, start):
 
 
 def emulate_combine(B, s, H, seq_lens, max_blocks, q, start, grid):
-    """The combine's loops: warp w of CTA blk takes item blk*8 + w, then
-    strides by grid*8 over the (listed sequence, row) items."""
+    """The combine's loops: CTA c takes blocks c, c + grid, ... of 8 rows of
+    the listed sequences; warp w of a block takes row 8 rb + w; thread 0
+    bulk-copies rows [8 rb, 8 rb + nr) of each piece's slot."""
     rows = s * H
+    nbr = (rows + COMBINE_WARPS - 1) // COMBINE_WARPS
     lst = combine_list(seq_lens, max_blocks, q, start)
-    items = len(lst) * rows
-    reads, writes, rows_seen = [], [], set()
-    for blk in range(grid):
-        for warp in range(COMBINE_WARPS):
-            for w in range(blk * COMBINE_WARPS + warp, items, grid * COMBINE_WARPS):
-                li, rr = divmod(w, rows)
-                b, a0, a1, L = lst[li]
-                c0 = a0 // q if a1 > a0 else 0
-                c1 = (a1 - 1) // q if a1 > a0 else 0
-                split = a1 > a0 and c0 != c1
-                if not split and L >= s:
+    nblk = len(lst) * nbr
+    reads, writes, rows_seen, copies = [], [], set(), []
+    for cta in range(grid):
+        for blk in range(cta, nblk, grid):
+            li, rb = divmod(blk, nbr)
+            b, a0, a1, L = lst[li]
+            c0 = a0 // q if a1 > a0 else 0
+            c1 = (a1 - 1) // q if a1 > a0 else 0
+            split = a1 > a0 and c0 != c1
+            rr0 = rb * COMBINE_WARPS
+            nr = min(COMBINE_WARPS, rows - rr0)
+            if split:
+                for c in range(c0, c1 + 1):
+                    slot = 2 * c + (1 if (c == c0 and a0 != c * q) else 0)
+                    copies.append((slot, rr0, rr0 + nr))
+            for warp in range(COMBINE_WARPS):
+                rr = rr0 + warp
+                if warp >= nr:
                     continue
                 assert rr < rows
-                t = rr // H
+                visible = L - s + rr // H + 1 > 0
+                if not split and visible:
+                    continue
                 orow = b * rows + rr
                 rows_seen.add((b, rr))
-                writes.append((orow * 512, orow * 512 + 32 * 16))   # 32 lanes x 16 columns
-                if L - s + t + 1 <= 0 or not split:
+                writes.append((orow * 512, orow * 512 + 4 * 32 * 4))   # 4 x 32 lanes x 4 columns
+                if not split or not visible:
                     continue
                 for c in range(c0, c1 + 1):
                     slot = 2 * c + (1 if (c == c0 and a0 != c * q) else 0)
                     reads.append((slot, rr))
-    return reads, writes, rows_seen
+    return reads, writes, rows_seen, copies
 
 
 @pytest.mark.parametrize("sms", [148, 132, 8, 1])
@@ -84,12 +95,14 @@ def test_combine_indices_stay_in_bounds(name, sms):
     ranges, groups = ranges_of(sms, cfg.s, cfg.H)
     q, total, start = plan(sl, cfg.s, max_blocks, ranges)
     assert q * ranges >= total                      # every tile lies in some range
-    grid = min((cfg.B * cfg.s * cfg.H + COMBINE_WARPS - 1) // COMBINE_WARPS, 3 * sms)
-    reads, writes, rows_seen = emulate_combine(cfg.B, cfg.s, cfg.H, sl, max_blocks, q, start, grid)
+    grid = min(cfg.B * ((cfg.s * cfg.H + COMBINE_WARPS - 1) // COMBINE_WARPS), 3 * sms)
+    reads, writes, rows_seen, copies = emulate_combine(cfg.B, cfg.s, cfg.H, sl, max_blocks, q, start, grid)
     rows = cfg.s * cfg.H
     nslot = workspace_slots(cfg.s, cfg.H)
     for slot, rr in reads:
         assert 0 <= slot < 2 * ranges <= nslot and 0 <= rr < rows
+    for slot, r0, r1 in copies:   # bulk copies stay inside the slot's rows
+        assert 0 <= slot < 2 * ranges <= nslot and 0 <= r0 < r1 <= rows and r1 - r0 <= COMBINE_WARPS
     for lo, hi in writes:
         assert 0 <= lo and hi <= cfg.B * rows * 512
     # every row of every cut sequence is written exactly by one warp of one item
@@ -106,7 +119,7 @@ def test_combine_rows_bound_at_sixteen_rows():
     of an empty sequence are still written (zeroed)."""
     sl = np.array([4096, 4096, 100, 0], np.int32)
     q, total, start = plan(sl, 1, 64, ranges=3)
-    reads, writes, rows_seen = emulate_combine(4, 1, 16, sl, 64, q, start, grid=3)
+    reads, writes, rows_seen, _ = emulate_combine(4, 1, 16, sl, 64, q, start, grid=3)
     assert all(rr < 16 for _, rr in reads)
     assert max(r for _, r in rows_seen) == 15
     # the empty sequence's rows are zeroed (written) though it has no partial
