@@ -145,23 +145,6 @@ bool tmap(CUtensorMap *m, const void *p, uint64_t inner, uint64_t rows, uint64_t
     return make_tmap_3d(m, p, inner, rows, batch, s1, s2, box_inner, box_rows, 1, swizzle_for(box_inner * 2));
 }
 
-// C = A B on tcgen05; `c` is the output tensor map of the staged (TMA store)
-// epilogue, unused by the others.
-template <int BN, bool kBmn, class Epi, bool kAmn = false>
-cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
-                           uint32_t *err, cudaStream_t st, const CUtensorMap *c = nullptr)
-{
-    using S = GemmSmem<BN>;
-    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kAmn>;
-    static std::atomic<bool> attr_set[kMaxDevices];
-    const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
-    if (e != cudaSuccess) return e;
-    dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
-    kern<<<grid, kGemmThreads, S::BYTES, st>>>(a, b, c ? *c : a, M, N, K, epi, err, kWaitLimitNs);
-    count_launch();
-    return cudaGetLastError();
-}
-
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel on the stream runs, and waits for it with pdl_wait().
 template <class... KArgs, class... Args>
@@ -179,6 +162,24 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// C = A B on tcgen05; `c` is the output tensor map of the staged (TMA store)
+// epilogue, unused by the others.
+template <int BN, bool kBmn, class Epi, bool kAmn = false>
+cudaError_t launch_tc_gemm(const CUtensorMap &a, const CUtensorMap &b, int M, int N, int K, int Z, const Epi &epi,
+                           uint32_t *err, cudaStream_t st, const CUtensorMap *c = nullptr)
+{
+    using S = GemmSmem<BN>;
+    auto kern = tc_gemm_kernel<BN, kBmn, Epi, kAmn>;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e = ensure_smem_attr(kern, S::BYTES, attr_set);
+    if (e != cudaSuccess) return e;
+    dim3 grid((N + BN - 1) / BN, (M + 127) / 128, Z);
+    const cudaError_t le = launch_pdl(kern, grid, dim3(kGemmThreads), S::BYTES, st, a, b, c ? *c : a, M, N, K, epi,
+                                      err, kWaitLimitNs);
+    count_launch();
+    return le;
 }
 
 // Workspace of the decode: [error word | pad] [partial latents] [partial lse2]

@@ -71,6 +71,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // launched with programmatic serialization: the set-up above overlaps the
+    // end of the kernel before, whose outputs are read only from here on
+    sm100::pdl_wait();
 
     const unsigned long long drain_ns = limit_ns > 200000000ull ? limit_ns : 200000000ull;
     if (warp == 0) {
