@@ -68,3 +68,24 @@ def test_noalloc_rejects_a_shape_beyond_its_scratch():
     with pytest.raises(M.MLAError) as e:
         M.mla_decode_noalloc(w.dims, q_abs, w.cache, bt, sl, 1, lat, None, flags=M.MLA_FORCE_SIMPLE)
     assert "WORKSPACE" in str(e.value)
+
+
+def test_noalloc_rejects_a_tensor_core_shape_beyond_its_scratch_before_any_launch():
+    """The tensor-core path's partials grow with s*H: 200 query tokens of 128
+    heads form 400 row groups, one range each, and their 51,200 partial rows
+    (105 MB) exceed the 40 MB array.  The call must refuse before launching."""
+    import torch
+    import head_latent_attention_10_b200 as M
+    M.load_library()
+    w = GpuWorkload(CASES[0])
+    s = 200
+    q_abs = torch.zeros(s, 128, 576, dtype=torch.bfloat16, device="cuda")
+    lat = torch.empty(s, 128, 512, dtype=torch.bfloat16, device="cuda")
+    sl = torch.full((1,), 900, dtype=torch.int32, device="cuda")
+    bt = w.block_table[:1].contiguous()
+    torch.cuda.synchronize()
+    n0 = M.mla_kernel_launches()
+    with pytest.raises(M.MLAError) as e:
+        M.mla_decode_noalloc(w.dims, q_abs, w.cache, bt, sl, s, lat, None)
+    assert "WORKSPACE" in str(e.value)
+    assert M.mla_kernel_launches() == n0
