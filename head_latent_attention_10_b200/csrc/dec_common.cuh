@@ -151,18 +151,28 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 // -------------------------------------------------------------------- plan
 // One warp of every decode CTA: the CTA's range of the batch's (sequence,
 // tile) list.  The list holds the ceil(L_b / 64) tiles of every sequence b
-// (its last query sees all L_b tokens) in sequence order; `ranges` contiguous
-// ranges of ceil(total / ranges) tiles cover it.  Lane l takes sequences
-// [l per, (l+1) per); a shuffle scan gives the prefix sums.
-// out = {tiles per range, total tiles, the sequence holding tile rng * quota,
-// that sequence's first tile} (the last two only when rng * quota < total).
-// With `publish` (CTA 0 of the grid), the warp also stores the plan the
-// combine kernel reads and flags invalid lengths:
-//   plan[0] = quota, plan[1] = total, plan[2] = ranges,
+// (its last query sees all L_b tokens) in sequence order.  Ranges are cut by
+// cost: every non-empty sequence also weighs kSwitchTiles virtual tiles
+// placed before its first tile (what a range pays to start a sequence: the
+// previous sequence's epilogue and the next one's queries, about four tiles'
+// time on every shape measured), and the ranges split the virtual list into
+// equal parts of Qv = ceil(VT / ranges) virtual tiles.  A virtual position v
+// inside sequence b (virtual start VA_b, real start A_b) maps to the real
+// tile A_b + max(0, v - VA_b - kSwitchTiles); range r covers the real tiles
+// [real(r Qv), real(min((r + 1) Qv, VT))), real(VT) = the total.  Lane l
+// takes sequences [l per, (l+1) per); shuffle scans give the prefix sums.
+// out = {first tile, end tile, the sequence holding the first tile, that
+// sequence's first tile} (the last two only when the range is not empty).
+// With `publish` (CTA 0 of the grid), the warp also stores what the combine
+// kernel reads, and flags invalid lengths:
+//   plan[0] = Qv, plan[1] = total tiles, plan[2] = ranges, plan[3] = kSwitchTiles,
 //   plan[4 + b] = first tile of sequence b (b = 0..B),
-//   plan[5 + B] = n, the number of sequences the combine finishes (those cut
-//   by a range end, and those with no tile), listed in sequence order as
-//   int4 {b, first tile, end tile, clamped length} from int plan_list_off(B).
+//   plan[5 + B] = n, the number of sequences the combine finishes (those
+//   whose tiles span more than one range, and those with no tile), listed in
+//   sequence order as int4 {b, VA_b, tiles, clamped length} from int
+//   plan_list_off(B).  Sequence b's tiles lie in ranges
+//   c0 = (VA_b + kSwitchTiles) / Qv .. c1 = (VA_b + kSwitchTiles + t_b - 1) / Qv.
+constexpr int kSwitchTiles = 4;
 __host__ __device__ inline int plan_list_off(int B) { return (B + 9) & ~3; }   // 16-byte aligned, after plan[5 + B]
 __host__ __device__ inline int plan_ints(int B) { return plan_list_off(B) + 4 * B; }
 
@@ -173,56 +183,68 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
     const int max_tok = max_blocks * kBlock;
     const int per = (B + 31) / 32;
     const int b0 = min(B, lane * per), b1 = min(B, b0 + per);
-    int sum = 0;
+    auto len_of = [&](int b) {
+        const int L = seq_lens[b];
+        return L < 0 ? 0 : min(L, max_tok);
+    };
+    int sum_t = 0, sum_v = 0;
     for (int b = b0; b < b1; ++b) {
-        int L = seq_lens[b];
+        const int L = seq_lens[b];
         // out of range, or some query sees no key
         if (publish && (L < 0 || L > max_tok || L < s)) set_error(err, MLA_DEVERR_SEQ_LEN);
-        L = L < 0 ? 0 : min(L, max_tok);
-        sum += (L + kBlock - 1) / kBlock;
+        const int t = (len_of(b) + kBlock - 1) / kBlock;
+        sum_t += t;
+        sum_v += t > 0 ? t + kSwitchTiles : 0;
     }
-    int inc = sum;
+    int inc_t = sum_t, inc_v = sum_v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += v;
-    }
-    const int total = __shfl_sync(0xffffffffu, inc, 31);
-    const int q = total > 0 ? (total + ranges - 1) / ranges : 1;
-    const int lo = rng * q;
-    int run = inc - sum;
-    for (int b = b0; b < b1; ++b) {
-        int L = seq_lens[b];
-        L = L < 0 ? 0 : min(L, max_tok);
-        const int t = (L + kBlock - 1) / kBlock;
-        if (publish) plan[4 + b] = run;
-        if (run <= lo && lo < run + t) {
-            out[2] = b;
-            out[3] = run;
+        const int vt = __shfl_up_sync(0xffffffffu, inc_t, o), vv = __shfl_up_sync(0xffffffffu, inc_v, o);
+        if (lane >= o) {
+            inc_t += vt;
+            inc_v += vv;
         }
-        run += t;
     }
-    if (lane == 0) {
-        out[0] = q;
+    const int total = __shfl_sync(0xffffffffu, inc_t, 31), vtot = __shfl_sync(0xffffffffu, inc_v, 31);
+    const int qv = vtot > 0 ? (vtot + ranges - 1) / ranges : 1;
+    const int v_lo = rng * qv, v_hi = min(v_lo + qv, vtot);
+    if (lane == 0) {   // a boundary at or past the end of the list
+        out[0] = total;
         out[1] = total;
-        if (publish) {
-            plan[0] = q;
-            plan[1] = total;
-            plan[2] = ranges;
-            plan[4 + B] = total;
+    }
+    __syncwarp();
+    int run_t = inc_t - sum_t, run_v = inc_v - sum_v;
+    for (int b = b0; b < b1; ++b) {
+        const int t = (len_of(b) + kBlock - 1) / kBlock;
+        const int w = t > 0 ? t + kSwitchTiles : 0;
+        if (v_lo >= run_v && v_lo < run_v + w) {
+            out[0] = run_t + max(0, v_lo - run_v - kSwitchTiles);
+            out[2] = b;
+            out[3] = run_t;
         }
+        if (v_hi >= run_v && v_hi < run_v + w) out[1] = run_t + max(0, v_hi - run_v - kSwitchTiles);
+        if (publish) plan[4 + b] = run_t;
+        run_t += t;
+        run_v += w;
     }
     if (publish) {
-        // the combine's list: sequences cut by a range end, or with no tile
-        auto listed = [&](int a0, int a1) { return a1 == a0 || a0 / q != (a1 - 1) / q; };
+        if (lane == 0) {
+            plan[0] = qv;
+            plan[1] = total;
+            plan[2] = ranges;
+            plan[3] = kSwitchTiles;
+            plan[4 + B] = total;
+        }
+        // the combine's list: sequences spanning more than one range, or with no tile
+        auto listed = [&](int va, int t) {
+            return t == 0 || (va + kSwitchTiles) / qv != (va + kSwitchTiles + t - 1) / qv;
+        };
         int cnt = 0;
-        run = inc - sum;
+        run_v = inc_v - sum_v;
         for (int b = b0; b < b1; ++b) {
-            int L = seq_lens[b];
-            L = L < 0 ? 0 : min(L, max_tok);
-            const int e = run + (L + kBlock - 1) / kBlock;
-            cnt += listed(run, e) ? 1 : 0;
-            run = e;
+            const int t = (len_of(b) + kBlock - 1) / kBlock;
+            cnt += listed(run_v, t) ? 1 : 0;
+            run_v += t > 0 ? t + kSwitchTiles : 0;
         }
         int ci = cnt;
 #pragma unroll
@@ -232,13 +254,12 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
         }
         int4 *list = reinterpret_cast<int4 *>(plan + plan_list_off(B));
         int at = ci - cnt;
-        run = inc - sum;
+        run_v = inc_v - sum_v;
         for (int b = b0; b < b1; ++b) {
-            int L = seq_lens[b];
-            L = L < 0 ? 0 : min(L, max_tok);
-            const int e = run + (L + kBlock - 1) / kBlock;
-            if (listed(run, e)) list[at++] = make_int4(b, run, e, L);
-            run = e;
+            const int L = len_of(b);
+            const int t = (L + kBlock - 1) / kBlock;
+            if (listed(run_v, t)) list[at++] = make_int4(b, run_v, t, L);
+            run_v += t > 0 ? t + kSwitchTiles : 0;
         }
         if (lane == 31) plan[5 + B] = ci;
     }
@@ -258,7 +279,7 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
 // the float4 columns l, 32 + l, 64 + l and 96 + l, so that the shared-memory
 // reads are conflict-free and the output stores contiguous across the warp.
 // Pieces are summed in range order.  Every partial slot lies in
-// [2 c0, 2 c1 + 1] with c1 < ranges.
+// [2 c0, 2 c1 + 1] with c1 < ranges (plan_range gives c0, c1 and the slots).
 constexpr int kCombineWarps = 8;                  // rows per block
 constexpr int kCombineThreads = 32 * kCombineWarps;
 constexpr int kCombinePieces = 4;                 // pieces per bulk round
@@ -271,10 +292,6 @@ __host__ __device__ inline int combine_blocks(int B, int s, int H)
     return B * ((s * H + kCombineWarps - 1) / kCombineWarps);
 }
 
-__device__ __forceinline__ int piece_slot(int c, int c0, int a0, int q)
-{
-    return 2 * c + ((c == c0 && a0 != c * q) ? 1 : 0);
-}
 
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm)
 dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
@@ -299,7 +316,7 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
     __syncthreads();
     sm100::pdl_wait();      // the decode kernel's partials, outputs and plan are complete
     const int rows = s * H, nbr = (rows + kCombineWarps - 1) / kCombineWarps;
-    const int q = plan[0];
+    const int qv = plan[0], pw = plan[3];
     const int nblk = plan[5 + B] * nbr;
     const int4 *list = reinterpret_cast<const int4 *>(plan + plan_list_off(B));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -308,9 +325,14 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
     for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
         const int li = blk / nbr, rb = blk - li * nbr;
         const int4 seq = list[li];
-        const int b = seq.x, a0 = seq.y, a1 = seq.z, L = seq.w;
-        const int c0 = a1 > a0 ? a0 / q : 0, c1 = a1 > a0 ? (a1 - 1) / q : 0;
-        const bool split = a1 > a0 && c0 != c1;
+        const int b = seq.x, va = seq.y, tb = seq.z, L = seq.w;
+        // the ranges holding the sequence's first and last tiles; the piece in
+        // range c0 is that range's first segment only if the range starts with
+        // the sequence (slot 2 c0), else its last (2 c0 + 1); every later piece
+        // is its range's first segment (slot 2 c)
+        const int c0 = tb > 0 ? (va + pw) / qv : 0, c1 = tb > 0 ? (va + pw + tb - 1) / qv : 0;
+        const bool split = tb > 0 && c0 != c1;
+        const int slot0 = 2 * c0 + (c0 * qv < va ? 1 : 0);
         const int rr0 = rb * kCombineWarps, nr = min(kCombineWarps, rows - rr0);
         const int rr = rr0 + warp;
         const bool row_ok = warp < nr;
@@ -327,7 +349,7 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
             continue;   // uniform: the whole block belongs to one sequence
         }
         const int n = c1 - c0 + 1;
-        auto lse_of = [&](int i) { return part_lse2[(long long)piece_slot(c0 + i, c0, a0, q) * rows + rr]; };
+        auto lse_of = [&](int i) { return part_lse2[(long long)(i == 0 ? slot0 : 2 * (c0 + i)) * rows + rr]; };
         const bool merge = row_ok && visible;
         const float l2_lane = (merge && lane < n) ? lse_of(lane) : -INFINITY;
         float M = l2_lane;
@@ -345,7 +367,7 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
                 sm100::mbar_arrive_expect_tx(bar, (uint32_t)(np * nr * kDc * 4));
                 for (int u = 0; u < np; ++u)
                     sm100::bulk_load(cb_smem + u * (kCombineWarps * kDc * 4),
-                                     part_o + ((long long)piece_slot(c0 + i0 + u, c0, a0, q) * rows + rr0) * kDc,
+                                     part_o + ((long long)(i0 + u == 0 ? slot0 : 2 * (c0 + i0 + u)) * rows + rr0) * kDc,
                                      (uint32_t)(nr * kDc * 4), bar);
             }
             bool ok = sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns);

@@ -49,9 +49,10 @@
 // Online softmax in the log2 domain with lazy rescaling (O and l are rescaled
 // only when the running max grows by more than 8, a factor 256).
 //
-// Work split: the (sequence, tile) list of the batch is cut into equal
-// contiguous ranges per row group (plan_range, one warp of every CTA).  A sequence a range covers
-// completely is normalized and written straight to the output.  A sequence cut
+// Work split: the (sequence, tile) list of the batch is cut into contiguous
+// ranges of equal cost per row group, a tile counting one and the start of a
+// sequence four (plan_range, one warp of every CTA).  A sequence a range
+// covers completely is normalized and written straight to the output.  A sequence cut
 // by range ends leaves one fp32 partial per piece (normalized, with its
 // log2-sum-exp), merged by dec_combine_kernel.  Every wait is bounded; a wait
 // that gives up sets MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own
@@ -168,8 +169,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     __syncthreads();
     sm100::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int q_per = rplan[0], total = rplan[1];
-    const int lo = rng * q_per, hi = min(lo + q_per, total);
+    const int lo = rplan[0], hi = rplan[1];
     if (lo >= hi) {   // no tile for this CTA
         if (warp == 1) sm100::tmem_dealloc(tmem, 512);
         return;

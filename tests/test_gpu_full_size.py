@@ -39,15 +39,21 @@ def run(request):
 def cut_sequences(g):
     """Sequences the decode's split plan cut across CTAs, from the plan the
     call left in its workspace (int32 words after the 256-byte error-word
-    slot: tiles per range, total tiles, ranges, -, then the first tile of
-    each sequence).  Their outputs come from the combine kernel."""
+    slot: virtual tiles per range, total tiles, ranges, the switch weight in
+    tiles, then the first tile of each sequence).  A sequence with t tiles and
+    virtual start VA (its first tile's start plus the weight of the non-empty
+    sequences before it) spans ranges (VA + w) // q .. (VA + w + t - 1) // q;
+    the outputs of those spanning more than one come from the combine."""
     import torch
     B = g.cfg.B
     plan = g.ws[256:256 + 4 * (4 + B + 1)].view(torch.int32).cpu().numpy()
-    q, total = int(plan[0]), int(plan[1])
-    start = plan[4:4 + B + 1]
+    q, total, w = int(plan[0]), int(plan[1]), int(plan[3])
+    start = plan[4:4 + B + 1].astype(np.int64)
     assert start[-1] == total
-    cut = [b for b in range(B) if start[b + 1] > start[b] and start[b] // q != (start[b + 1] - 1) // q]
+    tiles = np.diff(start)
+    vstart = np.concatenate([[0], np.cumsum(np.where(tiles > 0, tiles + w, 0))])
+    cut = [b for b in range(B)
+           if tiles[b] > 0 and (vstart[b] + w) // q != (vstart[b] + w + tiles[b] - 1) // q]
     return np.asarray(cut, np.int64)
 
 
