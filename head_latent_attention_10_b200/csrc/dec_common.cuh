@@ -10,6 +10,7 @@
 namespace mla {
 
 constexpr int kGroupRows = 64;                // rows of one work unit (the MMA M dimension)
+constexpr int kSwitchTiles = 4;               // the planning weight of a sequence start, in tiles
 constexpr int kMaxRanges = 148;               // ranges per row group at most (= CTAs / groups)
 constexpr float kRescaleThreshold = 8.0f;     // lazy rescale of the running max, log2 units
 
@@ -18,6 +19,9 @@ struct DecArgs {
     const int32_t *block_table;
     const int32_t *seq_lens;
     int32_t *plan;        // written by CTA 0 for the combine (plan_range)
+    int *flags;           // per (sequence, row group, warp quarter): [0, n) early piece written,
+                          // [n, 2n) merged by the late piece's CTA (n = B * groups * 4); [2n] the
+                          // combine's work count (0: nothing left to merge)
     bf16 *out;
     float *out_lse;
     float *part_o;        // [2*ranges][s*H][512] fp32
@@ -45,12 +49,13 @@ __device__ __forceinline__ int seq_len_clamped(const int32_t *seq_lens, int b, i
 
 // Walks a range of the (sequence, tile) list one tile at a time.  Sequence
 // r holds tiles [a_r, a_r + ceil(L_r / 64)); the walk starts in sequence r0,
-// whose first tile a0 the range's plan gives, and takes the later starts from
-// the sequence lengths.
+// whose first tile a0 and virtual start v0 the range's plan gives, and takes
+// the later starts from the sequence lengths.  seq_a, seq_t and seq_v are the
+// current segment's sequence's first tile, tile count and virtual start.
 struct TileIter {
     const int32_t *sl;
-    int max_tok, n, pos, hi, r, ar;
-    int seq, t0, t1, seg, tt, k;
+    int max_tok, n, pos, hi, r, ar, vr;
+    int seq, t0, t1, seg, tt, k, seq_a, seq_t, seq_v;
     bool complete, ok;
     __device__ int tiles(int b) const
     {
@@ -61,24 +66,26 @@ struct TileIter {
     __device__ bool next_seg()
     {
         if (pos >= hi) return false;
-        int e;
+        int t;
         for (;;) {
             if (r >= n) return false;
-            e = ar + tiles(r);
-            if (e > pos) break;
-            ar = e;   // an empty sequence, or one that ends before pos
+            t = tiles(r);
+            if (ar + t > pos) break;
+            ar += t;   // an empty sequence, or one that ends before pos
+            vr += t > 0 ? t + kSwitchTiles : 0;
             ++r;
         }
-        const int end = min(hi, e);
+        const int e = ar + t, end = min(hi, e);
         seq = r; t0 = pos - ar; t1 = end - ar;
+        seq_a = ar; seq_t = t; seq_v = vr;
         complete = (pos == ar) && (end == e);
-        pos = end; ar = e; ++r; ++seg;
+        pos = end; ar = e; vr += t + kSwitchTiles; ++r; ++seg;
         return true;
     }
-    __device__ void init(const int32_t *seq_lens, int max_blocks, int n_, int lo, int hi_, int r0, int a0)
+    __device__ void init(const int32_t *seq_lens, int max_blocks, int n_, int lo, int hi_, int r0, int a0, int v0)
     {
         sl = seq_lens; max_tok = max_blocks * kBlock; n = n_; pos = lo; hi = hi_; seg = -1; k = 0;
-        r = r0; ar = a0;
+        r = r0; ar = a0; vr = v0;
         ok = next_seg();
         tt = t0;
     }
@@ -140,6 +147,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
                  : "memory");
 }
 
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 {
     uint4 v;
@@ -162,7 +176,8 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 // [real(r Qv), real(min((r + 1) Qv, VT))), real(VT) = the total.  Lane l
 // takes sequences [l per, (l+1) per); shuffle scans give the prefix sums.
 // out = {first tile, end tile, the sequence holding the first tile, that
-// sequence's first tile} (the last two only when the range is not empty).
+// sequence's first tile, Qv, that sequence's virtual start} (the third,
+// fourth and sixth only when the range is not empty).
 // With `publish` (CTA 0 of the grid), the warp also stores what the combine
 // kernel reads, and flags invalid lengths:
 //   plan[0] = Qv, plan[1] = total tiles, plan[2] = ranges, plan[3] = kSwitchTiles,
@@ -172,12 +187,14 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
 //   sequence order as int4 {b, VA_b, tiles, clamped length} from int
 //   plan_list_off(B).  Sequence b's tiles lie in ranges
 //   c0 = (VA_b + kSwitchTiles) / Qv .. c1 = (VA_b + kSwitchTiles + t_b - 1) / Qv.
-constexpr int kSwitchTiles = 4;
 __host__ __device__ inline int plan_list_off(int B) { return (B + 9) & ~3; }   // 16-byte aligned, after plan[5 + B]
 __host__ __device__ inline int plan_ints(int B) { return plan_list_off(B) + 4 * B; }
 
+// `work` (with `publish`): raised by the number of listed sequences the
+// decode kernel does not merge itself (empty ones, those cut into three or
+// more pieces, and with !merge_two the two-piece ones too).
 __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int rng,
-                           bool publish, int32_t *plan, uint32_t *err, int *out)
+                           bool publish, bool merge_two, int32_t *plan, int *work, uint32_t *err, int *out)
 {
     const int lane = threadIdx.x & 31;
     const int max_tok = max_blocks * kBlock;
@@ -211,6 +228,7 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
     if (lane == 0) {   // a boundary at or past the end of the list
         out[0] = total;
         out[1] = total;
+        out[4] = qv;
     }
     __syncwarp();
     int run_t = inc_t - sum_t, run_v = inc_v - sum_v;
@@ -221,6 +239,7 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
             out[0] = run_t + max(0, v_lo - run_v - kSwitchTiles);
             out[2] = b;
             out[3] = run_t;
+            out[5] = run_v;
         }
         if (v_hi >= run_v && v_hi < run_v + w) out[1] = run_t + max(0, v_hi - run_v - kSwitchTiles);
         if (publish) plan[4 + b] = run_t;
@@ -239,13 +258,18 @@ __device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, i
         auto listed = [&](int va, int t) {
             return t == 0 || (va + kSwitchTiles) / qv != (va + kSwitchTiles + t - 1) / qv;
         };
-        int cnt = 0;
+        int cnt = 0, left = 0;
         run_v = inc_v - sum_v;
         for (int b = b0; b < b1; ++b) {
             const int t = (len_of(b) + kBlock - 1) / kBlock;
-            cnt += listed(run_v, t) ? 1 : 0;
+            if (listed(run_v, t)) {
+                ++cnt;
+                const int pieces = t > 0 ? (run_v + kSwitchTiles + t - 1) / qv - (run_v + kSwitchTiles) / qv + 1 : 0;
+                left += (pieces == 2 && merge_two) ? 0 : 1;
+            }
             run_v += t > 0 ? t + kSwitchTiles : 0;
         }
+        if (left) atomicAdd(work, left);
         int ci = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -294,27 +318,21 @@ __host__ __device__ inline int combine_blocks(int B, int s, int H)
 
 
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm)
-dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ part_o,
-                   const float *__restrict__ part_lse2, size_t part_bytes, int B, int s, int H,
-                   bf16 *__restrict__ out, float *__restrict__ out_lse, uint32_t *err, unsigned long long limit_ns)
+dec_combine_kernel(const int32_t *__restrict__ plan, const int *__restrict__ flags, const float *__restrict__ part_o,
+                   const float *__restrict__ part_lse2, int B, int s, int H, bf16 *__restrict__ out,
+                   float *__restrict__ out_lse, uint32_t *err, unsigned long long limit_ns)
 {
     extern __shared__ __align__(128) uint8_t cb_smem[];
     const float4 *buf = reinterpret_cast<const float4 *>(cb_smem);
     uint64_t *bar = reinterpret_cast<uint64_t *>(cb_smem + kCombineBuf);
     if (threadIdx.x == 0) {
-        // CTAs that start while the decode's last CTAs run bring the partial
-        // area back into L2 (the pieces written early in the decode have long
-        // been evicted by the streaming pages); a hint only: the values are
-        // read after the wait below
-        const size_t per = (part_bytes / gridDim.x + 255) & ~size_t(255);
-        const size_t o0 = (size_t)blockIdx.x * per, o1 = min(part_bytes, o0 + per);
-        for (size_t o = o0; o < o1; o += 16384)
-            sm100::bulk_prefetch_l2(reinterpret_cast<const char *>(part_o) + o, (uint32_t)min((size_t)16384, o1 - o));
         sm100::mbar_init(bar, 1);
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    sm100::pdl_wait();      // the decode kernel's partials, outputs and plan are complete
+    sm100::pdl_wait();      // the decode kernel's partials, outputs, plan and flags are complete
+    const int groups = (s * H + kGroupRows - 1) / kGroupRows;
+    if (flags[2 * B * groups * 4] == 0) return;   // the decode kernel merged every cut sequence
     const int rows = s * H, nbr = (rows + kCombineWarps - 1) / kCombineWarps;
     const int qv = plan[0], pw = plan[3];
     const int nblk = plan[5 + B] * nbr;
@@ -334,6 +352,10 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const float *__restrict__ p
         const bool split = tb > 0 && c0 != c1;
         const int slot0 = 2 * c0 + (c0 * qv < va ? 1 : 0);
         const int rr0 = rb * kCombineWarps, nr = min(kCombineWarps, rows - rr0);
+        // a two-piece sequence whose late piece merged this block's quarter
+        // itself (the decode kernel's epilogue) is already in place
+        if (split && c1 == c0 + 1 && flags[B * groups * 4 + (b * groups + rr0 / kGroupRows) * 4 + (rr0 % kGroupRows) / 16])
+            continue;
         const int rr = rr0 + warp;
         const bool row_ok = warp < nr;
         const bool visible = L - s + rr / H + 1 > 0;   // query rr / H sees some key

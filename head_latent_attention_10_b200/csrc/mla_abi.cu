@@ -201,8 +201,10 @@ SimpleWs simple_ws(int H, int T, int max_seq_len)
 }
 
 // Tensor-core decode workspace: [error word][plan][partial latents][partial lse2]
+// [merge flags][partial latents][partial lse2]; the first off_zero_end bytes
+// are zeroed per call
 struct TcWs {
-    size_t off_plan, off_o, off_lse, total;
+    size_t off_plan, off_flags, off_zero_end, off_o, off_lse, total;
 };
 
 inline int dec_groups(int H, int s) { return (s * H + kGroupRows - 1) / kGroupRows; }
@@ -213,7 +215,9 @@ TcWs tc_ws(int H, int s, int B)
     const int groups = dec_groups(H, s);
     const int ranges = kMaxRanges / groups > 0 ? kMaxRanges / groups : 1;
     w.off_plan = kWsAlign;
-    w.off_o = align_up(w.off_plan + (size_t)plan_ints(B) * sizeof(int32_t), kWsAlign);
+    w.off_flags = align_up(w.off_plan + (size_t)plan_ints(B) * sizeof(int32_t), 16);
+    w.off_zero_end = w.off_flags + (2 * (size_t)B * groups * 4 + 1) * sizeof(int);
+    w.off_o = align_up(w.off_zero_end, kWsAlign);
     const size_t slots = 2 * (size_t)ranges * s * H;
     w.off_lse = align_up(w.off_o + slots * kDc * sizeof(float), kWsAlign);
     w.total = align_up(w.off_lse + slots * sizeof(float), kWsAlign);
@@ -292,9 +296,11 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     } else {
         if (!tmap(&mkv, cache, kRow, (uint64_t)num_blocks * kBlock, 1, kRow, 0, 64, kT64)) return MLA_ERR_CUDA;
     }
-    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), strm) != cudaSuccess) return MLA_ERR_CUDA;
+    // the error word, the plan and the merge flags
+    if (cudaMemsetAsync(ws, 0, w.off_zero_end, strm) != cudaSuccess) return MLA_ERR_CUDA;
     int32_t *plan = (int32_t *)(ws + w.off_plan);
     DecArgs da;
+    da.flags = (int *)(ws + w.off_flags);
     da.q_abs = (const bf16 *)q_abs;
     da.block_table = block_table;
     da.seq_lens = seq_lens;
@@ -325,10 +331,9 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     if (ensure_smem_attr(dec_combine_kernel, kCombineSmem, attr_cb) != cudaSuccess) return MLA_ERR_CUDA;
     const int blocks = combine_blocks(B, s, H);
     const int cgrid = blocks < kCombineCtasPerSm * sm_count() ? blocks : kCombineCtasPerSm * sm_count();
-    const size_t part_bytes = 2 * (size_t)ranges * s * H * kDc * sizeof(float);
     e = launch_pdl(dec_combine_kernel, dim3(cgrid), dim3(kCombineThreads), kCombineSmem, strm, (const int32_t *)plan,
-                   (const float *)da.part_o, (const float *)da.part_lse2, part_bytes, B, s, H, (bf16 *)out_latent,
-                   out_lse, err, da.limit_ns);
+                   (const int *)da.flags, (const float *)da.part_o, (const float *)da.part_lse2, B, s, H,
+                   (bf16 *)out_latent, out_lse, err, da.limit_ns);
     count_launch();
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

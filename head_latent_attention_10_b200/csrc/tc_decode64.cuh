@@ -131,7 +131,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 17);
 
-    int *rplan = reinterpret_cast<int *>(bars + 40);   // this CTA's range (plan_range's out)
+    int *rplan = reinterpret_cast<int *>(bars + 40);   // this CTA's range (plan_range's out, 6 ints)
+    uint64_t *early_in = bars + 44;  // [4] a late piece's merge: the early piece's rows landed (softmax warp q)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = blockIdx.x % a.groups, rng = blockIdx.x / a.groups;
@@ -152,6 +153,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         if constexpr (kFp8)
             for (int i = 0; i < kD64Stages; ++i) sm100::mbar_init(&cv_full[i], kD64Cvt / 32);
         sm100::mbar_init(mma_done, 7);
+        for (int i = 0; i < 4; ++i) sm100::mbar_init(&early_in[i], 1);
         *abort_flag = 0;
         sm100::fence_mbar_init();
         sm100::prefetch_tensormap(&map_kv);
@@ -163,8 +165,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     // the sequence lengths and queries may come from the kernel before this one
     sm100::pdl_wait();
     if (warp == 2)
-        plan_range(a.seq_lens, a.B, a.s, a.max_blocks, gridDim.x / a.groups, rng, blockIdx.x == 0, a.plan, a.err,
-                   rplan);
+        plan_range(a.seq_lens, a.B, a.s, a.max_blocks, gridDim.x / a.groups, rng, blockIdx.x == 0, !kFp8, a.plan,
+                   a.flags + 2 * a.B * a.groups * 4, a.err, rplan);
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
@@ -175,6 +177,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         return;
     }
     const int seq0 = rplan[2], start0 = rplan[3];   // the sequence holding tile lo, its first tile
+    const int qv = rplan[4], va0 = rplan[5];         // the plan's virtual quota, seq0's virtual start
     const unsigned long long lim = a.limit_ns;
     const unsigned long long drain = lim > 200000000ull ? lim : 200000000ull;
     uint8_t *stages = smem + kD64OffStage;
@@ -188,7 +191,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             TileIter it, ahead;
-            it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
+            it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0, va0);
             ahead = it;
             for (int i = 0; i < kD64Ahead && ahead.ok; ++i) ahead.advance();
             // warm L2 with the page kD64Ahead tiles further on (and, when that tile
@@ -272,7 +275,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         const uint32_t scol = b < 2 ? 64u * b : kD64TmS2;
         const uint32_t idesc_s = kFp8 ? sm100::idesc_f16(kGroupRows, kT64, 0, 0) : sm100::idesc_bf16(kGroupRows, kT64, 0, 0);
         TileIter is;
-        is.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
+        is.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0, va0);
         int q_seg = -1;
         bool ok = true;
         while (ok && is.ok) {
@@ -321,7 +324,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         // ct % 4 of each 64-column chunk (a warp reads 512 contiguous bytes)
         const int ct = threadIdx.x - kD64Threads, g = ct & 3;
         TileIter it;
-        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
+        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0, va0);
         bool ok = true;
         while (ok && it.ok) {
             const int k = it.k, st = k % kD64Stages;
@@ -451,7 +454,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
             }
         };
         TileIter it;
-        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0);
+        it.init(a.seq_lens, a.max_blocks, a.B, lo, hi, seq0, start0, va0);
         float m_run = -INFINITY, l_run = 0.f;
         int nvis = 0, nseq = 0;
         const uint32_t idesc_o = kFp8 ? sm100::idesc_f16(kGroupRows, 256, 0, 1) : sm100::idesc_bf16(kGroupRows, 256, 0, 1);
@@ -465,6 +468,18 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 // query tq of a sequence of length L sees positions j <= L - s + tq
                 nseq = seq_len_clamped(a.seq_lens, it.seq, a.max_blocks);
                 nvis = nseq - a.s + tq + 1;
+            }
+            if (lane == 0 && (it.tt + 4 == it.t1 || (it.first() && it.t1 - it.t0 < 4))) {
+                // a late piece (see the epilogue): bring the early piece's rows of
+                // this warp's quarter into L2 before the merge reads them
+                const int cf = (it.seq_v + kSwitchTiles) / qv, cl = (it.seq_v + kSwitchTiles + it.seq_t - 1) / qv;
+                const int r0 = group * kGroupRows + 16 * qd;
+                if (!kFp8 && !it.complete && cl == cf + 1 && rng == cf && r0 < rows_per_seq) {
+                    const char *e = reinterpret_cast<const char *>(a.part_o + (2LL * cl * rows_per_seq + r0) * kDc);
+                    const int nr = min(16, rows_per_seq - r0);
+                    for (int o = 0; o < nr * kDc * 4; o += 16384)
+                        sm100::bulk_prefetch_l2(e + o, (uint32_t)min(16384, nr * kDc * 4 - o));
+                }
             }
             const int sb = k % 3;
             ok = sm100::warp_wait(&s_full[sb], (k / 3) & 1, abort_flag, a.err, lim);
@@ -630,20 +645,54 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 const uint32_t stg = sm100::smem_u32(smem + (kFp8 ? kD64OffEpiFp8 : kD64OffEpi)) + qd * 16 * RB;
                 const int lr_me = lane & 15, hh = srow ? 0 : 1;
                 auto swz = [](int row) { return (row * RB / 128) & (CPR - 1); };
-                auto drain = [&](auto f32_tag) {
+                // stage pk (the thread's half of its row's block, HB bytes) and
+                // write the warp's 16 rows of block c to base (EB-byte elements)
+                auto store_block = [&](auto f32_tag, int c, const uint4 *pk, char *base) {
                     constexpr bool F32 = decltype(f32_tag)::value;
                     constexpr int EB = F32 ? 4 : 2;          // output element bytes
                     constexpr int HB = 32 * EB;              // a thread's half of a row's block
                     constexpr int NR = 2 * HB / RB;          // staging rounds per block
+#pragma unroll
+                    for (int q = 0; q < NR; ++q) {
+                        // round q stages bytes [q RB, (q+1) RB) of the 16 rows' block
+                        if constexpr (RB >= HB) {
+                            if ((hh * HB) / RB == q) {
+                                const int c0 = (hh * HB - q * RB) >> 4;
+#pragma unroll
+                                for (int j = 0; j < HB / 16; ++j)
+                                    st_shared_v4(stg + lr_me * RB + (((c0 + j) ^ swz(lr_me)) << 4), pk[j]);
+                            }
+                        } else {
+                            constexpr int W = HB / RB;   // rounds per half
+                            if (q / W == hh) {
+#pragma unroll
+                                for (int j = 0; j < CPR; ++j)
+                                    st_shared_v4(stg + lr_me * RB + ((j ^ swz(lr_me)) << 4), pk[(q % W) * CPR + j]);
+                            }
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int e = 0; e < RB / 32; ++e) {
+                            const int f = e * 32 + lane, lr = f / CPR, ch = f % CPR;
+                            const uint4 v = ld_shared_v4(stg + lr * RB + ((ch ^ swz(lr)) << 4));
+                            const int grow = group * kGroupRows + 16 * qd + lr;
+                            if (grow < rows_per_seq)
+                                *reinterpret_cast<uint4 *>(base + ((long long)grow * kDc + c) * EB + q * RB + 16 * ch) = v;
+                        }
+                        __syncwarp();
+                    }
+                };
+                auto drain = [&](auto f32_tag) {
+                    constexpr bool F32 = decltype(f32_tag)::value;
                     char *base = F32 ? reinterpret_cast<char *>(a.part_o + slot * rows_per_seq * kDc)
                                      : reinterpret_cast<char *>(a.out + (long long)it.seq * rows_per_seq * kDc);
                     for (int c = 0; c < 512; c += 64) {
                         uint32_t ov[32];
                         sm100::tmem_ld16x2_32(o_base + c, ov);
                         sm100::tmem_wait_ld();
-                        uint4 pk[HB / 16];
+                        uint4 pk[F32 ? 8 : 4];
 #pragma unroll
-                        for (int j = 0; j < HB / 16; ++j) {
+                        for (int j = 0; j < (F32 ? 8 : 4); ++j) {
                             if constexpr (F32) {
                                 pk[j] = make_uint4(__float_as_uint(__uint_as_float(ov[4 * j]) * inv),
                                                    __float_as_uint(__uint_as_float(ov[4 * j + 1]) * inv),
@@ -656,46 +705,109 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                                                    pack_bf162(__uint_as_float(ov[8 * j + 6]) * inv, __uint_as_float(ov[8 * j + 7]) * inv));
                             }
                         }
-#pragma unroll
-                        for (int q = 0; q < NR; ++q) {
-                            // round q stages bytes [q RB, (q+1) RB) of the 16 rows' block
-                            if constexpr (RB >= HB) {
-                                if ((hh * HB) / RB == q) {
-                                    const int c0 = (hh * HB - q * RB) >> 4;
-#pragma unroll
-                                    for (int j = 0; j < HB / 16; ++j)
-                                        st_shared_v4(stg + lr_me * RB + (((c0 + j) ^ swz(lr_me)) << 4), pk[j]);
-                                }
-                            } else {
-                                constexpr int W = HB / RB;   // rounds per half
-                                if (q / W == hh) {
-#pragma unroll
-                                    for (int j = 0; j < CPR; ++j)
-                                        st_shared_v4(stg + lr_me * RB + ((j ^ swz(lr_me)) << 4), pk[(q % W) * CPR + j]);
-                                }
-                            }
-                            __syncwarp();
-#pragma unroll
-                            for (int e = 0; e < RB / 32; ++e) {
-                                const int f = e * 32 + lane, lr = f / CPR, ch = f % CPR;
-                                const uint4 v = ld_shared_v4(stg + lr * RB + ((ch ^ swz(lr)) << 4));
-                                const int grow = group * kGroupRows + 16 * qd + lr;
-                                if (grow < rows_per_seq)
-                                    *reinterpret_cast<uint4 *>(base + ((long long)grow * kDc + c) * EB + q * RB + 16 * ch) = v;
-                            }
-                            __syncwarp();
-                        }
+                        store_block(f32_tag, c, pk, base);
                     }
                 };
-                if (it.complete)
-                    drain(std::false_type{});
-                else
-                    drain(std::true_type{});
-                if (row_ok && srow) {
-                    if (it.complete) {
-                        if (a.out_lse) a.out_lse[orow] = lse2 * kLn2;
-                    } else {
-                        a.part_lse2[slot * rows_per_seq + grow_row] = lse2;
+                // A sequence cut into exactly two pieces: the piece that ends this
+                // range (late) merges the next range's first piece (early, in slot
+                // 2 c_last, finished long before) itself when that piece's rows of
+                // this warp's quarter are written, and marks them merged so that
+                // the combine leaves them; otherwise it writes its partial as any
+                // cut piece.  The merge is the combine's arithmetic in the
+                // combine's order, so the output bits do not depend on who merges.
+                const int c_first = (it.seq_v + kSwitchTiles) / qv;
+                const int c_last = (it.seq_v + kSwitchTiles + it.seq_t - 1) / qv;
+                const bool two = !it.complete && c_last == c_first + 1;
+                int *qflag = a.flags + (it.seq * a.groups + group) * 4 + qd;   // early; merged at + B groups 4
+                const int nq = a.B * a.groups * 4;
+                bool merge = false;
+                if (!kFp8 && two && rng == c_first) {   // (the FP8 kernel leaves every merge to the combine)
+                    int rd = 0;
+                    if (lane == 0) rd = ld_acquire_gpu(qflag);
+                    merge = __shfl_sync(0xffffffffu, rd, 0) != 0;
+                    __threadfence();
+                }
+                if (merge) {
+                    const long long eslot = 2LL * c_last;
+                    const float l2e = row_ok ? __ldcg(a.part_lse2 + eslot * rows_per_seq + grow_row) : -INFINITY;
+                    const float mx = fmaxf(lse2, l2e);
+                    const float w0 = lse2 == -INFINITY ? 0.f : exp2f(lse2 - mx);
+                    const float w1 = l2e == -INFINITY ? 0.f : exp2f(l2e - mx);
+                    float den = 0.f;
+                    den += w0;
+                    den += w1;
+                    const float invd = den > 0.f ? 1.f / den : 0.f;
+                    // the early piece's 16 rows of this quarter, one bulk copy per
+                    // row into the stage memory (idle: this is the range's last
+                    // segment, whose pages are all consumed), rows padded to
+                    // 2,064 bytes so that the row-per-thread reads below spread
+                    // over the banks
+                    constexpr int kRowPad = kDc * 4 + 16;
+                    uint8_t *erows = stages + qd * 16 * kRowPad;
+                    const int r0 = group * kGroupRows + 16 * qd;
+                    const int nr = max(0, min(16, rows_per_seq - r0));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        sm100::mbar_arrive_expect_tx(&early_in[qd], (uint32_t)(nr * kDc * 4));
+                        for (int r = 0; r < nr; ++r)
+                            sm100::bulk_load(erows + r * kRowPad, a.part_o + (eslot * rows_per_seq + r0 + r) * kDc, kDc * 4,
+                                             &early_in[qd]);
+                    }
+                    ok = sm100::warp_wait(&early_in[qd], 0, abort_flag, a.err, lim);
+                    if (!ok) {   // let the copies land before the CTA unwinds
+                        volatile int no_abort = 0;
+                        sm100::warp_wait(&early_in[qd], 0, &no_abort, a.err, lim > 200000000ull ? lim : 200000000ull);
+                        break;
+                    }
+                    char *obase = reinterpret_cast<char *>(a.out + (long long)it.seq * rows_per_seq * kDc);
+                    for (int c = 0; c < 512; c += 64) {
+                        uint32_t ov[32];
+                        sm100::tmem_ld16x2_32(o_base + c, ov);
+                        sm100::tmem_wait_ld();
+                        float ev[32];
+                        const uint32_t esrc = sm100::smem_u32(erows + lr_me * kRowPad + (c + 32 * hh) * 4);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint4 v = ld_shared_v4(esrc + 16 * j);
+                            ev[4 * j] = __uint_as_float(v.x);
+                            ev[4 * j + 1] = __uint_as_float(v.y);
+                            ev[4 * j + 2] = __uint_as_float(v.z);
+                            ev[4 * j + 3] = __uint_as_float(v.w);
+                        }
+                        auto mv = [&](int i) {
+                            return fmaf(w1, ev[i], fmaf(w0, __uint_as_float(ov[i]) * inv, 0.f)) * invd;
+                        };
+                        uint4 pk[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            pk[j] = make_uint4(pack_bf162(mv(8 * j), mv(8 * j + 1)), pack_bf162(mv(8 * j + 2), mv(8 * j + 3)),
+                                               pack_bf162(mv(8 * j + 4), mv(8 * j + 5)), pack_bf162(mv(8 * j + 6), mv(8 * j + 7)));
+                        store_block(std::false_type{}, c, pk, obase);
+                    }
+                    if (row_ok && srow && a.out_lse) a.out_lse[orow] = den > 0.f ? (mx + log2f(den)) * kLn2 : -INFINITY;
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicExch(qflag + nq, 1);
+                } else {
+                    if (it.complete)
+                        drain(std::false_type{});
+                    else
+                        drain(std::true_type{});
+                    if (row_ok && srow) {
+                        if (it.complete) {
+                            if (a.out_lse) a.out_lse[orow] = lse2 * kLn2;
+                        } else {
+                            a.part_lse2[slot * rows_per_seq + grow_row] = lse2;
+                        }
+                    }
+                    if (!kFp8 && two && rng == c_first && lane == 0)
+                        atomicAdd(a.flags + 2 * nq, 1);   // this quarter falls back to the combine
+                    if (!kFp8 && two && rng == c_last) {
+                        // the early piece's rows of this quarter are written
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) atomicExch(qflag, 1);
                     }
                 }
                 __syncwarp();
