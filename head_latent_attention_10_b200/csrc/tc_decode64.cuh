@@ -39,7 +39,9 @@
 // page).  P of a tile (64 x 64 bf16, 128-byte swizzle, 8 KB) is written over
 // the tile's RoPE chunk, which no MMA reads once the tile's logits are done,
 // so P has one buffer per stage and is freed with the stage.  Tiles three
-// ahead are prefetched into L2, so a freed stage refills from L2.
+// ahead are prefetched into L2, so a freed stage refills from L2; when that
+// tile starts a segment, the loader also bulk-prefetches the segment's Q
+// rows, which the softmax warps read at the switch.
 //
 // Softmax: warps 4-7, one per TMEM quarter.  Threads i and 16+i of a warp
 // share row 16q+i: each reads half of the row's 64 logits, frees the buffer
@@ -52,11 +54,15 @@
 // Work split: the (sequence, tile) list of the batch is cut into contiguous
 // ranges of equal cost per row group, a tile counting one and the start of a
 // sequence four (plan_range, one warp of every CTA).  A sequence a range
-// covers completely is normalized and written straight to the output.  A sequence cut
-// by range ends leaves one fp32 partial per piece (normalized, with its
-// log2-sum-exp), merged by dec_combine_kernel.  Every wait is bounded; a wait
-// that gives up sets MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own
-// copies in flight and frees its TMEM.
+// covers completely is normalized and written straight to the output.  A
+// sequence cut by range ends leaves one fp32 partial per piece (normalized,
+// with its log2-sum-exp), merged by dec_combine_kernel; a sequence cut into
+// exactly two pieces is merged here instead, by the CTA whose range ends
+// with its late piece (see the epilogue).  The epilogue stages each softmax
+// warp's 16 output rows through shared memory, so that they leave in whole
+// 128-byte lines.  Every wait is bounded; a wait that gives up sets
+// MLA_DEVERR_TIMEOUT, the CTA unwinds, waits for its own copies in flight and
+// frees its TMEM.
 //
 // FP8 cache (kFp8): a page is 576 E4M3 codes per token plus two fp32 scales
 // per token (csrc/fp8.cuh).  TMA lands the codes, one 64-column box per
