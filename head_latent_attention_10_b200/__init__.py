@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libmla_b200.so")
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_WORKSPACE, MLA_ERR_DEVICE = range(6)
 MLA_DEVERR_BLOCK_ID, MLA_DEVERR_SEQ_LEN, MLA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
-MLA_SYNC_CHECK, MLA_FORCE_SIMPLE, MLA_DEBUG_STALL = 0x1, 0x2, 0x100
+MLA_SYNC_CHECK, MLA_FORCE_SIMPLE, MLA_DEBUG_STALL, MLA_DEBUG_COMBINE_ALL = 0x1, 0x2, 0x100, 0x200
 
 EXPORTED = ("mla_status_string", "mla_append_cache", "mla_append_latent", "mla_absorb_q",
             "mla_decode_workspace_size", "mla_decode", "mla_decode_error", "mla_up_v",

@@ -29,6 +29,7 @@ struct DecArgs {
     uint32_t *err;
     unsigned long long limit_ns;
     int stall_tile;       // test hook: the page load of this tile of every range is never issued (-1: none)
+    int merges;           // merge two-piece sequences in the decode kernel (0: the combine merges all)
     const float *scales;  // FP8 cache only: [num_blocks][64][2] fp32 per-part scales
     float scale_log2;
     int max_blocks, num_blocks, s, H, B, groups;
@@ -193,8 +194,8 @@ __host__ __device__ inline int plan_ints(int B) { return plan_list_off(B) + 4 * 
 // `work` (with `publish`): raised by the number of listed sequences the
 // decode kernel does not merge itself (empty ones, those cut into three or
 // more pieces, and with !merge_two the two-piece ones too).
-__device__ void plan_range(const int32_t *__restrict__ seq_lens, int B, int s, int max_blocks, int ranges, int rng,
-                           bool publish, bool merge_two, int32_t *plan, int *work, uint32_t *err, int *out)
+__device__ void plan_range(const int32_t *seq_lens, int B, int s, int max_blocks, int ranges, int rng, bool publish,
+                           bool merge_two, int32_t *plan, int *work, uint32_t *err, int *out)
 {
     const int lane = threadIdx.x & 31;
     const int max_tok = max_blocks * kBlock;
@@ -318,9 +319,9 @@ __host__ __device__ inline int combine_blocks(int B, int s, int H)
 
 
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm)
-dec_combine_kernel(const int32_t *__restrict__ plan, const int *__restrict__ flags, const float *__restrict__ part_o,
-                   const float *__restrict__ part_lse2, int B, int s, int H, bf16 *__restrict__ out,
-                   float *__restrict__ out_lse, uint32_t *err, unsigned long long limit_ns)
+dec_combine_kernel(const int32_t *plan, const int *flags, const float *part_o, const float *part_lse2, int B, int s,
+                   int H, bf16 *__restrict__ out, float *__restrict__ out_lse, uint32_t *err,
+                   unsigned long long limit_ns)
 {
     extern __shared__ __align__(128) uint8_t cb_smem[];
     const float4 *buf = reinterpret_cast<const float4 *>(cb_smem);
@@ -330,19 +331,24 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const int *__restrict__ fla
         sm100::fence_mbar_init();
     }
     __syncthreads();
-    sm100::pdl_wait();      // the decode kernel's partials, outputs, plan and flags are complete
+    // The decode kernel's partials, plan and flags are complete from here on.
+    // This kernel starts while the decode kernel still runs, so what that
+    // kernel writes is read only after the wait and only through L2 (__ldcg,
+    // bulk copies), never through the read-only path, and the pointers carry
+    // no __restrict__: either would let a load be served early or stale.
+    sm100::pdl_wait();
     const int groups = (s * H + kGroupRows - 1) / kGroupRows;
-    if (flags[2 * B * groups * 4] == 0) return;   // the decode kernel merged every cut sequence
+    if (__ldcg(flags + 2 * B * groups * 4) == 0) return;   // the decode kernel merged every cut sequence
     const int rows = s * H, nbr = (rows + kCombineWarps - 1) / kCombineWarps;
-    const int qv = plan[0], pw = plan[3];
-    const int nblk = plan[5 + B] * nbr;
+    const int qv = __ldcg(plan), pw = __ldcg(plan + 3);
+    const int nblk = __ldcg(plan + 5 + B) * nbr;
     const int4 *list = reinterpret_cast<const int4 *>(plan + plan_list_off(B));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int no_abort = 0;
     uint32_t phase = 0;
     for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
         const int li = blk / nbr, rb = blk - li * nbr;
-        const int4 seq = list[li];
+        const int4 seq = __ldcg(list + li);
         const int b = seq.x, va = seq.y, tb = seq.z, L = seq.w;
         // the ranges holding the sequence's first and last tiles; the piece in
         // range c0 is that range's first segment only if the range starts with
@@ -354,7 +360,7 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const int *__restrict__ fla
         const int rr0 = rb * kCombineWarps, nr = min(kCombineWarps, rows - rr0);
         // a two-piece sequence whose late piece merged this block's quarter
         // itself (the decode kernel's epilogue) is already in place
-        if (split && c1 == c0 + 1 && flags[B * groups * 4 + (b * groups + rr0 / kGroupRows) * 4 + (rr0 % kGroupRows) / 16])
+        if (split && c1 == c0 + 1 && __ldcg(flags + B * groups * 4 + (b * groups + rr0 / kGroupRows) * 4 + (rr0 % kGroupRows) / 16))
             continue;
         const int rr = rr0 + warp;
         const bool row_ok = warp < nr;
@@ -371,7 +377,7 @@ dec_combine_kernel(const int32_t *__restrict__ plan, const int *__restrict__ fla
             continue;   // uniform: the whole block belongs to one sequence
         }
         const int n = c1 - c0 + 1;
-        auto lse_of = [&](int i) { return part_lse2[(long long)(i == 0 ? slot0 : 2 * (c0 + i)) * rows + rr]; };
+        auto lse_of = [&](int i) { return __ldcg(part_lse2 + (long long)(i == 0 ? slot0 : 2 * (c0 + i)) * rows + rr); };
         const bool merge = row_ok && visible;
         const float l2_lane = (merge && lane < n) ? lse_of(lane) : -INFINITY;
         float M = l2_lane;

@@ -312,6 +312,7 @@ mla_status_t run_tc_decode(const mla_dims_t *dims, const void *q_abs, const void
     da.err = err;
     da.limit_ns = (flags & MLA_DEBUG_STALL) ? kStallWaitLimitNs : kWaitLimitNs;
     da.stall_tile = (flags & MLA_DEBUG_STALL) ? 0 : -1;
+    da.merges = (flags & MLA_DEBUG_COMBINE_ALL) ? 0 : 1;
     da.scales = scales;
     da.scale_log2 = softmax_scale(dims) * kLog2e;
     da.max_blocks = max_blocks;

@@ -171,8 +171,8 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
     // the sequence lengths and queries may come from the kernel before this one
     sm100::pdl_wait();
     if (warp == 2)
-        plan_range(a.seq_lens, a.B, a.s, a.max_blocks, gridDim.x / a.groups, rng, blockIdx.x == 0, !kFp8, a.plan,
-                   a.flags + 2 * a.B * a.groups * 4, a.err, rplan);
+        plan_range(a.seq_lens, a.B, a.s, a.max_blocks, gridDim.x / a.groups, rng, blockIdx.x == 0,
+                   !kFp8 && a.merges, a.plan, a.flags + 2 * a.B * a.groups * 4, a.err, rplan);
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
@@ -430,11 +430,13 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
         auto write_q = [&](int seq) {
             const uint4 *q4 = reinterpret_cast<const uint4 *>(
                 a.q_abs + ((long long)seq * rows_per_seq + (row_ok ? grow_row : 0)) * kRow) + (srow ? 0 : 4);
-            // all 36 loads in flight at once (one memory latency per switch)
+            // all 36 loads in flight at once (one memory latency per switch),
+            // through L2: the kernel that wrote the queries may have been
+            // running when this one started, so the read-only path is out
             uint4 v[36];
 #pragma unroll
             for (int e = 0; e < 36; ++e)
-                v[e] = row_ok ? __ldg(q4 + 8 * (e >> 2) + (e & 3)) : make_uint4(0, 0, 0, 0);
+                v[e] = row_ok ? __ldcg(q4 + 8 * (e >> 2) + (e & 3)) : make_uint4(0, 0, 0, 0);
             if constexpr (kFp8) {
                 // the FP8 path's MMAs take f16 operands
 #pragma unroll
@@ -480,7 +482,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 // this warp's quarter into L2 before the merge reads them
                 const int cf = (it.seq_v + kSwitchTiles) / qv, cl = (it.seq_v + kSwitchTiles + it.seq_t - 1) / qv;
                 const int r0 = group * kGroupRows + 16 * qd;
-                if (!kFp8 && !it.complete && cl == cf + 1 && rng == cf && r0 < rows_per_seq) {
+                if (!kFp8 && a.merges && !it.complete && cl == cf + 1 && rng == cf && r0 < rows_per_seq) {
                     const char *e = reinterpret_cast<const char *>(a.part_o + (2LL * cl * rows_per_seq + r0) * kDc);
                     const int nr = min(16, rows_per_seq - r0);
                     for (int o = 0; o < nr * kDc * 4; o += 16384)
@@ -723,7 +725,7 @@ tc_decode64_kernel(const __grid_constant__ CUtensorMap map_kv, const DecArgs a)
                 // combine's order, so the output bits do not depend on who merges.
                 const int c_first = (it.seq_v + kSwitchTiles) / qv;
                 const int c_last = (it.seq_v + kSwitchTiles + it.seq_t - 1) / qv;
-                const bool two = !it.complete && c_last == c_first + 1;
+                const bool two = a.merges && !it.complete && c_last == c_first + 1;
                 int *qflag = a.flags + (it.seq * a.groups + group) * 4 + qd;   // early; merged at + B groups 4
                 const int nq = a.B * a.groups * 4;
                 bool merge = false;

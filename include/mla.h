@@ -84,6 +84,11 @@ typedef enum {
                                   up after 20 ms, so the call records
                                   MLA_DEVERR_TIMEOUT and unwinds; the output is
                                   then unspecified.  Never set in production. */
+#define MLA_DEBUG_COMBINE_ALL 0x200u /* test hook: every cut sequence is merged
+                                  by the combine kernel, none inside the
+                                  decode kernel; the results are the same bits
+                                  either way (the two merges take the same
+                                  steps in the same order). */
 
 typedef struct {
     int32_t num_heads;   /* H */
@@ -198,7 +203,8 @@ size_t mla_decode_workspace_size(const mla_dims_t *dims, int B, int s, int max_s
  *   workspace   device buffer of ws_bytes >= mla_decode_workspace_size();
  *               its first 4 bytes are the device error word (cleared by the
  *               call); the rest holds the split plan and partial results.
- *   flags       MLA_SYNC_CHECK, MLA_FORCE_SIMPLE (MLA_DEBUG_STALL: tests only).
+ *   flags       MLA_SYNC_CHECK, MLA_FORCE_SIMPLE (MLA_DEBUG_STALL,
+ *               MLA_DEBUG_COMBINE_ALL: tests only).
  * Sequences are independent; calls that share a workspace must not overlap
  * on the GPU.  B = 0 is a no-op.  With B > 0, num_blocks and max_blocks must
  * be at least 1 (MLA_ERR_INVALID_ARG otherwise).
