@@ -69,10 +69,10 @@ def algorithmic_fp8(cfg: W.MLAConfig, seq_lens: np.ndarray, max_blocks: int):
 
 # DRAM bytes (read + write) the current decode kernel moves per cache token,
 # from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
-# tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (157.8 MB read
-# + 9.1 MB written for 131,072 tokens).  Set to None whenever the decode kernel
+# tc_decode64_kernel on the V2-shaped batch cut to 32 sequences (157.7 MB read
+# + 7.5 MB written for 131,072 tokens).  Set to None whenever the decode kernel
 # changes.
-DECODE_DRAM_BYTES_PER_TOKEN = (157.766912e6 + 9.122048e6) / (32 * 4096)
+DECODE_DRAM_BYTES_PER_TOKEN = (157.684992e6 + 7.459840e6) / (32 * 4096)
 
 
 class ClockSampler:

@@ -338,17 +338,32 @@ dec_combine_kernel(const int32_t *plan, const int *flags, const float *part_o, c
     // no __restrict__: either would let a load be served early or stale.
     sm100::pdl_wait();
     const int groups = (s * H + kGroupRows - 1) / kGroupRows;
-    if (__ldcg(flags + 2 * B * groups * 4) == 0) return;   // the decode kernel merged every cut sequence
     const int rows = s * H, nbr = (rows + kCombineWarps - 1) / kCombineWarps;
-    const int qv = __ldcg(plan), pw = __ldcg(plan + 3);
-    const int nblk = __ldcg(plan + 5 + B) * nbr;
     const int4 *list = reinterpret_cast<const int4 *>(plan + plan_list_off(B));
+    // L2 round trips follow one another here, so the loads go out in as few
+    // rounds as they can: first the work count, the plan's quota and list
+    // length and this CTA's first list entry (the grid has at most B nbr
+    // CTAs, so the entry lies in the list area even past the list's end)
+    const int work = __ldcg(flags + 2 * B * groups * 4);
+    const int qv = __ldcg(plan), pw = __ldcg(plan + 3), nlist = __ldcg(plan + 5 + B);
+    int4 seq = __ldcg(list + blockIdx.x / nbr);
+    if (work == 0) return;   // the decode kernel merged every cut sequence
+    const int nblk = nlist * nbr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int no_abort = 0;
     uint32_t phase = 0;
+    auto copy_pieces = [&](int i0, int np, int slot0, int c0, int rr0, int nr) {
+        if (threadIdx.x == 0) {
+            sm100::mbar_arrive_expect_tx(bar, (uint32_t)(np * nr * kDc * 4));
+            for (int u = 0; u < np; ++u)
+                sm100::bulk_load(cb_smem + u * (kCombineWarps * kDc * 4),
+                                 part_o + ((long long)(i0 + u == 0 ? slot0 : 2 * (c0 + i0 + u)) * rows + rr0) * kDc,
+                                 (uint32_t)(nr * kDc * 4), bar);
+        }
+    };
     for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
         const int li = blk / nbr, rb = blk - li * nbr;
-        const int4 seq = __ldcg(list + li);
+        if (blk != blockIdx.x) seq = __ldcg(list + li);
         const int b = seq.x, va = seq.y, tb = seq.z, L = seq.w;
         // the ranges holding the sequence's first and last tiles; the piece in
         // range c0 is that range's first segment only if the range starts with
@@ -358,15 +373,36 @@ dec_combine_kernel(const int32_t *plan, const int *flags, const float *part_o, c
         const bool split = tb > 0 && c0 != c1;
         const int slot0 = 2 * c0 + (c0 * qv < va ? 1 : 0);
         const int rr0 = rb * kCombineWarps, nr = min(kCombineWarps, rows - rr0);
-        // a two-piece sequence whose late piece merged this block's quarter
-        // itself (the decode kernel's epilogue) is already in place
-        if (split && c1 == c0 + 1 && __ldcg(flags + B * groups * 4 + (b * groups + rr0 / kGroupRows) * 4 + (rr0 % kGroupRows) / 16))
-            continue;
         const int rr = rr0 + warp;
         const bool row_ok = warp < nr;
         const bool visible = L - s + rr / H + 1 > 0;   // query rr / H sees some key
         const long long orow = (long long)b * rows + rr;
         uint2 *dst = reinterpret_cast<uint2 *>(out + orow * kDc) + lane;   // + 32 e: columns 4 (32 e + lane) ..
+        const int n = c1 - c0 + 1;
+        auto lse_of = [&](int i) { return __ldcg(part_lse2 + (long long)(i == 0 ? slot0 : 2 * (c0 + i)) * rows + rr); };
+        const bool merge = split && row_ok && visible;
+        // the second round: the first pieces' rows, their log2-sum-exps and
+        // the merged flag together
+        if (split) {
+            __syncthreads();   // every warp is done with the previous block's rows
+            copy_pieces(0, min(kCombinePieces, n), slot0, c0, rr0, nr);
+        }
+        const float l2_lane = (merge && lane < n) ? lse_of(lane) : -INFINITY;
+        // a two-piece sequence whose late piece merged this block's quarter
+        // itself (the decode kernel's epilogue) is already in place
+        const int merged = (split && c1 == c0 + 1)
+                               ? __ldcg(flags + B * groups * 4 + (b * groups + rr0 / kGroupRows) * 4 + (rr0 % kGroupRows) / 16)
+                               : 0;
+        if (merged) {
+            // the copies land before their buffer is used again
+            const bool ok = sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns);
+            if (!__syncthreads_and(ok)) {
+                sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns > 200000000ull ? limit_ns : 200000000ull);
+                return;
+            }
+            phase ^= 1;
+            continue;
+        }
         if (!split) {
             // a sequence with no tile: every query row is zero
             if (row_ok && !visible) {
@@ -376,10 +412,6 @@ dec_combine_kernel(const int32_t *plan, const int *flags, const float *part_o, c
             }
             continue;   // uniform: the whole block belongs to one sequence
         }
-        const int n = c1 - c0 + 1;
-        auto lse_of = [&](int i) { return __ldcg(part_lse2 + (long long)(i == 0 ? slot0 : 2 * (c0 + i)) * rows + rr); };
-        const bool merge = row_ok && visible;
-        const float l2_lane = (merge && lane < n) ? lse_of(lane) : -INFINITY;
         float M = l2_lane;
         if (merge)
             for (int i = lane + 32; i < n; i += 32) M = fmaxf(M, lse_of(i));
@@ -390,13 +422,9 @@ dec_combine_kernel(const int32_t *plan, const int *flags, const float *part_o, c
         float den = 0.f;
         for (int i0 = 0; i0 < n; i0 += kCombinePieces) {
             const int np = min(kCombinePieces, n - i0);
-            __syncthreads();   // every warp is done with the previous round's rows
-            if (threadIdx.x == 0) {
-                sm100::mbar_arrive_expect_tx(bar, (uint32_t)(np * nr * kDc * 4));
-                for (int u = 0; u < np; ++u)
-                    sm100::bulk_load(cb_smem + u * (kCombineWarps * kDc * 4),
-                                     part_o + ((long long)(i0 + u == 0 ? slot0 : 2 * (c0 + i0 + u)) * rows + rr0) * kDc,
-                                     (uint32_t)(nr * kDc * 4), bar);
+            if (i0 > 0) {
+                __syncthreads();   // every warp is done with the previous round's rows
+                copy_pieces(i0, np, slot0, c0, rr0, nr);
             }
             bool ok = sm100::mbar_wait(bar, phase, &no_abort, err, limit_ns);
             if (!__syncthreads_and(ok)) {

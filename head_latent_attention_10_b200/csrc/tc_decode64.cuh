@@ -100,7 +100,7 @@ constexpr int kD64Smem = kD64OffEpi + 4 * 16 * kD64EpiRow + 1024;  // + alignmen
 constexpr uint32_t kD64TmO = 16u << 16;           // O: lanes 16-31, columns 0-511
 constexpr uint32_t kD64TmQ = 128;                 // Q: lanes 0-15, columns 128-415 (S: 0-127)
 constexpr uint32_t kD64TmS2 = 416;                // third logits buffer: lanes 0-15, columns 416-479
-constexpr int kD64Ahead = 3;                      // tiles prefetched into L2 ahead of the load
+constexpr int kD64Ahead = 1;                      // tiles prefetched into L2 ahead of the load
 // FP8 cache: 128 more threads (the converters), per-stage scale slots
 // ([64][2] fp32) and per-token factored scales s_j ([64] fp32) after the stages
 constexpr int kD64Cvt = 128;                       // converter threads (warps 8-11)
