@@ -485,7 +485,7 @@ mla_status_t mla_absorb_q(const mla_dims_t *dims, const void *q_nope, const void
         return MLA_ERR_CUDA;
     static std::atomic<bool> attr_set[kMaxDevices];
     if (ensure_smem_attr(absorb_kernel, kAbSmem, attr_set) != cudaSuccess) return MLA_ERR_CUDA;
-    absorb_kernel<<<dim3(H, (T + 127) / 128), kAbThreads, kAbSmem, s>>>(ma, mb, mo, (const bf16 *)q_rope, q_pos, T, H,
+    absorb_kernel<<<dim3(H, (T + 127) / 128, kAbParts), kAbThreads, kAbSmem, s>>>(ma, mb, mo, (const bf16 *)q_rope, q_pos, T, H,
                                                                          (bf16 *)q_abs, rope_table(dims), nullptr,
                                                                          kWaitLimitNs);
     count_launch();
