@@ -131,7 +131,11 @@ def emulate_combine(B, s, H, p, grid):
     lst = combine_list(p)
     nblk = len(lst) * nbr
     reads, writes, rows_seen, copies = [], [], set(), []
+    # every CTA reads list entry cta // nbr before it knows the list's
+    # length: the entry must lie in the list area (B entries)
+    assert grid <= B * nbr
     for cta in range(grid):
+        assert 0 <= cta // nbr < B
         for blk in range(cta, nblk, grid):
             li, rb = divmod(blk, nbr)
             b, va, t, L = lst[li]
