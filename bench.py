@@ -429,7 +429,8 @@ def per_config(M, names, iters=30, fp8=False):
     latent query N(0,1/4), a random block permutation, the workload's own
     sequence lengths); timing does not depend on their values.  Workloads
     whose cache fits in L2 are timed with a 256 MB L2 flush before each call
-    and also warm (no flush)."""
+    and also warm (no flush).  `graph_us` is the same call captured once as a
+    CUDA graph and replayed (the flush, if any, outside the timed replay)."""
     import torch
     out = {}
     pk = peaks()
@@ -497,6 +498,31 @@ def per_config(M, names, iters=30, fp8=False):
              "l2": "flushed before each call" if small else "cache larger than L2"}
         if small:
             r["warm_l2_us"] = timed(False) * 1e6
+        # the same call captured once as a CUDA graph and replayed, as a
+        # serving loop would run it: on the small batches the eager time above
+        # is mostly the host's launch cost
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            call()
+            side.synchronize()
+            with torch.cuda.graph(graph, stream=side):
+                call()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        gts = []
+        for _ in range(iters):
+            if small:
+                flush.fill_(1)
+            a, b = E(enable_timing=True), E(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            gts.append((a, b))
+        torch.cuda.synchronize()
+        r["graph_us"] = float(np.mean([x.elapsed_time(y) for x, y in gts])) * 1e3
+        del graph
         out[name] = r
         del cache, q, lat, lse, ws, bt, slt
         if fp8:
