@@ -38,10 +38,12 @@
 // tiles (73,728 B each; TMA loads one 64 x 64 box per chunk from the tile's
 // page).  P of a tile (64 x 64 bf16, 128-byte swizzle, 8 KB) is written over
 // the tile's RoPE chunk, which no MMA reads once the tile's logits are done,
-// so P has one buffer per stage and is freed with the stage.  Tiles three
-// ahead are prefetched into L2, so a freed stage refills from L2; when that
-// tile starts a segment, the loader also bulk-prefetches the segment's Q
-// rows, which the softmax warps read at the switch.
+// so P has one buffer per stage and is freed with the stage.  After each page
+// load the loader prefetches the next page it will load into L2, so a freed
+// stage refills from L2 (prefetching farther ahead competes with the other
+// SMs' loads); when that tile starts a segment, the loader also
+// bulk-prefetches the segment's Q rows, which the softmax warps read at the
+// switch.
 //
 // Softmax: warps 4-7, one per TMEM quarter.  Threads i and 16+i of a warp
 // share row 16q+i: each reads half of the row's 64 logits, frees the buffer
