@@ -77,18 +77,26 @@ def test_in_kernel_merges_equal_the_combine_bit_for_bit(case):
     np.testing.assert_allclose(lse_k.cpu().numpy()[rows], wlse, atol=1e-2, rtol=0)
 
 
-def test_repeated_calls_with_fallbacks_to_the_combine():
-    """74 sequences of 4096 tokens, 16 heads: the plan gives each sequence two
-    ranges of its own, the second (the early piece, 34 tiles) no shorter than
-    the first (the late piece, 30 tiles and the switch), so the late piece
-    often finds the early one unfinished and leaves the sequence to the
-    combine at the very end of the decode kernel.  The combine starts while
-    the decode kernel still runs (programmatic dependent launch) and must
-    see that late work: every call gives the combine-only bits, and over the
-    calls some sequences are left to the combine."""
+RACING = [
+    # 16 heads: one warp quarter of one row group holds every row
+    W.MLAConfig("h16_two_ranges", B=74, s=1, H=16, L=4096, paged=True, seed=605, d_model=2048),
+    # 128 heads: two row groups, all four quarters of each
+    W.MLAConfig("h128_two_ranges", B=37, s=1, H=128, L=4096, paged=True, seed=606, d_model=5120),
+]
+
+
+@pytest.mark.parametrize("cfg", RACING, ids=lambda c: c.name)
+def test_repeated_calls_with_fallbacks_to_the_combine(cfg):
+    """Sequences of 4096 tokens, as many as give each one two ranges of its
+    own: the second (the early piece, 34 tiles) is no shorter than the first
+    (the late piece, 30 tiles and the switch), so the late piece often finds
+    the early one unfinished and leaves the sequence to the combine at the
+    very end of the decode kernel.  The combine starts while the decode
+    kernel still runs (programmatic dependent launch) and must see that late
+    work: every call gives the combine-only bits, and over the calls some
+    sequences are left to the combine."""
     import torch
     import head_latent_attention_10_b200 as M
-    cfg = W.MLAConfig("h16_two_ranges", B=74, s=1, H=16, L=4096, paged=True, seed=605, d_model=2048)
     npc = pieces(cfg)
     assert (npc == 2).all(), np.bincount(npc)
     M.load_library()
@@ -96,7 +104,7 @@ def test_repeated_calls_with_fallbacks_to_the_combine():
     q_abs = g.absorb()
     lat_c, lse_c = g.decode(q_abs, flags=M.MLA_DEBUG_COMBINE_ALL)
     want, wlse = host_bits(lat_c), lse_c.cpu().numpy().view(np.uint32)
-    B, groups = cfg.B, 1
+    B, groups = cfg.B, (cfg.s * cfg.H + 63) // 64
     # the work count: after the plan (16-byte aligned) and two flag arrays
     plan_ints = ((B + 9) & ~3) + 4 * B
     off_flags = (256 + 4 * plan_ints + 15) // 16 * 16
